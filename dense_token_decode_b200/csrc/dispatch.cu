@@ -1,0 +1,50 @@
+// Chooses the kernel sequence for each forward call.
+#include <atomic>
+
+#include "runtime.h"
+
+namespace fs {
+
+fs_status init_extras(fs_model* m) {
+  (void)m;
+  return FS_OK;
+}
+
+void release_extras(fs_model* m) { (void)m; }
+
+fs_status ensure_gen_buffer(fs_model* m, int n) {
+  if (n <= m->gen_cap) return FS_OK;
+  if (m->gen_tok) cudaFree(m->gen_tok);
+  m->gen_tok = nullptr;
+  m->gen_cap = 0;
+  if (cudaMalloc(&m->gen_tok, (size_t)n * sizeof(int32_t)) != cudaSuccess) {
+    cudaGetLastError();
+    set_error("out of device memory for greedy ids");
+    return FS_ERR_OOM;
+  }
+  m->gen_cap = n;
+  return FS_OK;
+}
+
+fs_status prefill_chunk(fs_model* m, const fs_kv* kv, const RowMap& map, int rows,
+                        const int32_t* tok, int head_first, float* logits, int32_t* argmax,
+                        int capture_row0, int capture_rows, cudaStream_t st) {
+  return forward_general(m, kv, map, rows, tok, head_first, logits, argmax, capture_row0,
+                         capture_rows, st);
+}
+
+fs_status decode_rows(fs_model* m, const fs_kv* kv, const RowMap& map, int rows,
+                      const int32_t* tok, float* logits, int32_t* argmax, cudaStream_t st) {
+  return forward_general(m, kv, map, rows, tok, 0, logits, argmax, 0, rows, st);
+}
+
+}  // namespace fs
+
+namespace fs {
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace fs
+
+extern "C" uint64_t fs_debug_kernel_launches(void) { return fs::g_launches.load(); }

@@ -1,0 +1,125 @@
+// Internal declarations shared by the libfs CUDA sources (not part of the ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "fs.h"
+
+namespace fs {
+
+// Kernel launches issued by the library (fs_debug_kernel_launches).
+void count_launches(int n = 1);
+
+constexpr int kPage = 64;        // positions per KV page
+constexpr int kMaxBatch = 64;    // rows of one decode step
+constexpr int kMaxHeadDim = 128;
+
+// Device error word values (fs_device_error).
+constexpr int kErrToken = 1;
+constexpr int kErrBounds = 2;
+constexpr int kErrTimeout = 3;
+
+// Index of each linear layer in LayerDev::w / LayerDev::s.
+enum Lin { kWq = 0, kWk, kWv, kWo, kWg, kWu, kWd, kNumLin };
+
+struct LayerDev {
+  const void* w[kNumLin];   // bf16 [N,K] or int8 codes [N,K]
+  const __half* s[kNumLin]; // Q8_0 scales [N,K/32] (nullptr for bf16)
+  const __nv_bfloat16* attn_norm;
+  const __nv_bfloat16* ffn_norm;
+  const __nv_bfloat16* q_norm;
+  const __nv_bfloat16* k_norm;
+};
+
+// Paged KV cache as the kernels see it. K and V pools are
+// [layer][page][kv_head][slot 0..63][head_dim] bf16.
+struct KVView {
+  __nv_bfloat16* k;
+  __nv_bfloat16* v;
+  const int32_t* block_table;  // [max_seqs][pages_per_seq] physical page ids
+  int32_t pages_per_seq;
+  int32_t n_pages;
+  int32_t n_kv_heads;
+  int32_t head_dim;
+  __host__ __device__ size_t layer_elems() const {
+    return (size_t)n_pages * n_kv_heads * kPage * head_dim;
+  }
+  // Element offset of (layer, seq, pos, kv_head, 0).
+  __device__ __forceinline__ size_t offset(int layer, int seq, int pos, int g) const {
+    int page = block_table[(size_t)seq * pages_per_seq + pos / kPage];
+    return (size_t)layer * layer_elems() +
+           (((size_t)page * n_kv_heads + g) * kPage + (pos % kPage)) * head_dim;
+  }
+};
+
+// Per-row (token) description of one forward call: which sequence it belongs
+// to and at which position it sits.
+struct RowInfo {
+  int32_t seq;
+  int32_t pos;
+};
+
+// Row map of one forward call, passed to kernels by value (no staging
+// buffer): either `n_list` explicit (seq, pos) pairs (a decode batch) or, with
+// n_list == 0, consecutive positions pos0, pos0+1, ... of one sequence seq0
+// (a prefill chunk).
+struct RowMap {
+  int32_t n_list;
+  int32_t seq0;
+  int32_t pos0;
+  int32_t seq[kMaxBatch];
+  int32_t pos[kMaxBatch];
+  __host__ __device__ __forceinline__ RowInfo get(int r) const {
+    return n_list ? RowInfo{seq[r], pos[r]} : RowInfo{seq0, pos0 + r};
+  }
+};
+
+struct Shape {
+  int L, H, nq, nkv, d, I, V;
+  float eps;
+  int q_dim() const { return nq * d; }
+  int kv_dim() const { return nkv * d; }
+  int qkv_dim() const { return (nq + 2 * nkv) * d; }
+};
+
+// ---------------------------------------------------------------------------
+// Kernel launchers (each defined next to its kernel). All return
+// cudaGetLastError() after the launch.
+
+cudaError_t launch_embed(const int32_t* tokens, int rows, const __nv_bfloat16* E, int H, int V,
+                         float* h, int* err, cudaStream_t st);
+cudaError_t launch_rmsnorm(const float* x, int rows, int H, const __nv_bfloat16* g, float eps,
+                           float* out, cudaStream_t st);
+// y = x . W^T over rows; epilogue: 0 store y, 1 y += into out (residual).
+cudaError_t launch_gemv(const float* x, int rows, int K, const void* W, const __half* scales,
+                        int N, float* out, int ldo, bool accumulate, cudaStream_t st);
+// act[r, j] = silu(x . Wg[j]) * (x . Wu[j])
+cudaError_t launch_gemv_swiglu(const float* x, int rows, int K, const void* Wg, const __half* sg,
+                               const void* Wu, const __half* su, int N, float* act,
+                               cudaStream_t st);
+cudaError_t launch_gemm_simt(const float* A, int M, int K, const void* W, const __half* scales,
+                             int N, float* C, int ldc, bool accumulate, cudaStream_t st);
+cudaError_t launch_swiglu(const float* gu, int rows, int I, float* act, cudaStream_t st);
+cudaError_t launch_qk_norm_rope_append(const float* qkv, int rows, const RowMap& map,
+                                       const Shape& s, const __nv_bfloat16* q_norm,
+                                       const __nv_bfloat16* k_norm, const float2* rope,
+                                       float* q_out, KVView kv, int layer, cudaStream_t st);
+cudaError_t launch_attention_simple(const float* q, int rows, const RowMap& map,
+                                    const Shape& s, KVView kv, int layer, float* o,
+                                    cudaStream_t st);
+// x: final-normed rows fp32 [rows, H]; partial: scratch of rows * n_part float2.
+cudaError_t launch_lm_head(const float* xf, int rows, const Shape& s, const __nv_bfloat16* E,
+                           float* logits, int32_t* argmax, float2* partial, int n_part, int* err,
+                           cudaStream_t st);
+cudaError_t launch_dequant_q8_0(const int8_t* codes, const __half* scales, int n, int k,
+                                float* out, cudaStream_t st);
+cudaError_t launch_kv_copy(KVView kv, int seq, int layer, int pos0, int n, __nv_bfloat16* k,
+                           __nv_bfloat16* v, bool import, cudaStream_t st);
+
+}  // namespace fs

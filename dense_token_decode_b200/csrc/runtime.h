@@ -1,0 +1,85 @@
+// Handle structs behind the opaque fs_model / fs_kv of the C ABI, and the
+// internal entry points the fast paths plug into.
+#pragma once
+
+#include <string>
+#include <vector>
+
+#include "fs_internal.h"
+
+struct fs_model {
+  fs_config cfg{};
+  fs::Shape s{};
+  bool q8 = false;
+  int device = 0;
+  int num_sms = 0;
+  const __nv_bfloat16* embed = nullptr;       // caller-owned
+  const __nv_bfloat16* final_norm = nullptr;  // caller-owned
+  std::vector<fs::LayerDev> layers;           // caller-owned pointers
+  // Library-owned buffers.
+  float2* rope = nullptr;  // [max_pos][d/2] (cos, sin)
+  int max_rows = 0;        // rows of one forward chunk
+  float* h = nullptr;      // residual stream [max_rows, H]
+  float* xn = nullptr;     // normalised rows [max_rows, max(H, nq*d, I)]
+  float* qkv = nullptr;    // [max_rows, (nq+2nkv)*d]
+  float* q = nullptr;      // rotated queries [max_rows, nq*d]
+  float* o = nullptr;      // attention output [max_rows, nq*d]
+  float* gu = nullptr;     // gate||up [max_rows, 2I]
+  float* act = nullptr;    // SwiGLU output [max_rows, I]
+  float* xf = nullptr;     // final-normed rows [64, H]
+  int32_t* tok = nullptr;  // staged token ids [max_rows]
+  float2* partial = nullptr;  // LM-head argmax partials [64, n_part]
+  int n_part = 0;
+  int* err = nullptr;         // device error word
+  int32_t* gen_tok = nullptr; // greedy ids
+  int gen_cap = 0;
+  void* scratch = nullptr;
+  float* capture = nullptr;   // armed fs_debug_capture buffer
+  int capture_max_rows = 0;
+  int prefill_split = 1;
+  void* extras = nullptr;     // fast-path state
+};
+
+struct fs_kv {
+  const fs_model* model = nullptr;
+  int max_seqs = 0;
+  int max_tokens = 0;
+  int pages_per_seq = 0;
+  int n_pages = 0;
+  __nv_bfloat16* k = nullptr;
+  __nv_bfloat16* v = nullptr;
+  int32_t* block_table = nullptr;
+  std::vector<int32_t> len;  // host-tracked lengths
+};
+
+namespace fs {
+
+KVView kv_view(const fs_kv* kv);
+int kv_capacity(const fs_kv* kv);
+const char* set_error(const std::string& msg);
+void model_free_buffers(fs_model* m);
+
+fs_status init_extras(fs_model* m);
+void release_extras(fs_model* m);
+fs_status ensure_gen_buffer(fs_model* m, int n);
+
+// The unfused general forward (any rows): see runtime.cu.
+fs_status forward_general(fs_model* m, const fs_kv* kv, const RowMap& map, int rows,
+                          const int32_t* tok, int head_first, float* logits, int32_t* argmax,
+                          int capture_row0, int capture_rows, cudaStream_t st);
+
+// One prefill chunk (consecutive positions of one sequence).
+fs_status prefill_chunk(fs_model* m, const fs_kv* kv, const RowMap& map, int rows,
+                        const int32_t* tok, int head_first, float* logits, int32_t* argmax,
+                        int capture_row0, int capture_rows, cudaStream_t st);
+
+// One decode step over a batch of sequences.
+fs_status decode_rows(fs_model* m, const fs_kv* kv, const RowMap& map, int rows,
+                      const int32_t* tok, float* logits, int32_t* argmax, cudaStream_t st);
+
+fs_status prefill_impl(fs_model* m, fs_kv* kv, int32_t seq, const int32_t* tokens, int32_t n,
+                       float* logits, int32_t* argmax, cudaStream_t st);
+fs_status decode_impl(fs_model* m, fs_kv* kv, const int32_t* seqs, const int32_t* tokens,
+                      int32_t batch, float* logits, int32_t* argmax, cudaStream_t st);
+
+}  // namespace fs

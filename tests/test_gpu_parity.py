@@ -1,0 +1,405 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the fp64
+oracle on the same seeded inputs.
+
+Bars (written in parity_util): per-block hidden-state relative L2 <= 1e-3,
+max |delta logit| <= 2e-2, greedy ids identical for 32 steps (a step whose
+oracle top-2 gap is below twice the measured logit error is "ambiguous": it
+passes if the GPU picked either candidate, and both sides continue on the
+oracle's id), Q8_0 dequantisation bit-exact.
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from conftest import oracle_weights
+from dense_token_decode_b200 import abi, synth
+from dense_token_decode_b200.engine import Model
+from parity_util import (BLOCK_REL_L2, GREEDY_STEPS, LOGIT_ABS, assert_blocks_close,
+                         assert_logits_close, check_greedy_step, oracle_tensor, rel_l2)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+QWEN_SEED = 1     # decode / prefill / batched-decode configs share these bf16 weights
+Q8_SEED = 4
+
+
+# --------------------------------------------------------------------------- fixtures
+
+class Pair:
+    """A GPU model and the oracle over the same weights."""
+
+    def __init__(self, shape, seed, fmt="bf16", max_pos=None):
+        self.shape = shape
+        w = synth.model_weights(shape, seed, fmt)
+        self.model = Model(shape, w, DEV, max_pos=max_pos)
+        self._w = w
+        self._oracle = None
+
+    @property
+    def oracle(self):
+        if self._oracle is None:
+            self._oracle = oracle.Qwen3Oracle(self.shape, oracle_weights(self._w))
+        return self._oracle
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return Pair(synth.TINY, 0)
+
+
+@pytest.fixture(scope="module")
+def qwen():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return Pair(synth.QWEN3_0P6B, QWEN_SEED, max_pos=8192 + 256)
+
+
+def _dev_i32(xs):
+    return torch.tensor(list(xs), dtype=torch.int32, device=DEV)
+
+
+def prefill_with_capture(pair, kv, seq, toks):
+    m, s = pair.model, pair.shape
+    n = len(toks)
+    hidden = torch.zeros((s.n_layers + 1, n, s.hidden), dtype=torch.float32, device=DEV)
+    logits = torch.empty(s.vocab, dtype=torch.float32, device=DEV)
+    am = torch.empty(1, dtype=torch.int32, device=DEV)
+    m.capture(hidden, n)
+    m.prefill(kv, seq, _dev_i32(toks), logits, am)
+    torch.cuda.synchronize()
+    return oracle_tensor(logits), oracle_tensor(hidden), int(am.item())
+
+
+def decode_teacher_forced(pair, kv, seq, first_tok, ref_ids, ref_logits, capture_steps=()):
+    """GPU decode fed the oracle's ids; checks every step. Returns ambiguous count."""
+    m, s = pair.model, pair.shape
+    logits = torch.empty(s.vocab, dtype=torch.float32, device=DEV)
+    am = torch.empty(1, dtype=torch.int32, device=DEV)
+    ambiguous = 0
+    inputs = [first_tok] + list(ref_ids[:-1])
+    hiddens = {}
+    for i, tok in enumerate(inputs):
+        hid = None
+        if i in capture_steps:
+            hid = torch.zeros((s.n_layers + 1, 1, s.hidden), dtype=torch.float32, device=DEV)
+            m.capture(hid, 1)
+        m.decode_step(kv, [seq], _dev_i32([tok]), logits, am)
+        torch.cuda.synchronize()
+        gl = oracle_tensor(logits)
+        assert_logits_close(gl, ref_logits[i], what=f"decode step {i}")
+        if not check_greedy_step(int(am.item()), gl, ref_logits[i]):
+            ambiguous += 1
+        if hid is not None:
+            hiddens[i] = oracle_tensor(hid)
+    return ambiguous, hiddens
+
+
+# --------------------------------------------------------------------------- tiny config
+
+def test_tiny_prefill_logits_blocks_and_cache(tiny):
+    toks = synth.token_ids(16, tiny.shape.vocab, seed=0).tolist()
+    kv = tiny.model.kv(2, 64)
+    gl, gh, am = prefill_with_capture(tiny, kv, 0, toks)
+    rl, rh, cache = tiny.oracle.forward(toks)
+    assert_blocks_close(gh, rh, what="tiny prefill")
+    assert_logits_close(gl, rl, what="tiny prefill")
+    assert am == oracle.greedy_select(rl) or abs(rl[am] - rl.max()) < 2 * np.abs(gl - rl).max()
+    for l in range(tiny.shape.n_layers):
+        k, v = kv.export(0, l, 0, 16)
+        assert rel_l2(oracle_tensor(k), cache.k[l]) <= BLOCK_REL_L2
+        assert rel_l2(oracle_tensor(v), cache.v[l]) <= BLOCK_REL_L2
+    assert kv.length(0) == 16
+
+
+def test_tiny_decode_teacher_forced(tiny):
+    toks = synth.token_ids(16, tiny.shape.vocab, seed=0).tolist()
+    ids, why, ref_logits = oracle.generate_greedy(tiny.oracle, toks, 17)
+    kv = tiny.model.kv(1, 64)
+    gl, _, am = prefill_with_capture(tiny, kv, 0, toks)
+    check_greedy_step(am, gl, ref_logits[0])
+    amb, hid = decode_teacher_forced(tiny, kv, 0, ids[0], ids[1:], ref_logits[1:],
+                                     capture_steps=(0, 15))
+    # per-block hidden states at two decode steps, against a cached oracle run
+    cache = tiny.oracle.forward(toks)[2]
+    prefix_ids = [ids[0]] + ids[1:16]
+    for i, tok in enumerate(prefix_ids):
+        _, rh, cache = tiny.oracle.forward([tok], cache)
+        if i in hid:
+            assert_blocks_close(hid[i], rh, what=f"tiny decode step {i}")
+    assert amb <= 4
+
+
+def test_tiny_fs_greedy_matches_oracle(tiny):
+    toks = synth.token_ids(16, tiny.shape.vocab, seed=0).tolist()
+    ref, why, ref_logits = oracle.generate_greedy(tiny.oracle, toks, 16)
+    kv = tiny.model.kv(1, 64)
+    ids, reason = tiny.model.greedy(kv, 0, toks, 16)
+    assert reason == abi.FS_STOP_BUDGET and len(ids) == 16
+    for i, (a, b) in enumerate(zip(ids, ref)):
+        if a != b:  # allowed only at an ambiguous step; then the runs diverge
+            gap = np.sort(ref_logits[i])[-1] - np.sort(ref_logits[i])[-2]
+            assert gap < 2 * LOGIT_ABS, f"step {i}: {a} != {b} with gap {gap}"
+            break
+    assert kv.length(0) == 16 + 15
+
+
+def test_tiny_stop_rules(tiny):
+    m = tiny.model
+    prompt = synth.token_ids(5, tiny.shape.vocab, seed=4).tolist()
+    kv = m.kv(1, 64)
+    assert m.greedy(kv, 0, prompt, 0) == ([], abi.FS_STOP_BUDGET)
+    assert kv.length(0) == 0
+    first, _ = m.greedy(kv, 0, prompt, 1)
+    kv.reset(0)
+    ids, why = m.greedy(kv, 0, prompt, 5, eos=[first[0]])
+    assert ids == first and why == abi.FS_STOP_EOS
+    assert kv.length(0) == 5
+    # capacity 7: forwards at prefix lengths 5, 6, 7 -> 3 ids, then the context stop
+    for max_new, want_n, want_why in ((4, 3, abi.FS_STOP_CONTEXT), (3, 3, abi.FS_STOP_BUDGET)):
+        kv7 = m.kv(1, 7)
+        ids, why = m.greedy(kv7, 0, prompt, max_new)
+        ref, rwhy, _ = oracle.generate_greedy(tiny.oracle, prompt, max_new, max_context=7)
+        assert (len(ids), why) == (want_n, want_why)
+        assert rwhy == {abi.FS_STOP_CONTEXT: oracle.STOP_CONTEXT,
+                        abi.FS_STOP_BUDGET: oracle.STOP_BUDGET}[want_why]
+        assert kv7.length(0) == 7
+    kv4 = m.kv(1, 4)
+    with pytest.raises(abi.FsError) as e:
+        m.greedy(kv4, 0, prompt, 3)
+    assert e.value.status == abi.FS_ERR_CONTEXT
+    with pytest.raises(abi.FsError) as e:
+        m.greedy(kv, 0, [], 3)
+    assert e.value.status == abi.FS_ERR_EMPTY
+
+
+def test_tiny_chunked_prefill_and_page_crossing(tiny):
+    toks = synth.token_ids(150, tiny.shape.vocab, seed=11).tolist()
+    rl, rh, cache = tiny.oracle.forward(toks)
+    kv = tiny.model.kv(3, 256)
+    s = tiny.shape
+    logits = torch.empty(s.vocab, device=DEV)
+    # one call, and three calls ending on / across page boundaries (64, 128)
+    tiny.model.prefill(kv, 0, _dev_i32(toks), logits)
+    torch.cuda.synchronize()
+    assert_logits_close(oracle_tensor(logits), rl, what="one-shot 150")
+    for cut in ((64, 100), (63, 129)):
+        kv.reset(1)
+        a, b = cut
+        tiny.model.prefill(kv, 1, torch.tensor(toks[:a], dtype=torch.int32), None)  # host ids
+        tiny.model.prefill(kv, 1, _dev_i32(toks[a:b]), None)
+        tiny.model.prefill(kv, 1, _dev_i32(toks[b:]), logits)
+        torch.cuda.synchronize()
+        assert_logits_close(oracle_tensor(logits), rl, what=f"chunks {cut}")
+        for l in range(s.n_layers):
+            k, v = kv.export(1, l, 0, 150)
+            assert rel_l2(oracle_tensor(k), cache.k[l]) <= BLOCK_REL_L2
+            assert rel_l2(oracle_tensor(v), cache.v[l]) <= BLOCK_REL_L2
+
+
+def test_tiny_single_token_prefill_returns_v_path(tiny):
+    kv = tiny.model.kv(1, 8)
+    gl, gh, _ = prefill_with_capture(tiny, kv, 0, [7])
+    rl, rh, _ = tiny.oracle.forward([7])
+    assert_blocks_close(gh, rh, what="S=1")
+    assert_logits_close(gl, rl, what="S=1")
+
+
+def test_tiny_batched_decode_mixed_positions(tiny):
+    s = tiny.shape
+    lens = [5, 64, 63, 1]
+    prompts = [synth.token_ids(n, s.vocab, seed=20 + i).tolist() for i, n in enumerate(lens)]
+    kv = tiny.model.kv(4, 128)
+    caches = []
+    for i, p in enumerate(prompts):
+        tiny.model.prefill(kv, i, _dev_i32(p))
+        caches.append(tiny.oracle.forward(p)[2])
+    nxt = [3, 4000, 17, 99]
+    order = [2, 0, 3, 1]  # batch rows in a different order than sequence ids
+    logits = torch.empty((4, s.vocab), device=DEV)
+    am = torch.empty(4, dtype=torch.int32, device=DEV)
+    tiny.model.decode_step(kv, order, _dev_i32([nxt[q] for q in order]), logits, am)
+    torch.cuda.synchronize()
+    for b, q in enumerate(order):
+        rl = tiny.oracle.forward([nxt[q]], caches[q])[0]
+        assert_logits_close(oracle_tensor(logits[b]), rl, what=f"batch row {b}")
+        check_greedy_step(int(am[b]), oracle_tensor(logits[b]), rl)
+        assert kv.length(q) == lens[q] + 1
+
+
+def test_tiny_errors_are_reported_not_faulted(tiny):
+    m, s = tiny.model, tiny.shape
+    kv = m.kv(2, 16)
+    with pytest.raises(abi.FsError) as e:
+        m.prefill(kv, 0, torch.tensor([1, s.vocab], dtype=torch.int32))  # host id out of range
+    assert e.value.status == abi.FS_ERR_TOKEN
+    with pytest.raises(abi.FsError) as e:
+        m.prefill(kv, 0, torch.tensor([], dtype=torch.int32))
+    assert e.value.status == abi.FS_ERR_EMPTY
+    with pytest.raises(abi.FsError) as e:
+        m.prefill(kv, 0, torch.zeros(17, dtype=torch.int32))
+    assert e.value.status == abi.FS_ERR_CONTEXT
+    with pytest.raises(abi.FsError) as e:
+        m.prefill(kv, 5, torch.zeros(2, dtype=torch.int32))
+    assert e.value.status == abi.FS_ERR_SEQ
+    with pytest.raises(abi.FsError) as e:
+        m.decode_step(kv, [1, 1], torch.zeros(2, dtype=torch.int32))
+    assert e.value.status == abi.FS_ERR_SEQ
+    bad = torch.empty(s.vocab + 4, device=DEV)[1:]
+    with pytest.raises(abi.FsError) as e:
+        m.prefill(kv, 0, torch.zeros(2, dtype=torch.int32), bad)
+    assert e.value.status == abi.FS_ERR_ALIGN
+    assert kv.length(0) == 0
+    # a device id out of range is replaced by 0 and flagged in the device error word
+    assert m.device_error() == 0
+    m.prefill(kv, 0, _dev_i32([3, s.vocab + 5]))
+    torch.cuda.synchronize()
+    assert m.device_error() == 1
+    assert m.device_error() == 0
+
+
+def test_q8_0_dequant_bit_exact():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    abi.load()
+    codes, scales = synth.q8_0_blocks(96, 1024, seed=77)
+    codes[0, :3] = torch.tensor([-127, 127, 0], dtype=torch.int8)
+    out = torch.empty((96, 1024), dtype=torch.float32, device=DEV)
+    c, sc = codes.to(DEV), scales.to(DEV)
+    abi.check(abi.fs_debug_dequant_q8_0(c.data_ptr(), sc.data_ptr(), 96, 1024, out.data_ptr(),
+                                        torch.cuda.current_stream().cuda_stream), "dequant")
+    torch.cuda.synchronize()
+    want = oracle.q8_0_dequant(codes.numpy(), scales.numpy()).astype(np.float32)
+    np.testing.assert_array_equal(out.cpu().numpy().view(np.uint32), want.view(np.uint32))
+
+
+def test_lm_head_exact_tie_goes_to_lowest_id():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    s = synth.TINY
+    w = synth.model_weights(s, 0)
+    E = w["embed"].clone()
+    E[3001] = E[57]     # equal rows -> exactly equal logits
+    E[4095] = E[57]
+    w["embed"] = E
+    m = Model(s, w, DEV)
+    x = E[[57, 3001, 100]].float().to(DEV) * 7.0
+    x[2] = x[0]
+    logits = torch.empty((3, s.vocab), device=DEV)
+    am = torch.empty(3, dtype=torch.int32, device=DEV)
+    m.lm_head(x.contiguous(), logits, am)
+    torch.cuda.synchronize()
+    assert am.tolist() == [57, 57, 57]
+    assert logits[0, 57].item() == logits[0, 3001].item() == logits[0, 4095].item()
+    m.close()
+
+
+# --------------------------------------------------------------------------- Qwen3-0.6B shape
+
+def test_qwen_decode_bs1_parity(qwen):
+    """8-token prompt, 32 greedy decode steps at batch 1 (teacher-forced)."""
+    toks = synth.token_ids(8, qwen.shape.vocab, seed=1).tolist()
+    ids, _, ref_logits = oracle.generate_greedy(qwen.oracle, toks, GREEDY_STEPS + 1)
+    kv = qwen.model.kv(1, 512)
+    gl, gh, am = prefill_with_capture(qwen, kv, 0, toks)
+    _, rh, _ = qwen.oracle.forward(toks)
+    assert_blocks_close(gh, rh, what="qwen prefill 8")
+    assert_logits_close(gl, ref_logits[0])
+    check_greedy_step(am, gl, ref_logits[0])
+    amb, hid = decode_teacher_forced(qwen, kv, 0, ids[0], ids[1:], ref_logits[1:],
+                                     capture_steps=(0, 31))
+    cache = qwen.oracle.forward(toks)[2]
+    for i, tok in enumerate([ids[0]] + ids[1:32]):
+        _, rh, cache = qwen.oracle.forward([tok], cache)
+        if i in hid:
+            assert_blocks_close(hid[i], rh, what=f"qwen decode step {i}")
+    assert amb <= 8
+
+
+def test_qwen_fs_greedy_free_running(qwen):
+    toks = synth.token_ids(8, qwen.shape.vocab, seed=1).tolist()
+    ref, _, ref_logits = oracle.generate_greedy(qwen.oracle, toks, GREEDY_STEPS)
+    kv = qwen.model.kv(1, 512)
+    ids, why = qwen.model.greedy(kv, 0, toks, GREEDY_STEPS)
+    assert why == abi.FS_STOP_BUDGET
+    for i, (a, b) in enumerate(zip(ids, ref)):
+        if a != b:
+            gap = np.sort(ref_logits[i])[-1] - np.sort(ref_logits[i])[-2]
+            assert gap < 2 * LOGIT_ABS, f"step {i}: {a} != {b} with gap {gap}"
+            break
+
+
+def test_qwen_q8_0_decode_parity():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    pair = Pair(synth.QWEN3_0P6B, Q8_SEED, "q8_0", max_pos=1024)
+    toks = synth.token_ids(8, pair.shape.vocab, seed=4).tolist()
+    ids, _, ref_logits = oracle.generate_greedy(pair.oracle, toks, GREEDY_STEPS + 1)
+    kv = pair.model.kv(1, 512)
+    gl, gh, am = prefill_with_capture(pair, kv, 0, toks)
+    _, rh, _ = pair.oracle.forward(toks)
+    assert_blocks_close(gh, rh, what="q8_0 prefill 8")
+    check_greedy_step(am, gl, ref_logits[0])
+    amb, _ = decode_teacher_forced(pair, kv, 0, ids[0], ids[1:], ref_logits[1:])
+    assert amb <= 8
+    pair.model.close()
+
+
+def test_qwen_prefill_2048(qwen):
+    """2048-token prefill: last-row logits, every block's hidden state and the
+    filled KV cache against the oracle."""
+    S = 2048
+    toks = synth.token_ids(S, qwen.shape.vocab, seed=2).tolist()
+    kv = qwen.model.kv(1, S)
+    gl, gh, am = prefill_with_capture(qwen, kv, 0, toks)
+    rl, rh, cache = qwen.oracle.forward(toks)
+    assert_blocks_close(gh, rh, what="prefill 2048")
+    assert_logits_close(gl, rl, what="prefill 2048")
+    check_greedy_step(am, gl, rl)
+    for l in range(qwen.shape.n_layers):
+        k, v = kv.export(0, l, 0, S)
+        assert rel_l2(oracle_tensor(k), cache.k[l]) <= BLOCK_REL_L2, l
+        assert rel_l2(oracle_tensor(v), cache.v[l]) <= BLOCK_REL_L2, l
+
+
+def test_qwen_batched_decode_long_context(qwen):
+    """Batch 16, 8192 pre-filled N(0,1) bf16 K/V per sequence, greedy steps;
+    sequences 0 and 15 checked against the oracle at every step."""
+    s, B, CTX, STEPS = qwen.shape, 16, 8192, 4
+    kv = qwen.model.kv(B, CTX + 64)
+    host_kv = {}
+    for q in range(B):
+        for l in range(s.n_layers):
+            k, v = synth.prefilled_kv(s, CTX, seed=3, seq=q, layer=l, device=DEV)
+            kv.import_(q, l, 0, k, v)
+            if q in (0, B - 1):
+                host_kv[(q, l)] = (oracle_tensor(k), oracle_tensor(v))
+        kv.set_length(q, CTX)
+    first = synth.token_ids(B, s.vocab, seed=3).tolist()
+    caches = {q: oracle.KVCache(k=[host_kv[(q, l)][0] for l in range(s.n_layers)],
+                                v=[host_kv[(q, l)][1] for l in range(s.n_layers)])
+              for q in (0, B - 1)}
+    del host_kv
+    tok = list(first)
+    logits = torch.empty((B, s.vocab), device=DEV)
+    am = torch.empty(B, dtype=torch.int32, device=DEV)
+    for step in range(STEPS):
+        qwen.model.decode_step(kv, list(range(B)), _dev_i32(tok), logits, am)
+        torch.cuda.synchronize()
+        gpu_am = am.tolist()
+        for q in (0, B - 1):
+            rl, _, caches[q] = qwen.oracle.forward([tok[q]], caches[q])
+            assert_logits_close(oracle_tensor(logits[q]), rl, what=f"seq {q} step {step}")
+            check_greedy_step(gpu_am[q], oracle_tensor(logits[q]), rl)
+            gpu_am[q] = oracle.greedy_select(rl)   # both continue on the oracle's id
+        tok = gpu_am
+    for q in range(B):
+        assert kv.length(q) == CTX + STEPS
