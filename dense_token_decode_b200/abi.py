@@ -83,6 +83,7 @@ SIGNATURES = {
     "fs_debug_lm_head": (_I, [_P, _P, _I, _P, _P, _P]),
     "fs_device_error": (_I, [_P, _PI]),
     "fs_set_prefill_split": (_I, [_P, _I]),
+    "fs_lm_head_argmax_noalloc": (_I, [_P, _P, _I, _I, C.c_float, _P, _I, _P, _P, _P]),
     "fs_debug_kernel_launches": (C.c_uint64, []),
     "fs_last_error_string": (C.c_char_p, []),
     "fs_status_string": (C.c_char_p, [_I]),
@@ -151,6 +152,7 @@ fs_debug_dequant_q8_0 = _wrap("fs_debug_dequant_q8_0")
 fs_debug_lm_head = _wrap("fs_debug_lm_head")
 fs_device_error = _wrap("fs_device_error")
 fs_set_prefill_split = _wrap("fs_set_prefill_split")
+fs_lm_head_argmax_noalloc = _wrap("fs_lm_head_argmax_noalloc")
 fs_debug_kernel_launches = _wrap("fs_debug_kernel_launches")
 fs_last_error_string = _wrap("fs_last_error_string")
 fs_status_string = _wrap("fs_status_string")

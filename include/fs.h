@@ -234,6 +234,36 @@ fs_status fs_device_error(fs_model* model, int32_t* code);
  * Default: 1. */
 fs_status fs_set_prefill_split(fs_model* model, int32_t split);
 
+/* The final RMSNorm + tied LM head + greedy selection of fs_debug_lm_head,
+ * for callers that may not allocate device memory. The paper has no
+ * counterpart: this is a deployment convenience, not a step of the method.
+ *
+ * Who it is for: callers that cannot call cudaMalloc — a host thread with a
+ * latency budget (cudaMalloc can block on device-wide synchronisation and
+ * driver locks), a process whose device memory is all reserved by another
+ * framework's pool, or an embedding that lends us its buffers and forbids us
+ * to own any. It needs no fs_model: pass the bf16 embedding [vocab, hidden]
+ * (the tied LM head), the bf16 final-norm gains [hidden], and x, fp32
+ * [rows, hidden] device rows. Outputs (device; either may be NULL, not both):
+ * logits fp32 [rows, vocab], argmax int32 [rows] (lowest id on exact ties;
+ * 0 if a row has no finite logit). Nothing is allocated: the normalised rows
+ * and the per-block argmax partials live in one fixed 512 KiB array compiled
+ * into the library, which every GPU that loads libfs holds until the process
+ * exits. A call needs rows*hidden*4 (rounded up to 256) + rows*4*SMs*8 bytes
+ * of it (148 SMs: 16 rows of hidden 1024 fit, 64 rows do not); larger calls
+ * are rejected with FS_ERR_INVALID before anything runs.
+ * The first call on a device looks up the array's device address (a one-time
+ * set-up per device, done with that device current); make that first call
+ * before any stream capture. All calls share the one array: two calls whose
+ * work overlaps on the GPU (different streams, or different host threads on
+ * one device) race on it and may return wrong results; serialise them.
+ * Requirements: hidden % 64 == 0, 1 <= rows <= 64, rms_eps > 0, pointers
+ * 16-byte aligned (argmax 4-byte). Errors: FS_ERR_NULL, FS_ERR_INVALID,
+ * FS_ERR_ALIGN, FS_ERR_CUDA. */
+fs_status fs_lm_head_argmax_noalloc(const void* embed, const void* final_norm, int32_t hidden,
+                                    int32_t vocab, float rms_eps, const float* x, int32_t rows,
+                                    float* logits, int32_t* argmax, void* stream);
+
 /* Number of kernels libfs has launched in this process so far (all models,
  * all threads). For accounting in benchmarks; never reset. */
 uint64_t fs_debug_kernel_launches(void);
