@@ -530,8 +530,8 @@ extern "C" fs_status fs_greedy(fs_model* m, fs_kv* kv, int32_t seq, const int32_
                                int32_t* stop_reason, void* stream) {
   if (!m || !kv || !n_out || !stop_reason) return fail(FS_ERR_NULL, "NULL argument");
   if (kv->model != m) return fail(FS_ERR_INVALID, "kv belongs to another model");
-  if (!prompt) return fail(FS_ERR_NULL, "prompt is NULL");
   if (n_prompt <= 0) return fail(FS_ERR_EMPTY, "empty prompt");
+  if (!prompt) return fail(FS_ERR_NULL, "prompt is NULL");
   if (max_new < 0) return fail(FS_ERR_INVALID, "max_new < 0");
   if (n_eos < 0 || (n_eos > 0 && !eos)) return fail(FS_ERR_INVALID, "bad EOS list");
   if (seq < 0 || seq >= kv->max_seqs) return fail(FS_ERR_SEQ, "sequence out of range");
