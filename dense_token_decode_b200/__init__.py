@@ -8,6 +8,7 @@ handles that take torch tensors; ``synth`` draws the seeded synthetic inputs.
 
 from . import abi, synth  # noqa: F401
 from .abi import (  # noqa: F401
+    fs_debug_block,
     fs_debug_capture,
     fs_debug_dequant_q8_0,
     fs_debug_lm_head,

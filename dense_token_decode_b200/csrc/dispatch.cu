@@ -5,12 +5,9 @@
 
 namespace fs {
 
-fs_status init_extras(fs_model* m) {
-  (void)m;
-  return FS_OK;
-}
+fs_status init_extras(fs_model* m) { return mega_init(m); }
 
-void release_extras(fs_model* m) { (void)m; }
+void release_extras(fs_model* m) { mega_release(m); }
 
 fs_status ensure_gen_buffer(fs_model* m, int n) {
   if (n <= m->gen_cap) return FS_OK;
@@ -33,8 +30,17 @@ fs_status prefill_chunk(fs_model* m, const fs_kv* kv, const RowMap& map, int row
                          capture_rows, st);
 }
 
+fs_status block_prefill_or_general(fs_model* m, const fs_kv* kv, const RowMap& map, int rows,
+                                   int l, cudaStream_t st) {
+  return layer_general(m, kv, map, rows, l, st);
+}
+
 fs_status decode_rows(fs_model* m, const fs_kv* kv, const RowMap& map, int rows,
                       const int32_t* tok, float* logits, int32_t* argmax, cudaStream_t st) {
+  // Distinct sequences (checked by the caller), at most 4: the persistent kernel.
+  fs_status s = decode_mega(m, kv, map, rows, tok, nullptr, nullptr, 0, m->s.L, true, logits,
+                            argmax, st);
+  if (s != FS_ERR_UNSUPPORTED) return s;
   return forward_general(m, kv, map, rows, tok, 0, logits, argmax, 0, rows, st);
 }
 

@@ -221,6 +221,7 @@ extern "C" fs_status fs_device_error(fs_model* m, int32_t* code) {
   int v = 0;
   FS_CUDA(cudaMemcpy(&v, m->err, sizeof(int), cudaMemcpyDeviceToHost));
   FS_CUDA(cudaMemset(m->err, 0, sizeof(int)));
+  if (v) fs::mega_reset(m);
   *code = v;
   return FS_OK;
 }
@@ -357,15 +358,44 @@ static cudaError_t linear(const fs_model* m, const float* x, int rows, int K, in
   return launch_gemm_simt(x, rows, K, L.w[which], L.s[which], N, out, ldo, acc, st);
 }
 
+// One block over m->h (in place): RMSNorm, Q/K/V, head norm + RoPE + KV
+// append, attention, O + residual, RMSNorm, SwiGLU MLP + residual.
+fs_status layer_general(fs_model* m, const fs_kv* kv, const RowMap& map, int rows, int l,
+                      cudaStream_t st) {
+  const Shape& s = m->s;
+  const KVView kvv = kv_view(kv);
+  const int H = s.H, qd = s.q_dim(), kvd = s.kv_dim(), qkvd = s.qkv_dim();
+  const LayerDev& Lw = m->layers[l];
+  FS_CUDA(launch_rmsnorm(m->h, rows, H, Lw.attn_norm, s.eps, m->xn, st));
+  FS_CUDA(linear(m, m->xn, rows, H, l, kWq, qd, m->qkv, qkvd, false, st));
+  FS_CUDA(linear(m, m->xn, rows, H, l, kWk, kvd, m->qkv + qd, qkvd, false, st));
+  FS_CUDA(linear(m, m->xn, rows, H, l, kWv, kvd, m->qkv + qd + kvd, qkvd, false, st));
+  FS_CUDA(launch_qk_norm_rope_append(m->qkv, rows, map, s, Lw.q_norm, Lw.k_norm, m->rope, m->q,
+                                     kvv, l, st));
+  FS_CUDA(launch_attention_simple(m->q, rows, map, s, kvv, l, m->o, st));
+  FS_CUDA(linear(m, m->o, rows, qd, l, kWo, H, m->h, H, true, st));
+  FS_CUDA(launch_rmsnorm(m->h, rows, H, Lw.ffn_norm, s.eps, m->xn, st));
+  if (rows <= 16) {
+    FS_CUDA(launch_gemv_swiglu(m->xn, rows, H, Lw.w[kWg], Lw.s[kWg], Lw.w[kWu], Lw.s[kWu], s.I,
+                               m->act, st));
+  } else {
+    FS_CUDA(linear(m, m->xn, rows, H, l, kWg, s.I, m->gu, 2 * s.I, false, st));
+    FS_CUDA(linear(m, m->xn, rows, H, l, kWu, s.I, m->gu + s.I, 2 * s.I, false, st));
+    FS_CUDA(launch_swiglu(m->gu, rows, s.I, m->act, st));
+  }
+  FS_CUDA(linear(m, m->act, rows, s.I, l, kWd, H, m->h, H, true, st));
+  return FS_OK;
+}
+
 // The general forward over `rows` rows described by `map`, tokens on the
 // device. Writes logits/argmax for the rows selected by `head_rows`:
 // head_first .. rows-1 (prefill: the last row; decode: every row).
 fs_status forward_general(fs_model* m, const fs_kv* kv, const RowMap& map, int rows,
                           const int32_t* tok, int head_first, float* logits, int32_t* argmax,
                           int capture_row0, int capture_rows, cudaStream_t st) {
+  (void)capture_rows;
   const Shape& s = m->s;
-  const KVView kvv = kv_view(kv);
-  const int H = s.H, qd = s.q_dim(), kvd = s.kv_dim(), qkvd = s.qkv_dim();
+  const int H = s.H;
   FS_CUDA(launch_embed(tok, rows, m->embed, H, s.V, m->h, m->err, st));
   auto capture = [&](int slot) -> cudaError_t {
     if (!m->capture) return cudaSuccess;
@@ -376,25 +406,8 @@ fs_status forward_general(fs_model* m, const fs_kv* kv, const RowMap& map, int r
   };
   FS_CUDA(capture(0));
   for (int l = 0; l < s.L; ++l) {
-    const LayerDev& Lw = m->layers[l];
-    FS_CUDA(launch_rmsnorm(m->h, rows, H, Lw.attn_norm, s.eps, m->xn, st));
-    FS_CUDA(linear(m, m->xn, rows, H, l, kWq, qd, m->qkv, qkvd, false, st));
-    FS_CUDA(linear(m, m->xn, rows, H, l, kWk, kvd, m->qkv + qd, qkvd, false, st));
-    FS_CUDA(linear(m, m->xn, rows, H, l, kWv, kvd, m->qkv + qd + kvd, qkvd, false, st));
-    FS_CUDA(launch_qk_norm_rope_append(m->qkv, rows, map, s, Lw.q_norm, Lw.k_norm, m->rope, m->q,
-                                       kvv, l, st));
-    FS_CUDA(launch_attention_simple(m->q, rows, map, s, kvv, l, m->o, st));
-    FS_CUDA(linear(m, m->o, rows, qd, l, kWo, H, m->h, H, true, st));
-    FS_CUDA(launch_rmsnorm(m->h, rows, H, Lw.ffn_norm, s.eps, m->xn, st));
-    if (rows <= 16) {
-      FS_CUDA(launch_gemv_swiglu(m->xn, rows, H, Lw.w[kWg], Lw.s[kWg], Lw.w[kWu], Lw.s[kWu], s.I,
-                                 m->act, st));
-    } else {
-      FS_CUDA(linear(m, m->xn, rows, H, l, kWg, s.I, m->gu, 2 * s.I, false, st));
-      FS_CUDA(linear(m, m->xn, rows, H, l, kWu, s.I, m->gu + s.I, 2 * s.I, false, st));
-      FS_CUDA(launch_swiglu(m->gu, rows, s.I, m->act, st));
-    }
-    FS_CUDA(linear(m, m->act, rows, s.I, l, kWd, H, m->h, H, true, st));
+    fs_status ls = layer_general(m, kv, map, rows, l, st);
+    if (ls != FS_OK) return ls;
     FS_CUDA(capture(l + 1));
   }
   const int nh = rows - head_first;
@@ -598,6 +611,7 @@ extern "C" fs_status fs_greedy(fs_model* m, fs_kv* kv, int32_t seq, const int32_
   FS_CUDA(cudaMemcpy(&derr, m->err, sizeof(int), cudaMemcpyDeviceToHost));
   if (derr) {
     cudaMemset(m->err, 0, sizeof(int));
+    fs::mega_reset(m);
     return fail(FS_ERR_DEVICE, "a kernel reported device error " + std::to_string(derr));
   }
   *n_out = produced;
@@ -619,6 +633,40 @@ extern "C" fs_status fs_debug_capture(fs_model* m, float* hidden, int32_t max_ro
   if (max_rows <= 0) return fail(FS_ERR_INVALID, "max_rows must be positive");
   m->capture = hidden;
   m->capture_max_rows = max_rows;
+  return FS_OK;
+}
+
+extern "C" fs_status fs_debug_block(fs_model* m, fs_kv* kv, int32_t seq, int32_t layer,
+                                    const float* h_in, int32_t rows, float* h_out, void* stream) {
+  if (!m || !kv) return fail(FS_ERR_NULL, "model or kv is NULL");
+  if (kv->model != m) return fail(FS_ERR_INVALID, "kv belongs to another model");
+  if (seq < 0 || seq >= kv->max_seqs) return fail(FS_ERR_SEQ, "sequence out of range");
+  if (layer < 0 || layer >= m->s.L) return fail(FS_ERR_INVALID, "layer out of range");
+  if (rows <= 0 || rows > m->max_rows) return fail(FS_ERR_INVALID, "rows out of range");
+  fs_status s;
+  if ((s = check_device_ptr(h_in, "h_in")) != FS_OK || (s = check_device_ptr(h_out, "h_out")) != FS_OK)
+    return s;
+  const int pos0 = kv->len[seq];
+  if ((long long)pos0 + rows > fs::kv_capacity(kv))
+    return fail(FS_ERR_CONTEXT, "block rows would exceed the KV capacity");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  fs::RowMap map{};
+  map.n_list = 0;
+  map.seq0 = seq;
+  map.pos0 = pos0;
+  if (rows == 1) {
+    map.n_list = 1;
+    map.seq[0] = seq;
+    map.pos[0] = pos0;
+    s = fs::decode_mega(m, kv, map, 1, nullptr, h_in, h_out, layer, layer + 1, false, nullptr,
+                        nullptr, st);
+    if (s != FS_ERR_UNSUPPORTED) return s;
+  }
+  FS_CUDA(cudaMemcpyAsync(m->h, h_in, (size_t)rows * m->s.H * sizeof(float),
+                          cudaMemcpyDeviceToDevice, st));
+  if ((s = fs::block_prefill_or_general(m, kv, map, rows, layer, st)) != FS_OK) return s;
+  FS_CUDA(cudaMemcpyAsync(h_out, m->h, (size_t)rows * m->s.H * sizeof(float),
+                          cudaMemcpyDeviceToDevice, st));
   return FS_OK;
 }
 
@@ -648,6 +696,16 @@ extern "C" fs_status fs_debug_lm_head(fs_model* m, const float* x, int32_t rows,
   FS_CUDA(fs::launch_rmsnorm(x, rows, m->s.H, m->final_norm, m->s.eps, m->xf, st));
   FS_CUDA(fs::launch_lm_head(m->xf, rows, m->s, m->embed, logits, argmax, m->partial, m->n_part,
                              m->err, st));
+  return FS_OK;
+}
+
+extern "C" fs_status fs_debug_trace(fs_model* m, uint64_t* buf) {
+  if (!m) return fail(FS_ERR_NULL, "model is NULL");
+  if (buf) {
+    fs_status s = check_device_ptr(buf, "trace buffer");
+    if (s != FS_OK) return s;
+  }
+  m->trace = reinterpret_cast<unsigned long long*>(buf);
   return FS_OK;
 }
 

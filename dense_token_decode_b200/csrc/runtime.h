@@ -37,6 +37,7 @@ struct fs_model {
   float* capture = nullptr;   // armed fs_debug_capture buffer
   int capture_max_rows = 0;
   int prefill_split = 1;
+  unsigned long long* trace = nullptr;  // armed fs_debug_trace buffer
   void* extras = nullptr;     // fast-path state
 };
 
@@ -76,6 +77,22 @@ fs_status prefill_chunk(fs_model* m, const fs_kv* kv, const RowMap& map, int row
 // One decode step over a batch of sequences.
 fs_status decode_rows(fs_model* m, const fs_kv* kv, const RowMap& map, int rows,
                       const int32_t* tok, float* logits, int32_t* argmax, cudaStream_t st);
+
+// Persistent decode kernel (decode_mega.cu).
+fs_status mega_init(fs_model* m);
+void mega_release(fs_model* m);
+void mega_reset(fs_model* m);
+fs_status decode_mega(fs_model* m, const fs_kv* kv, const RowMap& map, int B, const int32_t* tok,
+                      const float* h_in, float* h_out, int l0, int l1, bool run_head,
+                      float* logits, int32_t* argmax, cudaStream_t stream);
+
+// One block of the general path on m->h (rows described by map).
+fs_status layer_general(fs_model* m, const fs_kv* kv, const RowMap& map, int rows, int l,
+                        cudaStream_t st);
+
+// The block kernels the prefill path uses for `rows` rows (debug entry point).
+fs_status block_prefill_or_general(fs_model* m, const fs_kv* kv, const RowMap& map, int rows,
+                                   int l, cudaStream_t st);
 
 fs_status prefill_impl(fs_model* m, fs_kv* kv, int32_t seq, const int32_t* tokens, int32_t n,
                        float* logits, int32_t* argmax, cudaStream_t st);

@@ -111,6 +111,14 @@ class Model:
     def capture(self, hidden: torch.Tensor | None, max_rows: int = 0):
         abi.check(abi.fs_debug_capture(self.handle, _ptr(hidden), max_rows), "fs_debug_capture")
 
+    def block(self, kv: "KV", seq: int, layer: int, h_in: torch.Tensor, stream=None):
+        """Run one block alone (fs_debug_block); returns h_out."""
+        h_out = torch.empty_like(h_in)
+        abi.check(abi.fs_debug_block(self.handle, kv.handle, seq, layer, h_in.data_ptr(),
+                                     h_in.shape[0], h_out.data_ptr(), _stream(stream)),
+                  "fs_debug_block")
+        return h_out
+
     def lm_head(self, x: torch.Tensor, logits=None, argmax=None, stream=None):
         abi.check(abi.fs_debug_lm_head(self.handle, _ptr(x), x.shape[0], _ptr(logits),
                                        _ptr(argmax), _stream(stream)), "fs_debug_lm_head")

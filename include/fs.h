@@ -211,6 +211,26 @@ fs_status fs_greedy(fs_model* model, fs_kv* kv, int32_t seq, const int32_t* prom
  * not captured. One-shot: capture is disarmed after that call. NULL disarms. */
 fs_status fs_debug_capture(fs_model* model, float* hidden, int32_t max_rows);
 
+/* Debug: run block `layer` alone on `rows` rows of sequence `seq` at positions
+ * length .. length+rows-1, from the residual-stream input h_in (device fp32
+ * [rows, H]) to the block output h_out (device fp32 [rows, H]). It uses the
+ * kernels the product path uses for that row count (one row: the persistent
+ * decode kernel), reads the layer's cached K/V of earlier positions and writes
+ * the layer's K/V for these positions; the sequence length is not changed.
+ * Used to measure each block's own error given a reference input.
+ * Errors: FS_ERR_NULL, FS_ERR_SEQ, FS_ERR_INVALID, FS_ERR_CONTEXT, FS_ERR_ALIGN. */
+fs_status fs_debug_block(fs_model* model, fs_kv* kv, int32_t seq, int32_t layer,
+                         const float* h_in, int32_t rows, float* h_out, void* stream);
+
+/* Debug: the next decode step that runs on the persistent decode kernel
+ * records %globaltimer stamps (ns) into `buf` (device uint64
+ * [SMs][n_layers+1][8]): per CTA and layer, slot 0 phase start, 1 block input
+ * ready, 2 attention input ready, 3 O start, 4 O input ready, 5 MLP input
+ * ready, 6 down input ready, 7 layer done; row n_layers holds the LM head
+ * (0 start, 1 input ready, 7 done). Slots a CTA never reaches are left as
+ * they were. One-shot; NULL disarms. Timing only: no work changes. */
+fs_status fs_debug_trace(fs_model* model, uint64_t* buf);
+
 /* Debug: dequantise Q8_0 blocks to fp32, out[n*k] = codes[n*k] * scales[n*(k/32)]
  * (all device, row-major). Bit-exact by construction. k % 32 == 0. */
 fs_status fs_debug_dequant_q8_0(const int8_t* codes, const void* scales, int32_t n, int32_t k,

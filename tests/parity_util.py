@@ -9,9 +9,15 @@ import torch
 import oracle
 
 # Acceptance bars of the forward pass against the fp64 oracle.
-BLOCK_REL_L2 = 1e-3   # per-block hidden-state relative L2
-LOGIT_ABS = 2e-2      # max |delta logit|
-GREEDY_STEPS = 32     # greedy ids must agree for this many steps
+BLOCK_REL_L2 = 1e-3   # per-block hidden-state relative L2: each block's own error,
+                      # the block fed the oracle's input to it (fs_debug_block)
+LOGIT_ABS = 2e-2      # max |delta logit|, end to end
+GREEDY_STEPS = 32     # greedy ids must agree for this many steps, end to end
+# Sanity bound on the hidden states of a whole end-to-end run. Rounding K and V
+# to bf16 (as the cache stores them) turns fp32 rounding noise into whole-ulp
+# flips, which adds about 4e-5 relative L2 per block; after 28 blocks an fp32
+# forward sits near 1.1e-3. This bound only catches gross errors.
+E2E_BLOCK_REL_L2 = 3e-3
 
 
 def rel_l2(a, b) -> float:
@@ -51,6 +57,10 @@ def check_greedy_step(gpu_id: int, gpu_logits, ref_logits) -> bool:
     close = np.flatnonzero(np.asarray(ref_logits) >= np.max(ref_logits) - margin)
     assert gpu_id in close, f"greedy id {gpu_id} not within the ambiguity margin of {ref_id}"
     return False
+
+
+def to_dev(a, device="cuda:0", dtype=torch.float32) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dtype).to(device)
 
 
 def oracle_tensor(t: torch.Tensor) -> np.ndarray:

@@ -20,8 +20,9 @@ import oracle
 from conftest import oracle_weights
 from dense_token_decode_b200 import abi, synth
 from dense_token_decode_b200.engine import Model
-from parity_util import (BLOCK_REL_L2, GREEDY_STEPS, LOGIT_ABS, assert_blocks_close,
-                         assert_logits_close, check_greedy_step, oracle_tensor, rel_l2)
+from parity_util import (BLOCK_REL_L2, E2E_BLOCK_REL_L2, GREEDY_STEPS, LOGIT_ABS,
+                         assert_blocks_close, assert_logits_close, check_greedy_step,
+                         oracle_tensor, rel_l2, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -79,6 +80,47 @@ def prefill_with_capture(pair, kv, seq, toks):
     return oracle_tensor(logits), oracle_tensor(hidden), int(am.item())
 
 
+def blocks_local_prefill(pair, toks, oracle_run=None):
+    """Each block alone on the oracle's input (a prefill of len(toks) rows at
+    positions 0..): its output and the K/V it stores, against the oracle."""
+    s = pair.shape
+    rl, rh, cache = oracle_run if oracle_run is not None else pair.oracle.forward(toks)
+    kv = pair.model.kv(1, len(toks))
+    errs, kv_errs = [], []
+    for l in range(s.n_layers):
+        out = pair.model.block(kv, 0, l, to_dev(rh[l]))
+        torch.cuda.synchronize()
+        errs.append(rel_l2(oracle_tensor(out), rh[l + 1]))
+        k, v = kv.export(0, l, 0, len(toks))
+        kv_errs.append(max(rel_l2(oracle_tensor(k), cache.k[l]),
+                           rel_l2(oracle_tensor(v), cache.v[l])))
+    assert max(errs) <= BLOCK_REL_L2, f"block-local rel-L2 {max(errs):.3e}: {errs}"
+    assert max(kv_errs) <= BLOCK_REL_L2, f"block-local KV rel-L2 {max(kv_errs):.3e}: {kv_errs}"
+    return errs
+
+
+def blocks_local_decode(pair, toks, next_tok):
+    """Each block alone at one decode position: the GPU cache holds the
+    oracle's K/V of the earlier positions and the block gets the oracle's input."""
+    s = pair.shape
+    _, _, cache = pair.oracle.forward(toks)
+    ref = oracle.KVCache(k=list(cache.k), v=list(cache.v))
+    _, rh, _ = pair.oracle.forward([next_tok], ref)
+    P = len(toks)
+    kv = pair.model.kv(1, P + 8)
+    for l in range(s.n_layers):
+        kv.import_(0, l, 0, to_dev(cache.k[l], dtype=torch.bfloat16),
+                   to_dev(cache.v[l], dtype=torch.bfloat16))
+    kv.set_length(0, P)
+    errs = []
+    for l in range(s.n_layers):
+        out = pair.model.block(kv, 0, l, to_dev(rh[l]))
+        torch.cuda.synchronize()
+        errs.append(rel_l2(oracle_tensor(out), rh[l + 1]))
+    assert max(errs) <= BLOCK_REL_L2, f"decode block-local rel-L2 {max(errs):.3e}: {errs}"
+    return errs
+
+
 def decode_teacher_forced(pair, kv, seq, first_tok, ref_ids, ref_logits, capture_steps=()):
     """GPU decode fed the oracle's ids; checks every step. Returns ambiguous count."""
     m, s = pair.model, pair.shape
@@ -110,8 +152,9 @@ def test_tiny_prefill_logits_blocks_and_cache(tiny):
     kv = tiny.model.kv(2, 64)
     gl, gh, am = prefill_with_capture(tiny, kv, 0, toks)
     rl, rh, cache = tiny.oracle.forward(toks)
-    assert_blocks_close(gh, rh, what="tiny prefill")
+    assert_blocks_close(gh, rh, tol=E2E_BLOCK_REL_L2, what="tiny prefill end to end")
     assert_logits_close(gl, rl, what="tiny prefill")
+    blocks_local_prefill(tiny, toks, (rl, rh, cache))
     assert am == oracle.greedy_select(rl) or abs(rl[am] - rl.max()) < 2 * np.abs(gl - rl).max()
     for l in range(tiny.shape.n_layers):
         k, v = kv.export(0, l, 0, 16)
@@ -134,8 +177,9 @@ def test_tiny_decode_teacher_forced(tiny):
     for i, tok in enumerate(prefix_ids):
         _, rh, cache = tiny.oracle.forward([tok], cache)
         if i in hid:
-            assert_blocks_close(hid[i], rh, what=f"tiny decode step {i}")
+            assert_blocks_close(hid[i], rh, tol=E2E_BLOCK_REL_L2, what=f"tiny decode step {i}")
     assert amb <= 4
+    blocks_local_decode(tiny, toks + ids[:10], ids[10])
 
 
 def test_tiny_fs_greedy_matches_oracle(tiny):
@@ -209,7 +253,7 @@ def test_tiny_single_token_prefill_returns_v_path(tiny):
     kv = tiny.model.kv(1, 8)
     gl, gh, _ = prefill_with_capture(tiny, kv, 0, [7])
     rl, rh, _ = tiny.oracle.forward([7])
-    assert_blocks_close(gh, rh, what="S=1")
+    assert_blocks_close(gh, rh, tol=E2E_BLOCK_REL_L2, what="S=1")
     assert_logits_close(gl, rl, what="S=1")
 
 
@@ -311,7 +355,7 @@ def test_qwen_decode_bs1_parity(qwen):
     kv = qwen.model.kv(1, 512)
     gl, gh, am = prefill_with_capture(qwen, kv, 0, toks)
     _, rh, _ = qwen.oracle.forward(toks)
-    assert_blocks_close(gh, rh, what="qwen prefill 8")
+    assert_blocks_close(gh, rh, tol=E2E_BLOCK_REL_L2, what="qwen prefill 8 end to end")
     assert_logits_close(gl, ref_logits[0])
     check_greedy_step(am, gl, ref_logits[0])
     amb, hid = decode_teacher_forced(qwen, kv, 0, ids[0], ids[1:], ref_logits[1:],
@@ -320,8 +364,11 @@ def test_qwen_decode_bs1_parity(qwen):
     for i, tok in enumerate([ids[0]] + ids[1:32]):
         _, rh, cache = qwen.oracle.forward([tok], cache)
         if i in hid:
-            assert_blocks_close(hid[i], rh, what=f"qwen decode step {i}")
+            assert_blocks_close(hid[i], rh, tol=E2E_BLOCK_REL_L2,
+                                what=f"qwen decode step {i} end to end")
     assert amb <= 8
+    blocks_local_decode(qwen, toks + ids[:31], ids[31])
+    blocks_local_prefill(qwen, toks)
 
 
 def test_qwen_fs_greedy_free_running(qwen):
@@ -346,10 +393,12 @@ def test_qwen_q8_0_decode_parity():
     kv = pair.model.kv(1, 512)
     gl, gh, am = prefill_with_capture(pair, kv, 0, toks)
     _, rh, _ = pair.oracle.forward(toks)
-    assert_blocks_close(gh, rh, what="q8_0 prefill 8")
+    assert_blocks_close(gh, rh, tol=E2E_BLOCK_REL_L2, what="q8_0 prefill 8 end to end")
     check_greedy_step(am, gl, ref_logits[0])
     amb, _ = decode_teacher_forced(pair, kv, 0, ids[0], ids[1:], ref_logits[1:])
     assert amb <= 8
+    blocks_local_decode(pair, toks + ids[:31], ids[31])
+    blocks_local_prefill(pair, toks)
     pair.model.close()
 
 
@@ -361,13 +410,15 @@ def test_qwen_prefill_2048(qwen):
     kv = qwen.model.kv(1, S)
     gl, gh, am = prefill_with_capture(qwen, kv, 0, toks)
     rl, rh, cache = qwen.oracle.forward(toks)
-    assert_blocks_close(gh, rh, what="prefill 2048")
+    assert_blocks_close(gh, rh, tol=E2E_BLOCK_REL_L2, what="prefill 2048 end to end")
     assert_logits_close(gl, rl, what="prefill 2048")
     check_greedy_step(am, gl, rl)
     for l in range(qwen.shape.n_layers):
         k, v = kv.export(0, l, 0, S)
-        assert rel_l2(oracle_tensor(k), cache.k[l]) <= BLOCK_REL_L2, l
-        assert rel_l2(oracle_tensor(v), cache.v[l]) <= BLOCK_REL_L2, l
+        assert rel_l2(oracle_tensor(k), cache.k[l]) <= E2E_BLOCK_REL_L2, l
+        assert rel_l2(oracle_tensor(v), cache.v[l]) <= E2E_BLOCK_REL_L2, l
+    kv.close()
+    blocks_local_prefill(qwen, toks, (rl, rh, cache))
 
 
 def test_qwen_batched_decode_long_context(qwen):
