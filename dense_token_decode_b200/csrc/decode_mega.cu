@@ -32,7 +32,7 @@
 namespace fs {
 namespace mega {
 
-constexpr int kConsumerWarps = 8;
+constexpr int kConsumerWarps = 11;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;  // + producer warp
 constexpr int kMaxB = 4;
@@ -77,11 +77,33 @@ struct Params {
   int capture_stride;
   int* err;
   int* abort_flag;  // set on a timeout: every wait gives up
-  unsigned long long* trace;  // optional: %globaltimer stamps [G][L+1][8]
+  unsigned long long* trace;  // optional: %globaltimer stamps [G][L+1][16]
   int n_stages;
   // smem carve-up (bytes)
-  int off_hs, off_xs, off_attn, off_red, off_bar, off_misc;
+  int off_hs, off_xs, off_attn, off_red, off_bar, off_misc, off_tab;
+  int bt_in_smem;  // block-table rows of the batch copied to shared memory
 };
+
+// Shared-memory copies of the per-layer weight pointers and of the batch's
+// block-table rows: the producer thread looks them up for every chunk, and a
+// global-memory round trip there would stall the whole weight stream.
+__device__ __forceinline__ const LayerDev* layers_s(const Params& p) {
+  extern __shared__ __align__(1024) unsigned char smem_base[];
+  return reinterpret_cast<const LayerDev*>(smem_base + p.off_tab);
+}
+__device__ __forceinline__ size_t kv_off(const Params& p, int layer, int b, int pos, int g) {
+  extern __shared__ __align__(1024) unsigned char smem_base[];
+  int page;
+  if (p.bt_in_smem) {
+    const int32_t* bt = reinterpret_cast<const int32_t*>(
+        smem_base + p.off_tab + (size_t)p.L * sizeof(LayerDev));
+    page = bt[b * p.kv.pages_per_seq + pos / kPage];
+  } else {
+    page = p.kv.block_table[(size_t)p.seq[b] * p.kv.pages_per_seq + pos / kPage];
+  }
+  return (size_t)layer * p.kv.layer_elems() +
+         (((size_t)page * p.kv.n_kv_heads + g) * kPage + (pos % kPage)) * p.kv.head_dim;
+}
 
 // ---------------------------------------------------------------------------
 // PTX helpers
@@ -107,6 +129,19 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
       " selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
       : "r"(su32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// As mbar_test, but a thread whose phase is not complete sleeps (up to
+// hint_ns) instead of returning at once, so waiting warps leave the issue
+// slots to the warps that compute; it wakes when the phase completes.
+__device__ __forceinline__ bool mbar_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(su32(bar)), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
@@ -166,16 +201,18 @@ __device__ __forceinline__ float hi16(uint32_t u) { return __uint_as_float(u & 0
 // Shapes of the chunk stream (identical in producer and consumers)
 
 struct ChunkShape {
-  int rows;  // weight rows per chunk (gate/up: pairs)
-  int segs;  // warps per row
+  int rows;  // weight rows per chunk (gate/up: pairs), at most one per consumer warp
 };
 
+// The largest power of two of whole rows (gate/up: row pairs) that fits one
+// stage, at most 8 rows or 4 pairs (one warp finishes at most 8 dot products
+// per chunk).
 __host__ __device__ inline ChunkShape chunk_shape(int K, bool q8, bool pair) {
-  const int row_bytes = q8 ? K : 2 * K;
-  const int mult = pair ? 2 : 1;
-  int rows = 8 / mult;
-  while (rows > 1 && rows * mult * row_bytes > kWeightBytes) rows >>= 1;
-  return ChunkShape{rows, kConsumerWarps / (rows * mult)};
+  const int row_bytes = (q8 ? K : 2 * K) * (pair ? 2 : 1);
+  const int cap = pair ? 4 : 8;
+  int rows = 1;
+  while (rows * 2 <= cap && rows * 2 * row_bytes <= kWeightBytes) rows *= 2;
+  return ChunkShape{rows * row_bytes <= kWeightBytes ? rows : 0};
 }
 
 __host__ __device__ inline int keys_per_chunk(int d) { return kWeightBytes / (4 * d); }
@@ -214,7 +251,7 @@ __device__ inline Item item_desc(const Params& p, int it) {
 // Source of weight row n of a phase (QKV rows span wq|wk|wv).
 __device__ inline const void* row_src(const Params& p, int phase, int layer, int n, int K,
                                       const __half** scale_row, int* limit) {
-  const LayerDev& Lw = p.layers[layer];
+  const LayerDev& Lw = layers_s(p)[layer];
   int which = 0, local = n, end = 0;
   const int qd = p.nq * p.d, kvd = p.nkv * p.d;
   switch (phase) {
@@ -359,9 +396,9 @@ struct Producer {
     const int s = stage;
     unsigned long long t0 = 0;
     int spins = 0;
-    while (!mbar_test(&r.empty[s], parity)) {
+    while (!mbar_wait_hint(&r.empty[s], parity, 20000)) {
       // The clock only starts after many failed polls: reading it is not free.
-      if ((++spins & 1023) == 0) {
+      if ((++spins & 15) == 0) {
         if (t0 == 0) t0 = now_ns();
         if (aborted(p.abort_flag) || now_ns() - t0 > kTimeoutNs) {
           if (!aborted(p.abort_flag)) raise_timeout(p);
@@ -389,7 +426,7 @@ struct Producer {
   __device__ void gemv(int phase, int layer, int n0, int nr, int K, ChunkShape cs) {
     if (quit) return;
     if (p.trace && phase == kLM) {
-      unsigned long long* t = p.trace + ((size_t)blockIdx.x * (p.L + 1) + p.L) * 8;
+      unsigned long long* t = p.trace + ((size_t)blockIdx.x * (p.L + 1) + p.L) * 16;
       if (!lm_started) t[2] = now_ns();
       lm_started = true;
     }
@@ -407,7 +444,7 @@ struct Producer {
     bulk_load(st, src, nr * rb, bar, policy);
     if (q8) bulk_load(st + kWeightBytes, sr, nr * sb, bar, policy);
     if (pair) {
-      const LayerDev& Lw = p.layers[layer];
+      const LayerDev& Lw = layers_s(p)[layer];
       if (q8) {
         bulk_load(st + cs.rows * rb, static_cast<const int8_t*>(Lw.w[kWu]) + (size_t)n0 * K,
                   nr * rb, bar, policy);
@@ -427,7 +464,7 @@ struct Producer {
     const uint32_t bytes = 2u * nk * p.d * 2;
     unsigned char* st = acquire(bytes);
     if (!st) return;
-    const size_t off = p.kv.offset(layer, p.seq[x.b], j, x.g);
+    const size_t off = kv_off(p, layer, x.b, j, x.g);
     uint64_t* bar = &r.full[stage];
     bulk_load(st, p.kv.k + off, nk * p.d * 2, bar, policy);
     bulk_load(st + kWeightBytes / 2, p.kv.v + off, nk * p.d * 2, bar, policy);
@@ -448,7 +485,7 @@ struct Consumer {
   float* comb;  // [stages][8 rows][2][kMaxB] partial sums of split rows
   int* ccnt;    // [stages][8 rows] arrivals per split row
   float* at;    // attention scratch
-  unsigned long long wbest = 0ull;  // lane b: this warp's greedy key of batch row b
+  unsigned long long wbest[kMaxB] = {0ull, 0ull, 0ull, 0ull};  // this lane's greedy keys
   unsigned long long* best;  // [kMaxB] greedy keys of this CTA
   int* flag;
   unsigned int i = 0;  // chunks consumed
@@ -480,7 +517,7 @@ struct Consumer {
 
   // Timestamp slot k of (this CTA, layer) into the optional trace.
   __device__ void tr(int layer, int k) {
-    if (p.trace && tid == 0) p.trace[((size_t)cta * (p.L + 1) + layer) * 8 + k] = now_ns();
+    if (p.trace && tid == 0) p.trace[((size_t)cta * (p.L + 1) + layer) * 16 + k] = now_ns();
   }
 
   __device__ uint32_t tag(int layer, int ph) const {
@@ -498,9 +535,9 @@ struct Consumer {
     // copy's bytes visible to it); the give-up decision is lane 0's, so the
     // warp stays converged for the shuffles that follow.
     while (true) {
-      const bool ok = quit || mbar_test(&r.full[s], parity);
+      const bool ok = quit || mbar_wait_hint(&r.full[s], parity, 20000);
       if (__all_sync(0xffffffffu, ok)) break;
-      if ((++spins & 1023) == 0) {
+      if ((++spins & 15) == 0) {
         int bad = 0;
         if (lane == 0) {
           if (t0 == 0) t0 = now_ns();
@@ -544,6 +581,7 @@ struct Consumer {
           unsigned long long t0 = 0;
           int spins = 0;
           do {
+            __nanosleep(32);
             w[u] = ld_tag(src + k);
             if ((++spins & 255) == 0) {
               if (t0 == 0) t0 = now_ns();
@@ -560,14 +598,28 @@ struct Consumer {
     }
   }
 
-  // RMSNorm of the B rows of hs into xs with bf16 gains g.
-  __device__ __forceinline__ void rmsnorm_rows(const __nv_bfloat16* g) {
+  // Gains of an RMSNorm, element tid + 256 j in register j (H <= 2048),
+  // fetched before the wait for the activations so their latency overlaps it.
+  __device__ __forceinline__ void load_gains(const __nv_bfloat16* g, float (&gr)[8]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int k = tid + kConsumers * j;
+      gr[j] = k < p.H ? __bfloat162float(g[k]) : 0.f;
+    }
+  }
+
+  // RMSNorm of the B rows of hs into xs with the preloaded gains.
+  __device__ __forceinline__ void rmsnorm_rows(const float (&gr)[8]) {
     const int H = p.H;
     for (int b = 0; b < p.B; ++b) {
       float ss = 0.f;
-      for (int k = tid; k < H; k += kConsumers) {
-        const float v = hs[b * H + k];
-        ss += v * v;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int k = tid + kConsumers * j;
+        if (k < H) {
+          const float v = hs[b * H + k];
+          ss += v * v;
+        }
       }
       for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
       if (lane == 0) at[warp] = ss;
@@ -576,8 +628,11 @@ struct Consumer {
 #pragma unroll
       for (int w = 0; w < kConsumerWarps; ++w) tot += at[w];
       const float inv = rsqrtf(tot / (float)H + p.eps);
-      for (int k = tid; k < H; k += kConsumers)
-        xs[b * H + k] = hs[b * H + k] * inv * __bfloat162float(g[k]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int k = tid + kConsumers * j;
+        if (k < H) xs[b * H + k] = hs[b * H + k] * inv * gr[j];
+      }
       consumer_sync();
     }
   }
@@ -586,12 +641,16 @@ struct Consumer {
     // Warps may still be on the previous phase's chunks (they read xs/hs).
     quit = consumer_sync_or(quit);
     if (quit) return;
+    if (ph == kGU) tr(layer, 10);
+    if (ph == kDown) tr(layer, 11);
     const int slot_layer = ph == kLM ? p.L : layer;
     if (ph == kQKV || ph == kO || ph == kLM) tr(slot_layer, ph == kO ? 3 : 0);
     const int H = p.H;
-    const LayerDev& Lw = p.layers[layer];
+    const LayerDev& Lw = layers_s(p)[layer];
+    float gr[8];
     switch (ph) {
       case kQKV:
+        load_gains(Lw.attn_norm, gr);
         if (layer == p.l0) {
           for (int b = 0; b < p.B; ++b) {
             if (p.h_in) {
@@ -617,7 +676,7 @@ struct Consumer {
           if (quit) return;
         }
         tr(layer, 1);
-        rmsnorm_rows(Lw.attn_norm);
+        rmsnorm_rows(gr);
         break;
       case kO:
         wait_words(p.xo, p.B * p.nq * p.d, tag(layer, 2), xs);
@@ -625,11 +684,12 @@ struct Consumer {
         tr(layer, 4);
         break;
       case kGU:
+        load_gains(Lw.ffn_norm, gr);
         wait_words(p.xh0, p.B * H, tag(layer, 3), hs);
         quit = consumer_sync_or(quit);
         if (quit) return;
         tr(layer, 5);
-        rmsnorm_rows(Lw.ffn_norm);
+        rmsnorm_rows(gr);
         break;
       case kDown:
         wait_words(p.xa, p.B * p.I, tag(layer, 4), xs);
@@ -637,6 +697,7 @@ struct Consumer {
         tr(layer, 6);
         break;
       case kLM:
+        load_gains(p.final_norm, gr);
         if (p.l1 > p.l0) {
           wait_words(p.xh1, p.B * H, tag(p.l1 - 1, 5), hs);
         } else {
@@ -645,7 +706,7 @@ struct Consumer {
         quit = consumer_sync_or(quit);
         if (quit) return;
         tr(p.L, 1);
-        rmsnorm_rows(p.final_norm);
+        rmsnorm_rows(gr);
         break;
     }
   }
@@ -659,149 +720,151 @@ struct Consumer {
   // split over several warps (or a gate/up pair) are summed in shared memory
   // and the last warp to add finishes the row.
   __device__ __forceinline__ void gemv_phase(int ph, int layer, int a, int b, int K, ChunkShape cs) {
-    const int it = (K / cs.segs) / 256;
     const bool q8 = Q8W && ph != kLM;
-#define FS_GP(IT, NB)                                                     \
-  if (it == IT) {                                                         \
-    if (q8) gemv_phase_t<IT, NB, Q8W>(ph, layer, a, b, K, cs);            \
-    else gemv_phase_t<IT, NB, false>(ph, layer, a, b, K, cs);             \
-    return;                                                               \
+#define FS_GP(R)                                               \
+  if (cs.rows == R) {                                          \
+    if (q8) gemv_phase_t<NB, Q8W, R>(ph, layer, a, b, K, cs);  \
+    else gemv_phase_t<NB, false, R>(ph, layer, a, b, K, cs);   \
+    return;                                                    \
   }
-#define FS_GP_B(NB) FS_GP(1, NB) FS_GP(2, NB) FS_GP(3, NB) FS_GP(4, NB) FS_GP(6, NB) FS_GP(8, NB)
-    FS_GP_B(NB)
-#undef FS_GP_B
+    FS_GP(8) FS_GP(4) FS_GP(2) FS_GP(1)
 #undef FS_GP
-    if (lane == 0) atomicCAS(p.err, 0, kErrBounds);  // unsupported chunk shape
+    if (lane == 0) atomicCAS(p.err, 0, kErrBounds);  // a row does not fit a stage
     quit = true;
   }
 
-  template <int IT, int NBT, bool Q8>
+  // Sum of 8 per-lane values v[0..7] over the warp in 9 shuffles: each step
+  // halves the values a lane keeps. Afterwards lane l holds the total of
+  // value r(l) = 4*bit4(l) + 2*bit3(l) + bit2(l).
+  __device__ __forceinline__ float reduce8(const float (&v)[8]) {
+    const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4;
+    float a[4], c[2];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float keep = h16 ? v[r + 4] : v[r];
+      const float send = h16 ? v[r] : v[r + 4];
+      a[r] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const float keep = h8 ? a[r + 2] : a[r];
+      const float send = h8 ? a[r] : a[r + 2];
+      c[r] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    const float keep = h4 ? c[1] : c[0];
+    const float send = h4 ? c[0] : c[1];
+    float t = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    t += __shfl_xor_sync(0xffffffffu, t, 2);
+    t += __shfl_xor_sync(0xffffffffu, t, 1);
+    return t;
+  }
+
+  // A phase's weight chunks. Chunk i of the stream belongs to consumer warp
+  // i % (consumer warps), which alone waits for it, computes all of its (up
+  // to 8) rows (gate/up: 4 gate and 4 up rows) over the whole input axis and
+  // releases it; consecutive chunks are worked on by different warps at the
+  // same time. The loop walks the input axis in blocks of 256: per block a
+  // lane loads its 8 activations once (per batch row) and uses them for all 8
+  // rows, whose FMA chains interleave. The code is the same for every K.
+  template <int NBT, bool Q8, int R>
   __device__ __forceinline__ void gemv_phase_t(int ph, int layer, int a, int b, int K, ChunkShape cs) {
-    constexpr bool XREG = NBT * IT * 8 <= 64;
     const bool pair = ph == kGU;
     const int rb = Q8 ? K : 2 * K;
-    const int seg_len = K / cs.segs;
-    const int ri = warp / cs.segs, seg = warp % cs.segs;
-    const int mrow = pair ? (ri < cs.rows ? ri : ri - cs.rows) : ri;
-    const int kb = seg * seg_len + lane * 8;  // this lane's first element; then +256 per j
-    const int B = p.B;
-    float xr[XREG ? NBT : 1][XREG ? IT : 1][8];
-    if (XREG) {
-#pragma unroll
-      for (int bb = 0; bb < NBT; ++bb)
-#pragma unroll
-        for (int j = 0; j < IT; ++j) {
-          const bool ok = bb < B;
-          const float4 a0 = ok ? *reinterpret_cast<const float4*>(xs + bb * K + kb + 256 * j)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-          const float4 a1 = ok ? *reinterpret_cast<const float4*>(xs + bb * K + kb + 256 * j + 4)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-          xr[bb][j][0] = a0.x; xr[bb][j][1] = a0.y; xr[bb][j][2] = a0.z; xr[bb][j][3] = a0.w;
-          xr[bb][j][4] = a1.x; xr[bb][j][5] = a1.y; xr[bb][j][6] = a1.z; xr[bb][j][7] = a1.w;
-        }
-    }
+    const int kb = lane * 8;
+    const int my_r = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
     for (int n = a; n < b && !quit;) {
       const int e = chunk_end(p, ph, n, b, cs);
       const int nr = e - n;
-      const unsigned char* st = stage_wait();
-      const bool valid = mrow < nr && !quit;
-      float part[NBT][IT];
+      if ((int)(i % kConsumerWarps) == warp) {
+        const unsigned char* st = stage_wait();
+        const __half* sbase = reinterpret_cast<const __half*>(st + kWeightBytes);
+        // row r of the work (pairs: r < 4 gate of pair r, r >= 4 up of pair r-4)
+        // The chunk's R rows (pairs: R gate rows in v[0..R), R up rows in
+        // v[4..4+R)) are computed without branches; in a short last chunk the
+        // missing rows repeat its last row (in bounds) and their sums are dropped.
+        constexpr int NV = 8;
+        int srow[NV];
+        bool used[NV];
 #pragma unroll
-      for (int bb = 0; bb < NBT; ++bb)
-#pragma unroll
-        for (int j = 0; j < IT; ++j) part[bb][j] = 0.f;
-      if (valid) {
-        const unsigned char* row = st + ri * rb;
-        float w[IT][8];
-        if (!Q8) {
-          uint4 u[IT];
-#pragma unroll
-          for (int j = 0; j < IT; ++j) u[j] = *reinterpret_cast<const uint4*>(row + (kb + 256 * j) * 2);
-#pragma unroll
-          for (int j = 0; j < IT; ++j) {
-            w[j][0] = lo16(u[j].x); w[j][1] = hi16(u[j].x); w[j][2] = lo16(u[j].y); w[j][3] = hi16(u[j].y);
-            w[j][4] = lo16(u[j].z); w[j][5] = hi16(u[j].z); w[j][6] = lo16(u[j].w); w[j][7] = hi16(u[j].w);
+        for (int r = 0; r < NV; ++r) {
+          const int pr = (r & 3) < R ? (r & 3) : 0;
+          const int cr = pr < nr ? pr : nr - 1;
+          if (R == 8) {
+            srow[r] = r < nr ? r : nr - 1;
+            used[r] = true;
+          } else if (pair) {
+            srow[r] = r < 4 ? cr : cs.rows + cr;
+            used[r] = (r & 3) < R;
+          } else {
+            srow[r] = r < R ? (r < nr ? r : nr - 1) : 0;
+            used[r] = r < R;
           }
-        } else {
-          uint2 u[IT];
-          float sc[IT];
-          const __half* srow = reinterpret_cast<const __half*>(st + kWeightBytes) + ri * (K / 32);
-#pragma unroll
-          for (int j = 0; j < IT; ++j) {
-            u[j] = *reinterpret_cast<const uint2*>(row + kb + 256 * j);
-            sc[j] = __half2float(srow[(kb + 256 * j) / 32]);
-          }
-#pragma unroll
-          for (int j = 0; j < IT; ++j)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              w[j][q] = (float)(int8_t)((u[j].x >> (8 * q)) & 0xff) * sc[j];
-              w[j][4 + q] = (float)(int8_t)((u[j].y >> (8 * q)) & 0xff) * sc[j];
-            }
         }
+        float acc[NV][NBT];
+#pragma unroll
+        for (int r = 0; r < NV; ++r)
+#pragma unroll
+          for (int bb = 0; bb < NBT; ++bb) acc[r][bb] = 0.f;
+#pragma unroll 1
+        for (int k0 = kb; k0 < K; k0 += 256) {
+          float x8[NBT][8];
+#pragma unroll
+          for (int bb = 0; bb < NBT; ++bb) {
+            if (bb < p.B) {
+              const float4 a0 = *reinterpret_cast<const float4*>(xs + bb * K + k0);
+              const float4 a1 = *reinterpret_cast<const float4*>(xs + bb * K + k0 + 4);
+              x8[bb][0] = a0.x; x8[bb][1] = a0.y; x8[bb][2] = a0.z; x8[bb][3] = a0.w;
+              x8[bb][4] = a1.x; x8[bb][5] = a1.y; x8[bb][6] = a1.z; x8[bb][7] = a1.w;
+            } else {
+#pragma unroll
+              for (int q = 0; q < 8; ++q) x8[bb][q] = 0.f;
+            }
+          }
+#pragma unroll
+          for (int r = 0; r < NV; ++r) {
+            if (!used[r]) continue;  // compile-time for a given R and phase kind
+            float w[8];
+            if (!Q8) {
+              const uint4 u = *reinterpret_cast<const uint4*>(st + srow[r] * rb + k0 * 2);
+              w[0] = lo16(u.x); w[1] = hi16(u.x); w[2] = lo16(u.y); w[3] = hi16(u.y);
+              w[4] = lo16(u.z); w[5] = hi16(u.z); w[6] = lo16(u.w); w[7] = hi16(u.w);
+            } else {
+              const uint2 u = *reinterpret_cast<const uint2*>(st + srow[r] * rb + k0);
+              const float sc = __half2float(sbase[srow[r] * (K / 32) + k0 / 32]);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                w[q] = (float)(int8_t)((u.x >> (8 * q)) & 0xff) * sc;
+                w[4 + q] = (float)(int8_t)((u.y >> (8 * q)) & 0xff) * sc;
+              }
+            }
+#pragma unroll
+            for (int bb = 0; bb < NBT; ++bb)
+#pragma unroll
+              for (int q = 0; q < 8; ++q) acc[r][bb] = fmaf(w[q], x8[bb][q], acc[r][bb]);
+          }
+        }
+        stage_release();
+        float tot[NBT], up[NBT];
 #pragma unroll
         for (int bb = 0; bb < NBT; ++bb) {
-          if (bb >= B) break;
+          float col[8];
 #pragma unroll
-          for (int j = 0; j < IT; ++j) {
-            float x8[8];
-            if (XREG) {
+          for (int r = 0; r < 8; ++r) col[r] = acc[r][bb];
+          tot[bb] = reduce8(col);
+          up[bb] = pair ? __shfl_xor_sync(0xffffffffu, tot[bb], 16) : 0.f;
+        }
+        const bool mine = (lane & 3) == 0 && (pair ? my_r < 4 : true) && my_r < nr && !quit;
+        if (mine) {
 #pragma unroll
-              for (int q = 0; q < 8; ++q) x8[q] = xr[XREG ? bb : 0][XREG ? j : 0][q];
-            } else {
-              const float4 a0 = *reinterpret_cast<const float4*>(xs + bb * K + kb + 256 * j);
-              const float4 a1 = *reinterpret_cast<const float4*>(xs + bb * K + kb + 256 * j + 4);
-              x8[0] = a0.x; x8[1] = a0.y; x8[2] = a0.z; x8[3] = a0.w;
-              x8[4] = a1.x; x8[5] = a1.y; x8[6] = a1.z; x8[7] = a1.w;
-            }
-            float acc = w[j][0] * x8[0];
-#pragma unroll
-            for (int q = 1; q < 8; ++q) acc = fmaf(w[j][q], x8[q], acc);
-            part[bb][j] = acc;
-          }
+          for (int bb = 0; bb < NBT; ++bb)
+            if (bb < p.B) epilogue(ph, layer, n + my_r, bb, tot[bb], up[bb]);
         }
       }
-      // Sum over the warp; lane b keeps the total of batch row b.
-      float mine = 0.f;
-#pragma unroll
-      for (int bb = 0; bb < NBT; ++bb) {
-        if (bb >= B) break;
-        float t = 0.f;
-#pragma unroll
-        for (int j = 0; j < IT; ++j) t += part[bb][j];
-        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-        if (lane == bb) mine = t;
-      }
-      const int slot = stage;
-      if (valid) {
-        const int need = cs.segs * (pair ? 2 : 1);
-        bool finish = need == 1;
-        float y = mine, u = 0.f;
-        if (!finish) {
-          float* cb = comb + ((slot * kConsumerWarps + mrow) * 2) * kMaxB;
-          if (lane < B) atomicAdd(cb + (pair && ri >= cs.rows ? kMaxB : 0) + lane, mine);
-          __syncwarp();
-          __threadfence_block();
-          int last = 0;
-          if (lane == 0) last = atomicAdd(ccnt + slot * kConsumerWarps + mrow, 1) == need - 1;
-          finish = __shfl_sync(0xffffffffu, last, 0) != 0;
-          if (finish) {
-            __threadfence_block();
-            if (lane < B) {
-              y = cb[lane];
-              u = cb[kMaxB + lane];
-              cb[lane] = 0.f;
-              cb[kMaxB + lane] = 0.f;
-            }
-            if (lane == 0) ccnt[slot * kConsumerWarps + mrow] = 0;
-          }
-        }
-        if (finish && lane < B) epilogue(ph, layer, n + mrow, lane, y, u);
-      }
-      stage_release();
       advance();
       n = e;
     }
+    if (p.trace && tid == 0 && (ph == kQKV || ph == kLM))
+      p.trace[((size_t)cta * (p.L + 1) + (ph == kLM ? p.L : layer)) * 16 + 8 + ph] = now_ns();
   }
 
   // Output of row n for batch row b (y = the dot product; u = the up row's
@@ -831,7 +894,9 @@ struct Consumer {
           const uint32_t ord = (uu & 0x80000000u) ? ~uu : (uu | 0x80000000u);
           const unsigned long long key =
               ((unsigned long long)ord << 32) | (0xffffffffu - (uint32_t)n);
-          if (key > wbest) wbest = key;
+#pragma unroll
+          for (int bb = 0; bb < kMaxB; ++bb)
+            if (bb == b && key > wbest[bb]) wbest[bb] = key;
         }
         break;
       }
@@ -846,8 +911,28 @@ struct Consumer {
   __device__ float* ml_s() { return v_s() + p.d; }
   __device__ float* acc_s() { return ml_s() + kConsumerWarps * (p.nq / p.nkv) * 2; }
 
-  // RMSNorm over one head in a warp + rotate-half RoPE at pos, in place.
-  __device__ __forceinline__ void head_norm_rope(float* x, const __nv_bfloat16* gain, int pos) {
+  // Per-lane constants of a head's RMSNorm + RoPE: gains of the lane's
+  // elements of both halves and cos/sin at pos. Loaded before the wait for the
+  // head's values, so their latency overlaps it.
+  struct HeadConst {
+    float g_lo[2], g_hi[2];
+    float2 cs[2];
+  };
+  __device__ __forceinline__ void head_const(const __nv_bfloat16* gain, int pos, HeadConst& hc) {
+    const int d = p.d, half = d / 2, E = d / 64;
+    const float2* rp = p.rope + (size_t)pos * half;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int i = lane * E + e;
+      const bool ok = e < E;
+      hc.g_lo[e] = ok ? __bfloat162float(gain[i]) : 0.f;
+      hc.g_hi[e] = ok ? __bfloat162float(gain[half + i]) : 0.f;
+      hc.cs[e] = ok ? rp[i] : make_float2(0.f, 0.f);
+    }
+  }
+
+  // RMSNorm over one head in a warp + rotate-half RoPE, in place.
+  __device__ __forceinline__ void head_norm_rope(float* x, const HeadConst& hc) {
     const int d = p.d, half = d / 2;
     const int E = d / 64;  // elements per lane per half
     float lo[2] = {0.f, 0.f}, hi[2] = {0.f, 0.f}, ss = 0.f;
@@ -861,16 +946,14 @@ struct Consumer {
     }
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float inv = rsqrtf(ss / (float)d + p.eps);
-    const float2* cs = p.rope + (size_t)pos * half;
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       if (e >= E) break;
       const int i = lane * E + e;
-      const float a = lo[e] * inv * __bfloat162float(gain[i]);
-      const float c = hi[e] * inv * __bfloat162float(gain[half + i]);
-      const float2 t = cs[i];
-      x[i] = a * t.x - c * t.y;
-      x[half + i] = c * t.x + a * t.y;
+      const float a = lo[e] * inv * hc.g_lo[e];
+      const float c = hi[e] * inv * hc.g_hi[e];
+      x[i] = a * hc.cs[e].x - c * hc.cs[e].y;
+      x[half + i] = c * hc.cs[e].x + a * hc.cs[e].y;
     }
   }
 
@@ -878,9 +961,15 @@ struct Consumer {
     // The QKV chunks before this end on no barrier: decide quit CTA-wide first.
     quit = consumer_sync_or(quit);
     if (quit) return;
+    tr(layer, 12);
     const int d = p.d, rep = p.nq / p.nkv, qd = p.nq * d, kvd = p.nkv * d;
     const unsigned long long* row = p.xq + (size_t)x.b * (qd + 2 * kvd);
     const uint32_t t1 = tag(layer, 1);
+    const LayerDev& Lw = layers_s(p)[layer];
+    const int pos = p.pos[x.b];
+    HeadConst hc;
+    if (warp < rep) head_const(Lw.q_norm, pos, hc);
+    if (x.owner && warp == rep) head_const(Lw.k_norm, pos, hc);
     wait_words(row + x.g * rep * d, rep * d, t1, q_s());
     if (x.owner) {
       wait_words(row + qd + x.g * d, d, t1, k_s());
@@ -889,12 +978,10 @@ struct Consumer {
     quit = consumer_sync_or(quit);
     if (quit) return;
     tr(layer, 2);
-    const LayerDev& Lw = p.layers[layer];
-    const int pos = p.pos[x.b];
-    if (warp < rep) head_norm_rope(q_s() + warp * d, Lw.q_norm, pos);
+    if (warp < rep) head_norm_rope(q_s() + warp * d, hc);
     if (x.owner && warp == rep) {
-      head_norm_rope(k_s(), Lw.k_norm, pos);
-      const size_t off = p.kv.offset(layer, p.seq[x.b], pos, x.g);
+      head_norm_rope(k_s(), hc);
+      const size_t off = kv_off(p, layer, x.b, pos, x.g);
       for (int i2 = lane; i2 < d; i2 += 32) {
         const __nv_bfloat16 kb = __float2bfloat16_rn(k_s()[i2]);
         const __nv_bfloat16 vb = __float2bfloat16_rn(v_s()[i2]);
@@ -938,7 +1025,7 @@ struct Consumer {
   }
 
   __device__ __forceinline__ void kv(int, const Item&, int, int nk) {
-    if (quit) return;  // no barrier in here: a per-thread exit is harmless
+    // Contains a CTA barrier: no early exit; a thread that gave up skips the work.
     const unsigned char* st = stage_wait();
     const int d = p.d, rep = p.nq / p.nkv, E = d / 32;
     const __nv_bfloat16* K = reinterpret_cast<const __nv_bfloat16*>(st);
@@ -958,7 +1045,10 @@ struct Consumer {
       }
       attend(kk, vv, rep);
     }
-    stage_release();
+    // Every consumer warp reads a KV chunk; the stage is released once, after
+    // all of them are done with it.
+    quit = consumer_sync_or(quit);
+    if (tid == 0) mbar_arrive(&r.empty[stage]);
     advance();
   }
 
@@ -1047,6 +1137,7 @@ struct Consumer {
       }
     }
     quit = consumer_sync_or(quit);
+    tr(layer, 9);
   }
 
   __device__ void end_layer() {
@@ -1059,7 +1150,15 @@ struct Consumer {
   // End of the step: fold this CTA's greedy keys; the last CTA writes ids.
   __device__ __forceinline__ void finish_head() {
     if (!p.run_head) return;
-    if (lane < p.B && wbest) atomicMax(best + lane, wbest);
+#pragma unroll
+    for (int bb = 0; bb < kMaxB; ++bb) {
+      unsigned long long k = wbest[bb];
+      for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long other = __shfl_xor_sync(0xffffffffu, k, o);
+        k = other > k ? other : k;
+      }
+      if (lane == 0 && bb < p.B && k) atomicMax(best + bb, k);
+    }
     quit = consumer_sync_or(quit);
     tr(p.L, 7);
     if (tid < p.B && !quit) atomicMax(p.am_key + tid, best[tid]);
@@ -1098,11 +1197,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mega_kernel(const __grid_c
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.n_stages; ++s) {
       mbar_init(&ring.full[s], 1);
-      mbar_init(&ring.empty[s], kConsumerWarps);
+      mbar_init(&ring.empty[s], 1);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     unsigned long long* best = reinterpret_cast<unsigned long long*>(smem + p.off_misc);
     for (int b = 0; b < kMaxB; ++b) best[b] = 0ull;
+  }
+  {
+    const unsigned* src = reinterpret_cast<const unsigned*>(p.layers);
+    unsigned* dst = reinterpret_cast<unsigned*>(smem + p.off_tab);
+    const int words = p.L * (int)sizeof(LayerDev) / 4;
+    for (int k = threadIdx.x; k < words; k += blockDim.x) dst[k] = src[k];
+    if (p.bt_in_smem) {
+      int32_t* bt = reinterpret_cast<int32_t*>(smem + p.off_tab + (size_t)p.L * sizeof(LayerDev));
+      const int pps = p.kv.pages_per_seq;
+      for (int k = threadIdx.x; k < p.B * pps; k += blockDim.x)
+        bt[k] = p.kv.block_table[(size_t)p.seq[k / pps] * pps + k % pps];
+    }
   }
   {
     float* cz = reinterpret_cast<float*>(smem + p.off_red);
@@ -1116,7 +1227,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mega_kernel(const __grid_c
     if ((threadIdx.x & 31) == 0) {
       Producer pr(p, ring);
       walk(p, blockIdx.x, gridDim.x, pr);
-      if (p.trace) p.trace[((size_t)blockIdx.x * (p.L + 1) + p.L) * 8 + 3] = now_ns();
+      if (p.trace) p.trace[((size_t)blockIdx.x * (p.L + 1) + p.L) * 16 + 3] = now_ns();
       reinterpret_cast<volatile unsigned int*>(smem + p.off_misc + 8 * kMaxB + 8)[0] = pr.i;
     }
   } else {
@@ -1167,21 +1278,29 @@ struct MegaState {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Keys per attention item of a decode step (the items of a kv head are merged
+// by the last one to finish).
+int kKeysPerSplit = 64;
+
 }  // namespace
 
 bool mega_shape_ok(const fs_model* m) {
   const Shape& s = m->s;
   const int rep = s.nq / s.nkv;
   if (rep > 2 || (s.d != 64 && s.d != 128)) return false;
-  if (s.V >= 0x7fffffff) return false;
-  const int Ks[4] = {s.H, s.q_dim(), s.H, s.I};
-  const bool pair[4] = {false, false, true, false};
-  for (int i = 0; i < 4; ++i) {
-    const mega::ChunkShape cs = mega::chunk_shape(Ks[i], m->q8, pair[i]);
-    if ((Ks[i] / cs.segs) % 256 || Ks[i] % cs.segs) return false;
-  }
-  const mega::ChunkShape lm = mega::chunk_shape(s.H, false, false);
-  if ((s.H / lm.segs) % 256) return false;
+  if (s.V >= 0x7fffffff || s.H > 2048) return false;
+  auto it_ok = [](int K) {
+    if (K % 256) return false;
+    const int it = K / 256;
+    return it == 1 || it == 2 || it == 3 || it == 4 || it == 6 || it == 8 || it == 12;
+  };
+  const int Ks[3] = {s.H, s.q_dim(), s.I};
+  for (int K : Ks)
+    if (!it_ok(K)) return false;
+  // every phase needs at least one whole row (pair) per stage
+  if (mega::chunk_shape(s.I, m->q8, false).rows < 1 || mega::chunk_shape(s.H, m->q8, true).rows < 1 ||
+      mega::chunk_shape(s.q_dim(), m->q8, false).rows < 1)
+    return false;
   return true;
 }
 
@@ -1294,7 +1413,7 @@ fs_status decode_mega(fs_model* m, const fs_kv* kv, const RowMap& map, int B, co
   p.am_key = st->am_key;
   p.am_cnt = st->am_cnt;
   // ~64 keys per attention item, at most one item per CTA
-  int ns = (cmax + 63) / 64;
+  int ns = (cmax + kKeysPerSplit - 1) / kKeysPerSplit;
   ns = std::max(1, std::min(ns, std::min(st->max_splits, st->sms / (B * s.nkv))));
   p.n_splits = ns;
   p.l0 = l0;
@@ -1335,7 +1454,10 @@ fs_status decode_mega(fs_model* m, const fs_kv* kv, const RowMap& map, int B, co
       align_up((size_t)mega::kMaxStages * mega::kConsumerWarps * (2 * mega::kMaxB + 1) * 4, 128);
   const size_t bars = 2 * mega::kMaxStages * 8;
   const size_t misc = 128;
-  const size_t fixed = fixed_hs + fixed_xs + attn + redb + bars + misc;
+  const size_t bt_bytes = (size_t)B * kv->pages_per_seq * sizeof(int32_t);
+  const bool bt_smem = bt_bytes <= 8192;
+  const size_t tab = align_up((size_t)s.L * sizeof(LayerDev) + (bt_smem ? bt_bytes : 0), 128);
+  const size_t fixed = fixed_hs + fixed_xs + attn + redb + bars + misc + tab;
   const size_t budget = 232448;
   int n_stages = (int)((budget - fixed) / mega::kStageBytes);
   n_stages = std::min(n_stages, mega::kMaxStages);
@@ -1347,6 +1469,8 @@ fs_status decode_mega(fs_model* m, const fs_kv* kv, const RowMap& map, int B, co
   p.off_red = (int)off; off += redb;
   p.off_bar = (int)off; off += bars;
   p.off_misc = (int)off; off += misc;
+  p.off_tab = (int)off; off += tab;
+  p.bt_in_smem = bt_smem ? 1 : 0;
   p.n_stages = n_stages;
   void* args[] = {&p};
   count_launches();

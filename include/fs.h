@@ -224,11 +224,14 @@ fs_status fs_debug_block(fs_model* model, fs_kv* kv, int32_t seq, int32_t layer,
 
 /* Debug: the next decode step that runs on the persistent decode kernel
  * records %globaltimer stamps (ns) into `buf` (device uint64
- * [SMs][n_layers+1][8]): per CTA and layer, slot 0 phase start, 1 block input
- * ready, 2 attention input ready, 3 O start, 4 O input ready, 5 MLP input
- * ready, 6 down input ready, 7 layer done; row n_layers holds the LM head
- * (0 start, 1 input ready, 7 done). Slots a CTA never reaches are left as
- * they were. One-shot; NULL disarms. Timing only: no work changes. */
+ * [SMs][n_layers+1][16]): per CTA and layer, slot 0 phase start, 1 block
+ * input ready, 2 attention input ready, 3 O start, 4 O input ready, 5 MLP
+ * input ready, 6 down input ready, 7 layer done, 8 warp 0's QKV rows done, 9
+ * attention item done, 10 O rows done by every warp, 11 gate/up rows done by
+ * every warp, 12 attention item start; row n_layers holds the LM head (0
+ * start, 1 input ready, 2 and 3 first and last weight copy issued, 13 warp
+ * 0's rows done, 7 done). Slots a CTA never reaches are
+ * left as they were. One-shot; NULL disarms. Timing only: no work changes. */
 fs_status fs_debug_trace(fs_model* model, uint64_t* buf);
 
 /* Debug: dequantise Q8_0 blocks to fp32, out[n*k] = codes[n*k] * scales[n*(k/32)]
