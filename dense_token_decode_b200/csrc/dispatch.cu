@@ -7,7 +7,10 @@ namespace fs {
 
 fs_status init_extras(fs_model* m) { return mega_init(m); }
 
-void release_extras(fs_model* m) { mega_release(m); }
+void release_extras(fs_model* m) {
+  mega_release(m);
+  tc_release(m);
+}
 
 fs_status ensure_gen_buffer(fs_model* m, int n) {
   if (n <= m->gen_cap) return FS_OK;
@@ -23,15 +26,18 @@ fs_status ensure_gen_buffer(fs_model* m, int n) {
   return FS_OK;
 }
 
+// Chunks of at least 128 rows run their GEMMs on the tensor cores.
 fs_status prefill_chunk(fs_model* m, const fs_kv* kv, const RowMap& map, int rows,
                         const int32_t* tok, int head_first, float* logits, int32_t* argmax,
                         int capture_row0, int capture_rows, cudaStream_t st) {
+  const bool tc = rows >= kTcMinRows && tc_available(m, st);
   return forward_general(m, kv, map, rows, tok, head_first, logits, argmax, capture_row0,
-                         capture_rows, st);
+                         capture_rows, st, tc);
 }
 
 fs_status block_prefill_or_general(fs_model* m, const fs_kv* kv, const RowMap& map, int rows,
                                    int l, cudaStream_t st) {
+  if (rows >= kTcMinRows && tc_available(m, st)) return layer_tc(m, kv, map, rows, l, st);
   return layer_general(m, kv, map, rows, l, st);
 }
 

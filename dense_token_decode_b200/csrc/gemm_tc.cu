@@ -1,0 +1,428 @@
+// Tensor-core GEMM of the prefill path on sm_100a (tcgen05 + TMEM + TMA):
+//   D[m, n] = sum_k A[m, k] * B[n, k]
+// A: activations fp16 [M, K] (optionally two fp16 terms, A = A_hi + A_lo),
+// B: weights fp16 [N, K] (the model's fp16 copy), both K-contiguous.
+// Tiles of 128 (M) x 128 (N) with 64-wide K blocks; fp32 accumulators live in
+// tensor memory, two buffers, so the epilogue of one tile runs while the
+// next tile's MMAs are issued.
+//
+// Warp roles in a CTA of 192 threads (one CTA per SM, persistent over tiles):
+//   warp 0: TMA producer (one lane) — A (and A_lo) and B blocks into a ring of
+//           shared-memory stages with 128-byte swizzle;
+//   warp 1: allocates TMEM, then one lane issues tcgen05.mma (M=128, N=128,
+//           K=16 per instruction) and tcgen05.commit to release stages and
+//           to hand finished accumulators to the epilogue;
+//   warps 2-5: epilogue — tcgen05.ld of their 32 TMEM lanes (= tile rows),
+//           then the fused output step of the GEMM kind.
+//
+// Every wait is bounded (%globaltimer); a timeout sets the error word and the
+// CTA drains and frees TMEM before it returns.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "runtime.h"
+
+namespace fs {
+namespace tc {
+
+constexpr int BM = 128, BN = 128, BK = 64;
+constexpr int kThreads = 192;
+constexpr int kTileBytes = BM * BK * 2;  // 16 KB for a 128 x 64 fp16 tile
+constexpr unsigned long long kTimeoutNs = 2000000000ull;
+
+enum Kind { kStore = 0, kResidual = 1, kSwiGLU = 2 };
+
+struct Params {
+  int M, N, K;       // N = output columns of D (SwiGLU: 2 x act columns per tile)
+  int kind;
+  int a_terms;       // 1 or 2
+  int n_tiles_m, n_tiles_n;
+  int stages;
+  float* out;        // kStore: fp32 [M, ldo]; kResidual: fp32 [M, ldo] (+=)
+  int ldo;
+  __half* act_hi;    // kSwiGLU: fp16 [M, I] outputs (hi and lo terms)
+  __half* act_lo;
+  int act_ld;
+  int* err;
+};
+
+__device__ __forceinline__ uint32_t su32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ unsigned long long now_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(su32(bar)), "r"(parity), "r"(1000000)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait; false on timeout (the error word is set).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
+  unsigned long long t0 = 0;
+  int spins = 0;
+  while (!mbar_try(bar, parity)) {
+    if ((++spins & 15) == 0) {
+      if (t0 == 0) t0 = now_ns();
+      if (*reinterpret_cast<volatile int*>(err) == kErrTimeout || now_ns() - t0 > kTimeoutNs) {
+        atomicCAS(err, 0, kErrTimeout);
+        return false;
+      }
+    }
+  }
+  return true;
+}
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(su32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(su32(bar))
+      : "memory");
+}
+// Shared-memory matrix descriptor of a K-major tile with 128-byte swizzle:
+// rows of 128 bytes, 8-row groups 1024 bytes apart (stride byte offset).
+__device__ __forceinline__ uint64_t smem_desc(const void* p) {
+  const uint64_t addr = su32(p);
+  uint64_t d = 0;
+  d |= (addr >> 4) & 0x3FFFull;        // start address
+  d |= 1ull << 16;                      // leading byte offset (unused with swizzle)
+  d |= (uint64_t)(1024 >> 4) << 32;     // stride byte offset
+  d |= 1ull << 46;                      // descriptor version for tcgen05
+  d |= 2ull << 61;                      // 128-byte swizzle
+  return d;
+}
+// Instruction descriptor: D fp32, A and B fp16, both K-major, M x N.
+__host__ __device__ constexpr uint32_t instr_desc(int m, int n) {
+  return (1u << 4)                    // D format: f32
+         | (0u << 7) | (0u << 10)     // A, B format: f16
+         | (0u << 15) | (0u << 16)    // A, B K-major
+         | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          su32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap map_a,
+                   const __grid_constant__ CUtensorMap map_a_lo,
+                   const __grid_constant__ CUtensorMap map_b,
+                   const __grid_constant__ CUtensorMap map_b2) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // 1024-byte aligned base for the swizzled tiles
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int S = p.stages;
+  const int stage_bytes = (p.a_terms + 1) * kTileBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * stage_bytes);
+  uint64_t* empty = full + S;
+  uint64_t* acc_full = empty + S;   // [2]
+  uint64_t* acc_empty = acc_full + 2;  // [2]
+  uint64_t* drain = acc_empty + 2;  // MMA completion before TMEM is freed
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(drain + 1);
+  uint32_t* counts = tmem_base_s + 1;  // [0] stages loaded, [1] stages consumed
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4);
+    }
+    mbar_init(drain, 1);
+    counts[0] = counts[1] = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     su32(tmem_base_s)),
+                 "r"(2 * BN)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tmem_base_s;
+
+  const int n_tiles = p.n_tiles_m * p.n_tiles_n;
+  const int kblocks = p.K / BK;
+  const bool swiglu = p.kind == kSwiGLU;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        const int mt = t % p.n_tiles_m, nt = t / p.n_tiles_m;
+        for (int kb = 0; kb < kblocks && ok; ++kb) {
+          ok = mbar_wait(&empty[s], ph ^ 1, p.err);
+          if (!ok) break;
+          unsigned char* st = smem + s * stage_bytes;
+          mbar_expect_tx(&full[s], stage_bytes);
+          tma_load_2d(st, &map_a, kb * BK, mt * BM, &full[s]);
+          if (p.a_terms == 2) tma_load_2d(st + kTileBytes, &map_a_lo, kb * BK, mt * BM, &full[s]);
+          unsigned char* sb = st + p.a_terms * kTileBytes;
+          if (swiglu) {
+            // 64 gate rows then 64 up rows of the same act columns
+            tma_load_2d(sb, &map_b, kb * BK, nt * (BN / 2), &full[s]);
+            tma_load_2d(sb + kTileBytes / 2, &map_b2, kb * BK, nt * (BN / 2), &full[s]);
+          } else {
+            tma_load_2d(sb, &map_b, kb * BK, nt * BN, &full[s]);
+          }
+          ++counts[0];
+          if (++s == S) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = instr_desc(BM, BN);
+      int s = 0;
+      uint32_t ph = 0;
+      int tcount = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tcount) {
+        const int abuf = tcount & 1;
+        const uint32_t aph = (tcount >> 1) & 1;
+        ok = mbar_wait(&acc_empty[abuf], aph ^ 1, p.err);
+        if (!ok) break;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t d_tmem = tmem + abuf * BN;
+        for (int kb = 0; kb < kblocks && ok; ++kb) {
+          ok = mbar_wait(&full[s], ph, p.err);
+          if (!ok) break;
+          asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+          unsigned char* st = smem + s * stage_bytes;
+          const unsigned char* sb = st + p.a_terms * kTileBytes;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t bdesc = smem_desc(sb + k * 32);
+            mma_f16(d_tmem, smem_desc(st + k * 32), bdesc, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+            if (p.a_terms == 2) mma_f16(d_tmem, smem_desc(st + kTileBytes + k * 32), bdesc, idesc, 1u);
+          }
+          mma_commit(&empty[s]);  // the stage is free once these MMAs have read it
+          ++counts[1];
+          if (++s == S) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        mma_commit(&acc_full[abuf]);  // accumulator complete
+      }
+      // Every MMA this thread issued has finished before TMEM is released.
+      mma_commit(drain);
+      const unsigned long long t0 = now_ns();
+      while (!mbar_try(drain, 0))
+        if (now_ns() - t0 > kTimeoutNs) break;
+    }
+  } else {
+    // epilogue warps 2..5: TMEM lane quadrant = warp % 4
+    const int quad = warp & 3;
+    const int row_in_tile = quad * 32 + lane;
+    int tcount = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tcount) {
+      const int mt = t % p.n_tiles_m, nt = t / p.n_tiles_m;
+      const int abuf = tcount & 1;
+      const uint32_t aph = (tcount >> 1) & 1;
+      if (!mbar_wait(&acc_full[abuf], aph, p.err)) break;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + abuf * BN;
+      const int m = mt * BM + row_in_tile;
+      const bool live = m < p.M;
+      if (!swiglu) {
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(taddr + c0, r);
+          if (!live) continue;
+          float* o = p.out + (size_t)m * p.ldo + nt * BN + c0;
+          if (p.kind == kResidual) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              float4 h = *reinterpret_cast<float4*>(o + j);
+              h.x += __uint_as_float(r[j]);
+              h.y += __uint_as_float(r[j + 1]);
+              h.z += __uint_as_float(r[j + 2]);
+              h.w += __uint_as_float(r[j + 3]);
+              *reinterpret_cast<float4*>(o + j) = h;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+              *reinterpret_cast<float4*>(o + j) =
+                  make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                              __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+          }
+        }
+      } else {
+        // columns [0, 64) gate, [64, 128) up of act columns nt*64 + c
+        for (int c0 = 0; c0 < BN / 2; c0 += 32) {
+          uint32_t g[32], u[32];
+          tmem_ld32(taddr + c0, g);
+          tmem_ld32(taddr + BN / 2 + c0, u);
+          if (!live) continue;
+          const size_t off = (size_t)m * p.act_ld + nt * (BN / 2) + c0;
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            __align__(16) __half hi[8], lo[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float gv = __uint_as_float(g[j + q]), uv = __uint_as_float(u[j + q]);
+              const float a = gv / (1.f + expf(-gv)) * uv;
+              hi[q] = __float2half_rn(a);
+              lo[q] = __float2half_rn(a - __half2float(hi[q]));
+            }
+            *reinterpret_cast<uint4*>(p.act_hi + off + j) = *reinterpret_cast<uint4*>(hi);
+            if (p.act_lo) *reinterpret_cast<uint4*>(p.act_lo + off + j) = *reinterpret_cast<uint4*>(lo);
+          }
+        }
+      }
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[abuf]);
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  // After a timeout: stages loaded but never consumed must land before the
+  // CTA's shared memory is released (bounded wait, 10 ms each).
+  if (threadIdx.x == 0 && counts[0] > counts[1]) {
+    for (uint32_t k = counts[1]; k < counts[0]; ++k) {
+      const unsigned long long t0 = now_ns();
+      while (!mbar_try(&full[k % S], (k / S) & 1))
+        if (now_ns() - t0 > 10000000ull) break;
+    }
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * BN)
+                 : "memory");
+  }
+}
+
+}  // namespace tc
+
+// ---------------------------------------------------------------------------
+// Host side
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+// 2-D fp16 tensor map over rows x cols (cols contiguous), box of box_rows x 64
+// columns with 128-byte swizzle. Returns false if the driver refuses it.
+bool make_tmap_f16(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)tc::BK, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Launch one tensor-core GEMM. a_lo may be null (one fp16 term). For kSwiGLU
+// b2 is the up matrix and N counts gate+up columns per tile pair (2 * I).
+cudaError_t launch_gemm_tc(const CUtensorMap* a, const CUtensorMap* a_lo, const CUtensorMap* b,
+                           const CUtensorMap* b2, int M, int N, int K, int kind, float* out,
+                           int ldo, __half* act_hi, __half* act_lo, int act_ld, int* err,
+                           int num_sms, cudaStream_t st) {
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaFuncSetAttribute(tc::gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+    attr_done = true;
+  }
+  tc::Params p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.kind = kind;
+  p.a_terms = a_lo ? 2 : 1;
+  p.n_tiles_m = (M + tc::BM - 1) / tc::BM;
+  p.n_tiles_n = N / tc::BN;
+  const int stage_bytes = (p.a_terms + 1) * tc::kTileBytes;
+  p.stages = std::min(8, (232448 - 2048) / stage_bytes);
+  p.out = out;
+  p.ldo = ldo;
+  p.act_hi = act_hi;
+  p.act_lo = act_lo;
+  p.act_ld = act_ld;
+  p.err = err;
+  const size_t smem = 1024 + (size_t)p.stages * stage_bytes + 1024;
+  const int tiles = p.n_tiles_m * p.n_tiles_n;
+  const int grid = std::min(tiles, num_sms);
+  count_launches();
+  tc::gemm_tc_kernel<<<grid, tc::kThreads, smem, st>>>(p, *a, a_lo ? *a_lo : *a, *b, b2 ? *b2 : *b);
+  return cudaGetLastError();
+}
+
+}  // namespace fs

@@ -392,7 +392,7 @@ fs_status layer_general(fs_model* m, const fs_kv* kv, const RowMap& map, int row
 // head_first .. rows-1 (prefill: the last row; decode: every row).
 fs_status forward_general(fs_model* m, const fs_kv* kv, const RowMap& map, int rows,
                           const int32_t* tok, int head_first, float* logits, int32_t* argmax,
-                          int capture_row0, int capture_rows, cudaStream_t st) {
+                          int capture_row0, int capture_rows, cudaStream_t st, bool tensor_cores) {
   (void)capture_rows;
   const Shape& s = m->s;
   const int H = s.H;
@@ -406,7 +406,8 @@ fs_status forward_general(fs_model* m, const fs_kv* kv, const RowMap& map, int r
   };
   FS_CUDA(capture(0));
   for (int l = 0; l < s.L; ++l) {
-    fs_status ls = layer_general(m, kv, map, rows, l, st);
+    fs_status ls = tensor_cores ? layer_tc(m, kv, map, rows, l, st)
+                                : layer_general(m, kv, map, rows, l, st);
     if (ls != FS_OK) return ls;
     FS_CUDA(capture(l + 1));
   }

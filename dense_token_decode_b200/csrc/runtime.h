@@ -38,7 +38,8 @@ struct fs_model {
   int capture_max_rows = 0;
   int prefill_split = 1;
   unsigned long long* trace = nullptr;  // armed fs_debug_trace buffer
-  void* extras = nullptr;     // fast-path state
+  void* extras = nullptr;     // persistent decode kernel state
+  void* tc_extras = nullptr;  // tensor-core prefill state
 };
 
 struct fs_kv {
@@ -67,7 +68,8 @@ fs_status ensure_gen_buffer(fs_model* m, int n);
 // The unfused general forward (any rows): see runtime.cu.
 fs_status forward_general(fs_model* m, const fs_kv* kv, const RowMap& map, int rows,
                           const int32_t* tok, int head_first, float* logits, int32_t* argmax,
-                          int capture_row0, int capture_rows, cudaStream_t st);
+                          int capture_row0, int capture_rows, cudaStream_t st,
+                          bool tensor_cores = false);
 
 // One prefill chunk (consecutive positions of one sequence).
 fs_status prefill_chunk(fs_model* m, const fs_kv* kv, const RowMap& map, int rows,
@@ -85,6 +87,14 @@ void mega_reset(fs_model* m);
 fs_status decode_mega(fs_model* m, const fs_kv* kv, const RowMap& map, int B, const int32_t* tok,
                       const float* h_in, float* h_out, int l0, int l1, bool run_head,
                       float* logits, int32_t* argmax, cudaStream_t stream);
+
+// Tensor-core prefill (prefill_tc.cu): available for this model (prepares
+// the fp16 weights on first use), one block on m->h, release.
+bool tc_available(fs_model* m, cudaStream_t st);
+fs_status layer_tc(fs_model* m, const fs_kv* kv, const RowMap& map, int rows, int l,
+                   cudaStream_t st);
+void tc_release(fs_model* m);
+constexpr int kTcMinRows = 128;
 
 // One block of the general path on m->h (rows described by map).
 fs_status layer_general(fs_model* m, const fs_kv* kv, const RowMap& map, int rows, int l,
