@@ -17,11 +17,10 @@
 //
 // Every wait is bounded (%globaltimer); a timeout sets the error word and the
 // CTA drains and frees TMEM before it returns.
-#include <cuda.h>
-
 #include <algorithm>
 
 #include "runtime.h"
+#include "tc_common.cuh"
 
 namespace fs {
 namespace tc {
@@ -29,7 +28,6 @@ namespace tc {
 constexpr int BM = 128, BN = 128, BK = 64;
 constexpr int kThreads = 192;
 constexpr int kTileBytes = BM * BK * 2;  // 16 KB for a 128 x 64 fp16 tile
-constexpr unsigned long long kTimeoutNs = 2000000000ull;
 
 enum Kind { kStore = 0, kResidual = 1, kSwiGLU = 2 };
 
@@ -46,104 +44,6 @@ struct Params {
   int act_ld;
   int* err;
 };
-
-__device__ __forceinline__ uint32_t su32(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ unsigned long long now_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(bar)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(su32(bar)), "r"(parity), "r"(1000000)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait; false on timeout (the error word is set).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
-  unsigned long long t0 = 0;
-  int spins = 0;
-  while (!mbar_try(bar, parity)) {
-    if ((++spins & 15) == 0) {
-      if (t0 == 0) t0 = now_ns();
-      if (*reinterpret_cast<volatile int*>(err) == kErrTimeout || now_ns() - t0 > kTimeoutNs) {
-        atomicCAS(err, 0, kErrTimeout);
-        return false;
-      }
-    }
-  }
-  return true;
-}
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(su32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(su32(bar))
-      : "memory");
-}
-// Shared-memory matrix descriptor of a K-major tile with 128-byte swizzle:
-// rows of 128 bytes, 8-row groups 1024 bytes apart (stride byte offset).
-__device__ __forceinline__ uint64_t smem_desc(const void* p) {
-  const uint64_t addr = su32(p);
-  uint64_t d = 0;
-  d |= (addr >> 4) & 0x3FFFull;        // start address
-  d |= 1ull << 16;                      // leading byte offset (unused with swizzle)
-  d |= (uint64_t)(1024 >> 4) << 32;     // stride byte offset
-  d |= 1ull << 46;                      // descriptor version for tcgen05
-  d |= 2ull << 61;                      // 128-byte swizzle
-  return d;
-}
-// Instruction descriptor: D fp32, A and B fp16, both K-major, M x N.
-__host__ __device__ constexpr uint32_t instr_desc(int m, int n) {
-  return (1u << 4)                    // D format: f32
-         | (0u << 7) | (0u << 10)     // A, B format: f16
-         | (0u << 15) | (0u << 16)    // A, B K-major
-         | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
-}
-__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                        uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          su32(bar))
-      : "memory");
-}
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap map_a,
@@ -376,18 +276,18 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-// 2-D fp16 tensor map over rows x cols (cols contiguous), box of box_rows x 64
-// columns with 128-byte swizzle. Returns false if the driver refuses it.
-bool make_tmap_f16(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
+bool make_tmap_16(CUtensorMap* map, const void* base, long long rows, int cols, int box_rows,
+                  bool bf16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)tc::BK, (cuuint32_t)box_rows};
+  const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+            const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Launch one tensor-core GEMM. a_lo may be null (one fp16 term). For kSwiGLU

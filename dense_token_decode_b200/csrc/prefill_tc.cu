@@ -2,7 +2,7 @@
 // copies of the weights, fp16 activation operands, TMA descriptors) and the
 // per-block kernel sequence
 //   RMSNorm -> fp16 operand (two terms when split) -> QKV GEMM (fp32 out)
-//   -> q/k head norm + RoPE + KV append -> attention -> fp16 operand
+//   -> q/k head norm + RoPE + KV append -> tensor-core attention (fp16 out)
 //   -> O GEMM (+= residual) -> RMSNorm -> fp16 operand
 //   -> gate/up GEMM with SwiGLU epilogue (fp16 act) -> down GEMM (+= residual).
 #include <cuda.h>
@@ -10,10 +10,10 @@
 #include <vector>
 
 #include "runtime.h"
+#include "tc_common.cuh"
 
 namespace fs {
 
-bool make_tmap_f16(CUtensorMap* map, const void* base, int rows, int cols, int box_rows);
 cudaError_t launch_gemm_tc(const CUtensorMap* a, const CUtensorMap* a_lo, const CUtensorMap* b,
                            const CUtensorMap* b2, int M, int N, int K, int kind, float* out,
                            int ldo, __half* act_hi, __half* act_lo, int act_ld, int* err,
@@ -168,22 +168,27 @@ static fs_status tc_prepare(fs_model* m, cudaStream_t st) {
             static_cast<const __nv_bfloat16*>(Lw.w[pt.which]), n, pt.dst);
     }
     LayerMaps& mp = t->maps[l];
-    if (!make_tmap_f16(&mp.qkv, wqkv, s.qkv_dim(), s.H, 128) ||
-        !make_tmap_f16(&mp.o, wo, s.H, s.q_dim(), 128) ||
-        !make_tmap_f16(&mp.g, wg, s.I, s.H, 64) || !make_tmap_f16(&mp.u, wu, s.I, s.H, 64) ||
-        !make_tmap_f16(&mp.d, wd, s.H, s.I, 128))
+    if (!make_tmap_16(&mp.qkv, wqkv, s.qkv_dim(), s.H, 128, false) ||
+        !make_tmap_16(&mp.o, wo, s.H, s.q_dim(), 128, false) ||
+        !make_tmap_16(&mp.g, wg, s.I, s.H, 64, false) || !make_tmap_16(&mp.u, wu, s.I, s.H, 64, false) ||
+        !make_tmap_16(&mp.d, wd, s.H, s.I, 128, false))
       return fail(FS_ERR_UNSUPPORTED, "the driver refused a TMA descriptor");
   }
-  if (!make_tmap_f16(&t->a_xn_hi, t->xn_hi, (int)R, s.H, 128) ||
-      !make_tmap_f16(&t->a_xn_lo, t->xn_lo, (int)R, s.H, 128) ||
-      !make_tmap_f16(&t->a_o, t->o_hi, (int)R, s.q_dim(), 128) ||
-      !make_tmap_f16(&t->a_act, t->act_hi, (int)R, s.I, 128))
+  if (!make_tmap_16(&t->a_xn_hi, t->xn_hi, (int)R, s.H, 128, false) ||
+      !make_tmap_16(&t->a_xn_lo, t->xn_lo, (int)R, s.H, 128, false) ||
+      !make_tmap_16(&t->a_o, t->o_hi, (int)R, s.q_dim(), 128, false) ||
+      !make_tmap_16(&t->a_act, t->act_hi, (int)R, s.I, 128, false))
     return fail(FS_ERR_UNSUPPORTED, "the driver refused a TMA descriptor");
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(FS_ERR_CUDA, "fp16 weight conversion failed");
   t->ready = true;
   return FS_OK;
 }
+
+bool attention_tc_supported(const Shape& s, const KVView& kv, const RowMap& map);
+cudaError_t launch_attention_tc(const float* q, int rows, const RowMap& map, const Shape& s,
+                                const KVView& kv, int layer, __half* o, int* err,
+                                cudaStream_t st);
 
 bool tc_available(fs_model* m, cudaStream_t st) { return tc_prepare(m, st) == FS_OK; }
 
@@ -214,11 +219,15 @@ fs_status layer_tc(fs_model* m, const fs_kv* kv, const RowMap& map, int rows, in
                         m->num_sms, st));
   FS_TRY(launch_qk_norm_rope_append(m->qkv, rows, map, s, Lw.q_norm, Lw.k_norm, m->rope, m->q,
                                     kvv, l, st));
-  FS_TRY(launch_attention_simple(m->q, rows, map, s, kvv, l, m->o, st));
-  const size_t no = (size_t)rows * s.q_dim();
-  count_launches();
-  f32_to_f16_kernel<<<grid_for(no), 256, 0, st>>>(m->o, no, t->o_hi);
-  FS_TRY(cudaGetLastError());
+  if (attention_tc_supported(s, kvv, map)) {
+    FS_TRY(launch_attention_tc(m->q, rows, map, s, kvv, l, t->o_hi, m->err, st));
+  } else {
+    FS_TRY(launch_attention_simple(m->q, rows, map, s, kvv, l, m->o, st));
+    const size_t no = (size_t)rows * s.q_dim();
+    count_launches();
+    f32_to_f16_kernel<<<grid_for(no), 256, 0, st>>>(m->o, no, t->o_hi);
+    FS_TRY(cudaGetLastError());
+  }
   FS_TRY(launch_gemm_tc(&t->a_o, nullptr, &mp.o, nullptr, rows, s.H, s.q_dim(), 1, m->h, s.H,
                         nullptr, nullptr, 0, m->err, m->num_sms, st));
   count_launches();

@@ -255,6 +255,13 @@ extern "C" fs_status fs_kv_alloc(const fs_model* m, int32_t max_seqs, int32_t ma
     fs_kv_free(kv);
     return st;
   }
+  // Attention kernels read whole pages and weight the slots past a sequence's
+  // length by exact zeros: those slots must hold finite values.
+  if (cudaMemset(kv->k, 0, elems * sizeof(__nv_bfloat16)) != cudaSuccess ||
+      cudaMemset(kv->v, 0, elems * sizeof(__nv_bfloat16)) != cudaSuccess) {
+    fs_kv_free(kv);
+    return cuda_fail(cudaGetLastError(), "KV page clear");
+  }
   // Page i of sequence s is physical page n_pages-1-(s*pps+i): the kernels
   // always go through the table, never assume contiguity.
   std::vector<int32_t> table(n_pages);

@@ -1,0 +1,181 @@
+// sm_100a building blocks shared by the tensor-core kernels: mbarriers with
+// bounded waits, TMA tile loads, shared-memory matrix descriptors,
+// tcgen05.mma / commit, and tensor-memory loads and stores.
+#pragma once
+
+#include <cuda.h>
+
+#include "fs_internal.h"
+
+namespace fs {
+namespace tc {
+
+constexpr unsigned long long kTimeoutNs = 2000000000ull;
+
+__device__ __forceinline__ uint32_t su32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ unsigned long long now_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(su32(bar)), "r"(parity), "r"(1000000)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait of one thread; false on timeout (the error word is set) or when
+// another thread of the grid has already timed out.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
+  unsigned long long t0 = 0;
+  int spins = 0;
+  while (!mbar_try(bar, parity)) {
+    if ((++spins & 15) == 0) {
+      if (t0 == 0) t0 = now_ns();
+      if (*reinterpret_cast<volatile int*>(err) == kErrTimeout || now_ns() - t0 > kTimeoutNs) {
+        atomicCAS(err, 0, kErrTimeout);
+        return false;
+      }
+    }
+  }
+  return true;
+}
+// Bounded wait of a whole warp with a warp-uniform outcome (for the
+// .sync.aligned tensor-memory instructions that follow it).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int* err) {
+  unsigned long long t0 = 0;
+  int spins = 0;
+  while (true) {
+    const bool ok = mbar_try(bar, parity);
+    if (__all_sync(0xffffffffu, ok)) return true;
+    if ((++spins & 15) == 0) {
+      if (t0 == 0) t0 = now_ns();
+      const bool late =
+          *reinterpret_cast<volatile int*>(err) == kErrTimeout || now_ns() - t0 > kTimeoutNs;
+      if (__any_sync(0xffffffffu, late)) {
+        atomicCAS(err, 0, kErrTimeout);
+        return false;
+      }
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(su32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(su32(bar))
+      : "memory");
+}
+// Shared-memory matrix descriptor, 128-byte swizzle. K-major tiles: rows of
+// 128 bytes, 8-row groups `sbo` bytes apart (lbo unused). MN-major tiles:
+// 128-byte rows hold 64 consecutive M/N elements of one k; `sbo` is the
+// distance between groups of 8 k, `lbo` between groups of 64 M/N elements.
+__device__ __forceinline__ uint64_t smem_desc(const void* p, uint32_t lbo = 16,
+                                              uint32_t sbo = 1024) {
+  const uint64_t addr = su32(p);
+  uint64_t d = 0;
+  d |= (addr >> 4) & 0x3FFFull;               // start address
+  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;  // leading byte offset
+  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;  // stride byte offset
+  d |= 1ull << 46;                             // descriptor version for tcgen05
+  d |= 2ull << 61;                             // 128-byte swizzle
+  return d;
+}
+// Instruction descriptor of kind::f16: D fp32, A and B of one 16-bit type
+// (bf16 = true: bf16, else fp16), M x N, B K-major or MN-major.
+__host__ __device__ constexpr uint32_t instr_desc(int m, int n, bool bf16 = false,
+                                                  bool b_mn_major = false) {
+  return (1u << 4)                                          // D format: f32
+         | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10)  // A, B format
+         | (0u << 15) | ((b_mn_major ? 1u : 0u) << 16)      // A K-major, B major
+         | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          su32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Generic-proxy shared-memory writes made visible to the tensor cores.
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t cols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   su32(dst_smem)),
+               "r"(cols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols)
+               : "memory");
+}
+
+}  // namespace tc
+
+// 2-D tensor map over rows x cols (cols contiguous) of a 16-bit type
+// (bf16 = true: bf16, else fp16), box of box_rows x 64 columns, 128-byte
+// swizzle. Returns false if the driver refuses it.
+bool make_tmap_16(CUtensorMap* map, const void* base, long long rows, int cols, int box_rows,
+                  bool bf16);
+
+}  // namespace fs

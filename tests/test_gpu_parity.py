@@ -249,6 +249,34 @@ def test_tiny_chunked_prefill_and_page_crossing(tiny):
             assert rel_l2(oracle_tensor(v), cache.v[l]) <= BLOCK_REL_L2
 
 
+def test_tiny_tensor_core_prefill_chunks(tiny):
+    """Chunks of >= 128 rows take the tensor-core blocks (GEMMs and attention):
+    chunks that start mid-page (positions 30 and 170), ragged query tiles
+    (140 and 130 rows), queries of one tile spanning three KV pages."""
+    toks = synth.token_ids(300, tiny.shape.vocab, seed=12).tolist()
+    rl, rh, cache = tiny.oracle.forward(toks)
+    s = tiny.shape
+    kv = tiny.model.kv(2, 320)
+    logits = torch.empty(s.vocab, device=DEV)
+    hidden = torch.zeros((s.n_layers + 1, 130, s.hidden), dtype=torch.float32, device=DEV)
+    tiny.model.prefill(kv, 1, _dev_i32(toks[:30]), None)
+    tiny.model.prefill(kv, 1, _dev_i32(toks[30:170]), None)
+    tiny.model.capture(hidden, 130)
+    tiny.model.prefill(kv, 1, _dev_i32(toks[170:]), logits)
+    torch.cuda.synchronize()
+    assert_logits_close(oracle_tensor(logits), rl, what="chunks 30/140/130")
+    assert_blocks_close(oracle_tensor(hidden), rh[:, 170:], tol=E2E_BLOCK_REL_L2,
+                        what="last chunk")
+    # end to end the cache takes the sanity bound; block-local below takes the bar
+    for l in range(s.n_layers):
+        k, v = kv.export(1, l, 0, 300)
+        assert rel_l2(oracle_tensor(k), cache.k[l]) <= E2E_BLOCK_REL_L2, l
+        assert rel_l2(oracle_tensor(v), cache.v[l]) <= E2E_BLOCK_REL_L2, l
+    # each block alone on the oracle's input, 300 rows from position 0
+    errs = blocks_local_prefill(tiny, toks, (rl, rh, cache))
+    print("tiny tensor-core block-local rel-L2:", errs)
+
+
 def test_tiny_single_token_prefill_returns_v_path(tiny):
     kv = tiny.model.kv(1, 8)
     gl, gh, _ = prefill_with_capture(tiny, kv, 0, [7])
