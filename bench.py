@@ -12,6 +12,8 @@ Also reported:
 * ``roofline``: the decode forward against HBM bandwidth (algorithmic weight +
   KV bytes per decode step / measured step time);
 * ``prefill``: a 2048-token prefill, tokens/s and TFLOP/s against bf16 peak;
+* ``batched_decode``: batch 16 with 8192 pre-filled KV positions per sequence,
+  tokens/s against HBM bandwidth (weights + KV bytes per step);
 * ``e2e``: the same job through ``fs_greedy`` with host buffers (prompt in,
   ids out, copies inside the timed region);
 * ``cpu_baseline``: the CPU oracle on a bounded sample of the same job.
@@ -238,7 +240,7 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     shape = synth.QWEN3_0P6B
     w = synth.model_weights(shape, SEED)
-    model = Model(shape, w, dev, max_pos=4096)
+    model = Model(shape, w, dev, max_pos=8192 + 256)
     del w
     kv = model.kv(1, PROMPT + DECODE_STEPS + 64)
     prompt = synth.token_ids(PROMPT, shape.vocab, seed=SEED).to(dev)
@@ -344,6 +346,53 @@ def run_ours(args, world, rank, local):
                                           "flops": flops, "peak_source": peak_src}}
         kvp.close()
 
+    # Batched decode: 16 sequences, each with 8192 pre-filled N(0,1) bf16 K/V
+    # positions, 32 greedy steps (ids stay on the device).
+    bat = None
+    if not args.no_batched:
+        B, CTX, BSTEPS = 16, 8192, 32
+        kvb = model.kv(B, CTX + BSTEPS + 8)
+        for q in range(B):
+            for l in range(shape.n_layers):
+                k, v = synth.prefilled_kv(shape, CTX, seed=3, seq=q, layer=l, device=dev)
+                kvb.import_(q, l, 0, k, v)
+        btok = synth.token_ids(B, shape.vocab, seed=3).to(dev)
+        bgen = torch.zeros((BSTEPS + 1, B), dtype=torch.int32, device=dev)
+        seqs = list(range(B))
+
+        def reset_batch():
+            torch.cuda.synchronize(dev)
+            for q in range(B):
+                kvb.set_length(q, CTX)
+            bgen[0].copy_(btok)
+
+        def bjob(n):
+            for i in range(n):
+                model.decode_step(kvb, seqs, bgen[i], None, bgen[i + 1])
+
+        reset_batch()
+        bjob(3)
+        reset_batch()
+        torch.cuda.synchronize(dev)
+        b0 = torch.cuda.Event(enable_timing=True)
+        b1 = torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        bjob(BSTEPS)
+        b1.record(stream)
+        torch.cuda.synchronize(dev)
+        bms = b0.elapsed_time(b1) / BSTEPS
+        kv_tok = shape.n_layers * 2 * shape.n_kv_heads * shape.head_dim * 2
+        bbytes = weight_bytes + sum(kv_tok * (CTX + i + 1) + kv_tok
+                                    for i in range(BSTEPS)) / BSTEPS * B
+        bach = bbytes / (bms / 1e3) / 1e9
+        bat = {"value": B / (bms / 1e3), "unit": "tok/s", "ms_per_step": bms,
+               "workload": f"batch {B}, {CTX} pre-filled positions per sequence, "
+                           f"{BSTEPS} greedy steps",
+               "roofline": {"bound": "hbm", "achieved": bach, "peak": hbm, "unit": "GB/s",
+                            "frac": bach / hbm, "bytes_per_step": bbytes,
+                            "peak_source": peak_src}}
+        kvb.close()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         sec, cores = oracle_decode_sample(shape, args.cpu_steps)
@@ -368,6 +417,7 @@ def run_ours(args, world, rank, local):
             "gpu_launches": int(launches),
             "clocks": clocks.summary(),
             "prefill": pre,
+            "batched_decode": bat,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line))
@@ -383,6 +433,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-batched", action="store_true")
     ap.add_argument("--cpu-steps", type=int, default=16)
     args = ap.parse_args()
     world, rank, local = dist_setup(args)

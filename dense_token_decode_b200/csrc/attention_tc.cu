@@ -15,9 +15,10 @@
 // updated lazily (only when it grows by more than 2^8 in the exp2 domain),
 // which keeps every P below 256 and the final O / l exact up to rounding.
 //
-// Warp roles (192 threads): warp 0 TMA producer; warp 1 TMEM owner and MMA
-// issuer (one lane); warps 2-5 softmax, one query row per thread (TMEM lane
-// quadrant = warp % 4), then the epilogue writing O / l as fp16.
+// Warp roles (320 threads): warp 0 TMA producer; warp 1 TMEM owner and MMA
+// issuer (one lane); warps 2-9 softmax, two warps per TMEM lane quadrant
+// (= warp % 4): each thread owns one query row and half of the columns, then
+// the epilogue writes its half of O / l as fp16.
 //
 // Requirement: KV slots past a sequence's length hold finite values (they are
 // multiplied by exact zeros); the cache is zeroed when allocated and only ever
@@ -32,7 +33,9 @@ namespace attn_tc {
 
 using namespace tc;
 
-constexpr int kThreads = 192;
+constexpr int kSoftWarps = 8;
+constexpr int kSoft = kSoftWarps * 32;
+constexpr int kThreads = 64 + kSoft;
 constexpr int kQTile = 128;
 constexpr int kKTile = kPage;  // 64 keys = one KV page
 constexpr float kRescaleLog2 = 8.0f;
@@ -43,7 +46,6 @@ struct Params {
   const int32_t* block_table;
   int pages_per_seq, n_pages, nkv, nq, group;
   int layer, seq, pos0, rows, n_qt;
-  int stages;
   float scale_log2;  // log2(e) / sqrt(d)
   int* err;
 };
@@ -53,7 +55,11 @@ struct Layout {
   static constexpr int kChunks = D / 64;             // 64-element (128-byte) column chunks
   static constexpr int kQBytes = 2 * kChunks * 16384;  // Q hi, Q lo: 128 rows x 128 B per chunk
   static constexpr int kPBytes = 4 * 16384;            // P[2 buffers][hi, lo]: 128 x 64 bf16
-  static constexpr int kStageBytes = 2 * kChunks * 8192;  // K and V pages: 64 rows x 128 B per chunk
+  static constexpr int kPageBytes = kChunks * 8192;  // one K or V page: 64 rows x 128 B per chunk
+  static constexpr int kNK = 3, kNV = 2;              // K and V ring stages
+  static constexpr int kKVBytes = (kNK + kNV) * kPageBytes;
+  static constexpr int kMiscBytes = 256 + 3 * 2 * kQTile * 4;  // barriers, row max / sum
+  static constexpr int kSmemBytes = 1024 + kQBytes + kPBytes + kKVBytes + kMiscBytes;
   static constexpr int kTmemCols = 256;                // S[2] (64 cols each) + O (d cols)
   static constexpr int kOCol = 128;
 };
@@ -88,21 +94,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int NK = Lay::kNK, NV = Lay::kNV;
   unsigned char* sQ = smem;
   unsigned char* sP = smem + Lay::kQBytes;
-  unsigned char* sKV = sP + Lay::kPBytes;
-  const int NS = p.stages;
-  uint64_t* kv_full = reinterpret_cast<uint64_t*>(sKV + NS * Lay::kStageBytes);
-  uint64_t* kv_empty = kv_full + NS;
-  uint64_t* s_full = kv_empty + NS;  // [2]
-  uint64_t* s_free = s_full + 2;     // [2]
-  uint64_t* p_full = s_free + 2;     // [2]
-  uint64_t* p_free = p_full + 2;     // [2]
+  unsigned char* sK = sP + Lay::kPBytes;
+  unsigned char* sV = sK + NK * Lay::kPageBytes;
+  uint64_t* k_full = reinterpret_cast<uint64_t*>(sV + NV * Lay::kPageBytes);
+  uint64_t* k_empty = k_full + NK;
+  uint64_t* v_full = k_empty + NK;
+  uint64_t* v_empty = v_full + NV;
+  uint64_t* s_full = v_empty + NV;  // [2]
+  uint64_t* s_free = s_full + 2;    // [2]
+  uint64_t* p_full = s_free + 2;    // [2]
+  uint64_t* p_free = p_full + 2;    // [2]
   uint64_t* q_full = p_free + 2;
   uint64_t* o_full = q_full + 1;
   uint64_t* drain = o_full + 1;
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(drain + 1);
-  uint32_t* counts = tmem_base_s + 1;  // [0] pages loaded, [1] pages waited for
+  uint32_t* counts = tmem_base_s + 1;  // K pages loaded / waited, V pages loaded / waited
+  float(*red_max)[2][kQTile] = reinterpret_cast<float(*)[2][kQTile]>(
+      reinterpret_cast<unsigned char*>(k_full) + 256);  // [page parity][half][row]
+  float(*red_sum)[kQTile] = reinterpret_cast<float(*)[kQTile]>(red_max + 2);  // [half][row]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = p.n_qt - 1 - (int)blockIdx.x / p.nq;
@@ -113,20 +125,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nt = (p.pos0 + last_row) / kKTile + 1;  // KV pages this tile attends
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+    for (int s = 0; s < NK; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < NV; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], 128);
-      mbar_init(&p_full[b], 128);
+      mbar_init(&s_free[b], kSoft);
+      mbar_init(&p_full[b], kSoft);
       mbar_init(&p_free[b], 1);
     }
-    mbar_init(q_full, 128);
+    mbar_init(q_full, kSoft);
     mbar_init(o_full, 1);
     mbar_init(drain, 1);
-    counts[0] = counts[1] = 0;
+    counts[0] = counts[1] = counts[2] = counts[3] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) tmem_alloc(tmem_base_s, Lay::kTmemCols);
@@ -139,22 +155,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       for (int j = 0; j < nt; ++j) {
-        const int s = j % NS;
-        if (!mbar_wait(&kv_empty[s], ((j / NS) & 1) ^ 1, p.err)) break;
         int page = p.block_table[(size_t)p.seq * p.pages_per_seq + j];
         if (page < 0 || page >= p.n_pages) {
           atomicCAS(p.err, 0, kErrBounds);
           page = 0;
         }
         const int row = ((p.layer * p.n_pages + page) * p.nkv + g) * kKTile;
-        unsigned char* st = sKV + s * Lay::kStageBytes;
-        mbar_expect_tx(&kv_full[s], Lay::kStageBytes);
+        const int sk = j % NK, sv = j % NV;
+        if (!mbar_wait(&k_empty[sk], ((j / NK) & 1) ^ 1, p.err)) break;
+        mbar_expect_tx(&k_full[sk], Lay::kPageBytes);
 #pragma unroll
-        for (int c = 0; c < Lay::kChunks; ++c) {
-          tma_load_2d(st + c * 8192, &map_k, c * 64, row, &kv_full[s]);
-          tma_load_2d(st + (Lay::kChunks + c) * 8192, &map_v, c * 64, row, &kv_full[s]);
-        }
+        for (int c = 0; c < Lay::kChunks; ++c)
+          tma_load_2d(sK + sk * Lay::kPageBytes + c * 8192, &map_k, c * 64, row, &k_full[sk]);
         ++counts[0];
+        if (!mbar_wait(&v_empty[sv], ((j / NV) & 1) ^ 1, p.err)) break;
+        mbar_expect_tx(&v_full[sv], Lay::kPageBytes);
+#pragma unroll
+        for (int c = 0; c < Lay::kChunks; ++c)
+          tma_load_2d(sV + sv * Lay::kPageBytes + c * 8192, &map_v, c * 64, row, &v_full[sv]);
+        ++counts[2];
       }
     }
   } else if (warp == 1) {
@@ -167,14 +186,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) fence_after();
       for (int j = 0; j <= nt && ok; ++j) {
         if (j < nt) {
-          const int s = j % NS, b = j & 1;
-          ok = mbar_wait(&kv_full[s], (j / NS) & 1, p.err);
+          const int sk = j % NK, b = j & 1;
+          ok = mbar_wait(&k_full[sk], (j / NK) & 1, p.err);
           if (!ok) break;
           ++counts[1];
           ok = mbar_wait(&s_free[b], ((j >> 1) & 1) ^ 1, p.err);
           if (!ok) break;
           fence_after();
-          const unsigned char* kst = sKV + s * Lay::kStageBytes;
+          const unsigned char* kst = sK + sk * Lay::kPageBytes;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const int c = kk >> 2, off = (kk & 3) * 32;
@@ -184,13 +203,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     1u);
           }
           mma_commit(&s_full[b]);
+          mma_commit(&k_empty[sk]);
         }
         if (j >= 1) {
-          const int i = j - 1, s = i % NS, b = i & 1;
+          const int i = j - 1, sv = i % NV, b = i & 1;
+          ok = mbar_wait(&v_full[sv], (i / NV) & 1, p.err);
+          if (!ok) break;
+          ++counts[3];
           ok = mbar_wait(&p_full[b], (i >> 1) & 1, p.err);
           if (!ok) break;
           fence_after();
-          const unsigned char* vst = sKV + s * Lay::kStageBytes + Lay::kChunks * 8192;
+          const unsigned char* vst = sV + sv * Lay::kPageBytes;
           const unsigned char* pb = sP + b * 2 * 16384;
 #pragma unroll
           for (int kk = 0; kk < kKTile / 16; ++kk) {
@@ -199,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_f16(t_o, smem_desc(pb + 16384 + kk * 32), bv, id_pv, 1u);
           }
           mma_commit(&p_free[b]);
-          mma_commit(&kv_empty[s]);
+          mma_commit(&v_empty[sv]);
         }
       }
       if (ok) mma_commit(o_full);
@@ -211,74 +234,104 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------------- softmax warps
+    // Two warps per TMEM lane quadrant: `half` 0 owns score columns 0..31 of
+    // each page and O columns 0..d/2-1, `half` 1 the rest. The row maximum is
+    // combined through shared memory (one named barrier per quadrant pair).
     const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row = quad * 32 + lane;
     const int r = q0 + row;
     const bool live = r < p.rows;
     const int qp = p.pos0 + (live ? r : p.rows - 1);  // position of this query
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    constexpr int kOHalf = D / 2;
+    auto pair_sync = [&]() {
+      asm volatile("bar.sync %0, 64;" ::"r"(1 + quad) : "memory");
+    };
+    auto pair_or = [&](int id, bool v) -> bool {
+      uint32_t r;
+      asm volatile(
+          "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, 64, p;\n"
+          " selp.u32 %0, 1, 0, q;\n}\n"
+          : "=r"(r)
+          : "r"((uint32_t)v), "r"(id)
+          : "memory");
+      return r != 0;
+    };
 
-    // Q row -> two bf16 terms in swizzled K-major layout.
+    // Q row -> two bf16 terms in swizzled K-major layout (this warp's half of the units).
     {
       const float4* src = reinterpret_cast<const float4*>(p.q + ((size_t)r * p.nq + h) * D);
+      constexpr int kUnits = Lay::kChunks * 8;  // 16-byte units of a row
 #pragma unroll
-      for (int c = 0; c < Lay::kChunks; ++c) {
+      for (int uu = 0; uu < kUnits / 2; ++uu) {
+        const int un = half * (kUnits / 2) + uu;
+        const int c = un >> 3, u = un & 7;
+        float x[8];
+        if (live) {
+          const float4 a = src[un * 2], b4 = src[un * 2 + 1];
+          x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+          x[4] = b4.x; x[5] = b4.y; x[6] = b4.z; x[7] = b4.w;
+        } else {
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          float x[8];
-          if (live) {
-            const float4 a = src[c * 16 + u * 2], b4 = src[c * 16 + u * 2 + 1];
-            x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-            x[4] = b4.x; x[5] = b4.y; x[6] = b4.z; x[7] = b4.w;
-          } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) x[i] = 0.f;
-          }
-          uint4 hi, lo;
-          split8(x, hi, lo);
-          *reinterpret_cast<uint4*>(sQ + c * 16384 + swz(row, u)) = hi;
-          *reinterpret_cast<uint4*>(sQ + (Lay::kChunks + c) * 16384 + swz(row, u)) = lo;
+          for (int i = 0; i < 8; ++i) x[i] = 0.f;
         }
+        uint4 hi, lo;
+        split8(x, hi, lo);
+        *reinterpret_cast<uint4*>(sQ + c * 16384 + swz(row, u)) = hi;
+        *reinterpret_cast<uint4*>(sQ + (Lay::kChunks + c) * 16384 + swz(row, u)) = lo;
       }
       fence_proxy_async();
       mbar_arrive(q_full);
     }
 
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY, l = 0.f;  // l: this warp's columns only
     bool ok = true;
-    for (int j = 0; j < nt && ok; ++j) {
+    // The two warps of a quadrant pair leave the loop together: every pass
+    // ends in one reducing barrier that ORs their failure flags (a timed-out
+    // warp skips the work but still takes part).
+    for (int j = 0; j < nt; ++j) {
       const int b = j & 1;
-      ok = mbar_wait_warp(&s_full[b], (j >> 1) & 1, p.err);
-      if (!ok) break;
-      fence_after();
-      float x[kKTile];
-      {
-        uint32_t ra[32], rb[32];
-        tmem_ld32(tmem + lane_off + b * kKTile, ra);
-        tmem_ld32(tmem + lane_off + b * kKTile + 32, rb);
+      float x[32];
+      float mx = -INFINITY;
+      if (ok) ok = mbar_wait_warp(&s_full[b], (j >> 1) & 1, p.err);
+      if (ok) {
+        fence_after();
+        uint32_t ra[32];
+        tmem_ld32(tmem + lane_off + b * kKTile + half * 32, ra);
         fence_before();
         mbar_arrive(&s_free[b]);
-        const int lim = qp - j * kKTile;  // keys c <= lim are visible
+        const int lim = qp - j * kKTile - half * 32;  // columns c <= lim are visible
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
+        for (int c = 0; c < 32; ++c)
           x[c] = c <= lim ? __uint_as_float(ra[c]) * p.scale_log2 : -INFINITY;
-          x[c + 32] = c + 32 <= lim ? __uint_as_float(rb[c]) * p.scale_log2 : -INFINITY;
-        }
-      }
-      float mx = x[0];
+        float mx4[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-      for (int c = 1; c < kKTile; ++c) mx = fmaxf(mx, x[c]);
+        for (int c = 4; c < 32; c += 4)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) mx4[i] = fmaxf(mx4[i], x[c + i]);
+        mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      }
+      red_max[b][half][row] = mx;
+      if (pair_or(1 + quad, !ok)) {
+        ok = false;
+        break;
+      }
+      mx = fmaxf(mx, red_max[b][half ^ 1][row]);
       const float m_new = fmaxf(m, mx);
       if (j == 0) {
         m = m_new;  // key 0 is visible to every row: finite
       } else if (__any_sync(0xffffffffu, m_new > m + kRescaleLog2)) {
+        // Both warps of the pair see the same rows and maxima: same decision.
         const float alpha = exp2f(m - m_new);
         // O may only be rescaled once the previous P V has landed in it.
-        ok = mbar_wait_warp(&p_free[(j - 1) & 1], ((j - 1) >> 1) & 1, p.err);
-        if (!ok) break;
+        if (!mbar_wait_warp(&p_free[(j - 1) & 1], ((j - 1) >> 1) & 1, p.err)) {
+          ok = false;
+          continue;
+        }
         fence_after();
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
+        for (int c0 = half * kOHalf; c0 < (half + 1) * kOHalf; c0 += 32) {
           uint32_t o[32];
           tmem_ld32(tmem + lane_off + Lay::kOCol + c0, o);
 #pragma unroll
@@ -288,35 +341,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         l *= alpha;
         m = m_new;
       }
-      float sum = 0.f;
+      float sm4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < kKTile; ++c) {
-        x[c] = exp2f(x[c] - m);
-        sum += x[c];
-      }
-      l += sum;
+      for (int c = 0; c < 32; c += 4)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          x[c + i] = exp2f(x[c + i] - m);
+          sm4[i] += x[c + i];
+        }
+      l += (sm4[0] + sm4[1]) + (sm4[2] + sm4[3]);
       // P buffer b is free once the P V of page j - 2 has completed.
-      ok = mbar_wait_warp(&p_free[b], ((j >> 1) & 1) ^ 1, p.err);
-      if (!ok) break;
+      if (!mbar_wait_warp(&p_free[b], ((j >> 1) & 1) ^ 1, p.err)) {
+        ok = false;
+        continue;
+      }
       unsigned char* pb = sP + b * 2 * 16384;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 4; ++u) {
         uint4 hi, lo;
         split8(x + u * 8, hi, lo);
-        *reinterpret_cast<uint4*>(pb + swz(row, u)) = hi;
-        *reinterpret_cast<uint4*>(pb + 16384 + swz(row, u)) = lo;
+        *reinterpret_cast<uint4*>(pb + swz(row, half * 4 + u)) = hi;
+        *reinterpret_cast<uint4*>(pb + 16384 + swz(row, half * 4 + u)) = lo;
       }
       fence_proxy_async();
       fence_before();
       mbar_arrive(&p_full[b]);
     }
+    // Full row sum from the two halves (uniform control flow for the barrier:
+    // a timed-out warp still takes part).
+    red_sum[half][row] = l;
+    pair_sync();
+    const float l_row = l + red_sum[half ^ 1][row];
     if (ok) ok = mbar_wait_warp(o_full, 0, p.err);
     if (ok) {
       fence_after();
-      const float inv = 1.f / l;
+      const float inv = 1.f / l_row;
       __half* dst = p.o + ((size_t)r * p.nq + h) * D;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = half * kOHalf; c0 < (half + 1) * kOHalf; c0 += 32) {
         uint32_t o[32];
         tmem_ld32(tmem + lane_off + Lay::kOCol + c0, o);
         if (live) {
@@ -335,10 +397,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   // After a timeout: pages loaded but never waited for must land before the
   // CTA's shared memory is released (bounded wait, 10 ms each).
-  if (threadIdx.x == 0 && counts[0] > counts[1]) {
+  if (threadIdx.x == 0) {
     for (uint32_t k = counts[1]; k < counts[0]; ++k) {
       const unsigned long long t0 = now_ns();
-      while (!mbar_try(&kv_full[k % NS], (k / NS) & 1))
+      while (!mbar_try(&k_full[k % NK], (k / NK) & 1))
+        if (now_ns() - t0 > 10000000ull) break;
+    }
+    for (uint32_t k = counts[3]; k < counts[2]; ++k) {
+      const unsigned long long t0 = now_ns();
+      while (!mbar_try(&v_full[k % NV], (k / NV) & 1))
         if (now_ns() - t0 > 10000000ull) break;
     }
   }
@@ -352,18 +419,15 @@ template <int D>
 cudaError_t launch(const Params& p, const CUtensorMap& mk, const CUtensorMap& mv, int grid,
                    cudaStream_t st) {
   using Lay = Layout<D>;
-  constexpr int kMaxSmem = 232448;
-  constexpr int kFixed = 1024 + Lay::kQBytes + Lay::kPBytes + 256;
+  static_assert(Lay::kSmemBytes <= 232448, "shared memory budget");
   static bool attr_done = false;
   if (!attr_done) {
     cudaFuncSetAttribute(attention_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         kMaxSmem);
+                         Lay::kSmemBytes);
     attr_done = true;
   }
-  Params q = p;
-  q.stages = std::min(4, (kMaxSmem - kFixed) / Lay::kStageBytes);
-  if (q.stages < 2) return cudaErrorInvalidValue;
-  const size_t smem = kFixed + (size_t)q.stages * Lay::kStageBytes;
+  const size_t smem = Lay::kSmemBytes;
+  const Params& q = p;
   count_launches();
   attention_tc_kernel<D><<<grid, kThreads, smem, st>>>(q, mk, mv);
   return cudaGetLastError();

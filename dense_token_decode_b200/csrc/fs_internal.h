@@ -113,6 +113,13 @@ cudaError_t launch_qk_norm_rope_append(const float* qkv, int rows, const RowMap&
 cudaError_t launch_attention_simple(const float* q, int rows, const RowMap& map,
                                     const Shape& s, KVView kv, int layer, float* o,
                                     cudaStream_t st);
+// Split-KV decode attention (rows <= 128, any positions); max_pos is the
+// largest position among the rows, part the model's partial buffer.
+bool attention_decode_supported(const Shape& s, int rows);
+size_t attention_decode_part_floats(const Shape& s);
+cudaError_t launch_attention_decode(const float* q, int rows, const RowMap& map, int max_pos,
+                                    const Shape& s, KVView kv, int layer, float* part, float* o,
+                                    int num_sms, cudaStream_t st);
 // x: final-normed rows fp32 [rows, H]; partial: scratch of rows * n_part float2.
 cudaError_t launch_lm_head(const float* xf, int rows, const Shape& s, const __nv_bfloat16* E,
                            float* logits, int32_t* argmax, float2* partial, int n_part, int* err,

@@ -68,7 +68,8 @@ namespace fs {
 
 void model_free_buffers(fs_model* m) {
   void* bufs[] = {m->rope, m->h,   m->xn,  m->qkv,     m->q,   m->o,       m->gu,
-                  m->act,  m->xf,  m->tok, m->partial, m->err, m->gen_tok, m->scratch};
+                  m->act,  m->xf,  m->tok, m->partial, m->err, m->gen_tok, m->scratch,
+                  m->attn_part};
   for (void* b : bufs)
     if (b) cudaFree(b);
   release_extras(m);
@@ -176,6 +177,7 @@ extern "C" fs_status fs_model_create(const fs_config* cfg, const fs_weights* w, 
       (st = dev_alloc(&m->qkv, R * s.qkv_dim(), "workspace")) != FS_OK ||
       (st = dev_alloc(&m->q, R * s.q_dim(), "workspace")) != FS_OK ||
       (st = dev_alloc(&m->o, R * s.q_dim(), "workspace")) != FS_OK ||
+      (st = dev_alloc(&m->attn_part, fs::attention_decode_part_floats(s), "workspace")) != FS_OK ||
       (st = dev_alloc(&m->gu, R * 2 * s.I, "workspace")) != FS_OK ||
       (st = dev_alloc(&m->act, R * s.I, "workspace")) != FS_OK ||
       (st = dev_alloc(&m->xf, (size_t)fs::kMaxBatch * s.H, "workspace")) != FS_OK ||
@@ -379,7 +381,14 @@ fs_status layer_general(fs_model* m, const fs_kv* kv, const RowMap& map, int row
   FS_CUDA(linear(m, m->xn, rows, H, l, kWv, kvd, m->qkv + qd + kvd, qkvd, false, st));
   FS_CUDA(launch_qk_norm_rope_append(m->qkv, rows, map, s, Lw.q_norm, Lw.k_norm, m->rope, m->q,
                                      kvv, l, st));
-  FS_CUDA(launch_attention_simple(m->q, rows, map, s, kvv, l, m->o, st));
+  if (attention_decode_supported(s, rows)) {
+    int max_pos = 0;
+    for (int r = 0; r < rows; ++r) max_pos = std::max(max_pos, map.get(r).pos);
+    FS_CUDA(launch_attention_decode(m->q, rows, map, max_pos, s, kvv, l, m->attn_part, m->o,
+                                    m->num_sms, st));
+  } else {
+    FS_CUDA(launch_attention_simple(m->q, rows, map, s, kvv, l, m->o, st));
+  }
   FS_CUDA(linear(m, m->o, rows, qd, l, kWo, H, m->h, H, true, st));
   FS_CUDA(launch_rmsnorm(m->h, rows, H, Lw.ffn_norm, s.eps, m->xn, st));
   if (rows <= 16) {

@@ -24,6 +24,7 @@ struct fs_model {
   float* qkv = nullptr;    // [max_rows, (nq+2nkv)*d]
   float* q = nullptr;      // rotated queries [max_rows, nq*d]
   float* o = nullptr;      // attention output [max_rows, nq*d]
+  float* attn_part = nullptr;  // split-KV attention partials (attention_decode.cu)
   float* gu = nullptr;     // gate||up [max_rows, 2I]
   float* act = nullptr;    // SwiGLU output [max_rows, I]
   float* xf = nullptr;     // final-normed rows [64, H]

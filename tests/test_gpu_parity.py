@@ -307,6 +307,32 @@ def test_tiny_batched_decode_mixed_positions(tiny):
         assert kv.length(q) == lens[q] + 1
 
 
+def test_tiny_split_kv_decode_batch_of_seven(tiny):
+    """A batch above the persistent kernel's 4 rows takes the split-KV decode
+    attention: contexts from 1 to 900 positions in one launch, so most rows
+    own fewer pages than the longest one (empty splits), and page-boundary
+    positions (64, 128, 512)."""
+    s = tiny.shape
+    lens = [900, 1, 64, 128, 5, 512, 300]
+    prompts = [synth.token_ids(n, s.vocab, seed=40 + i).tolist() for i, n in enumerate(lens)]
+    kv = tiny.model.kv(7, 1024)
+    caches = []
+    for i, p in enumerate(prompts):
+        tiny.model.prefill(kv, i, _dev_i32(p))
+        caches.append(tiny.oracle.forward(p)[2])
+    nxt = [11, 22, 33, 44, 55, 66, 77]
+    order = [6, 0, 5, 1, 4, 2, 3]
+    logits = torch.empty((7, s.vocab), device=DEV)
+    am = torch.empty(7, dtype=torch.int32, device=DEV)
+    tiny.model.decode_step(kv, order, _dev_i32([nxt[q] for q in order]), logits, am)
+    torch.cuda.synchronize()
+    for b, q in enumerate(order):
+        rl = tiny.oracle.forward([nxt[q]], caches[q])[0]
+        assert_logits_close(oracle_tensor(logits[b]), rl, what=f"batch row {b} (len {lens[q]})")
+        check_greedy_step(int(am[b]), oracle_tensor(logits[b]), rl)
+        assert kv.length(q) == lens[q] + 1
+
+
 def test_tiny_errors_are_reported_not_faulted(tiny):
     m, s = tiny.model, tiny.shape
     kv = m.kv(2, 16)
