@@ -80,7 +80,7 @@ struct Params {
   unsigned long long* trace;  // optional: %globaltimer stamps [G][L+1][16]
   int n_stages;
   // smem carve-up (bytes)
-  int off_hs, off_xs, off_attn, off_red, off_bar, off_misc, off_tab;
+  int off_hs, off_xs, off_attn, off_bar, off_misc, off_tab;
   int bt_in_smem;  // block-table rows of the batch copied to shared memory
 };
 
@@ -482,8 +482,6 @@ struct Consumer {
   unsigned char* smem;
   float* hs;  // [B][H] block input / mid residual
   float* xs;  // [B][max K] GEMV operand
-  float* comb;  // [stages][8 rows][2][kMaxB] partial sums of split rows
-  int* ccnt;    // [stages][8 rows] arrivals per split row
   float* at;    // attention scratch
   unsigned long long wbest[kMaxB] = {0ull, 0ull, 0ull, 0ull};  // this lane's greedy keys
   unsigned long long* best;  // [kMaxB] greedy keys of this CTA
@@ -502,8 +500,6 @@ struct Consumer {
     hs = reinterpret_cast<float*>(sm + p.off_hs);
     xs = reinterpret_cast<float*>(sm + p.off_xs);
     at = reinterpret_cast<float*>(sm + p.off_attn);
-    comb = reinterpret_cast<float*>(sm + p.off_red);
-    ccnt = reinterpret_cast<int*>(sm + p.off_red + kMaxStages * kConsumerWarps * 2 * kMaxB * 4);
     best = reinterpret_cast<unsigned long long*>(sm + p.off_misc);
     flag = reinterpret_cast<int*>(sm + p.off_misc + 8 * kMaxB);
     tid = threadIdx.x;
@@ -1024,26 +1020,123 @@ struct Consumer {
     }
   }
 
+  // Transposing butterfly: NV partial sums per lane -> the full sum of value
+  // lane >> (5 - log2 NV) in every lane.
+  template <int NV>
+  __device__ __forceinline__ float reduce_transpose(float (&v)[NV]) {
+    int w = NV / 2, mask = 16;
+#pragma unroll
+    for (; w >= 1; w >>= 1, mask >>= 1) {
+      const bool upper = (lane & mask) != 0;
+#pragma unroll
+      for (int i = 0; i < w; ++i) {
+        const float send = upper ? v[i] : v[i + w];
+        const float keep = upper ? v[i + w] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+      }
+    }
+    float t = v[0];
+#pragma unroll
+    for (; mask >= 1; mask >>= 1) t += __shfl_xor_sync(0xffffffffu, t, mask);
+    return t;
+  }
+
+  // Online-softmax update with this warp's keys of a KV chunk: keys warp,
+  // warp + 11, ... (at most KG). The KG x 2 partial dot products are reduced
+  // across the warp in one transposing butterfly; each lane pair / quad then
+  // holds one (key, head) score.
+  template <int E>
+  __device__ __forceinline__ void attend_group(const __nv_bfloat16* K, const __nv_bfloat16* Vv,
+                                               int nk) {
+    constexpr int KG = E == 4 ? 4 : 8;  // keys per warp: a chunk holds 32 (d=128) or 64 keys
+    constexpr int NV = 2 * KG;          // (key, head) pairs, head fastest
+    constexpr int SH = NV == 8 ? 2 : 1;
+    const int d = 32 * E;
+    uint32_t kr[KG][E / 2], vr[KG][E / 2];
+#pragma unroll
+    for (int i = 0; i < KG; ++i) {
+      const int j = warp + i * kConsumerWarps;
+#pragma unroll
+      for (int e = 0; e < E / 2; ++e) {
+        kr[i][e] = 0u;
+        vr[i][e] = 0u;
+      }
+      if (j < nk) {
+        if constexpr (E == 4) {
+          const uint2 ku = *reinterpret_cast<const uint2*>(K + j * d + lane * 4);
+          const uint2 vu = *reinterpret_cast<const uint2*>(Vv + j * d + lane * 4);
+          kr[i][0] = ku.x; kr[i][1] = ku.y;
+          vr[i][0] = vu.x; vr[i][1] = vu.y;
+        } else {
+          kr[i][0] = *reinterpret_cast<const uint32_t*>(K + j * d + lane * 2);
+          vr[i][0] = *reinterpret_cast<const uint32_t*>(Vv + j * d + lane * 2);
+        }
+      }
+    }
+    float part[NV];
+#pragma unroll
+    for (int i = 0; i < KG; ++i)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float t = 0.f;
+#pragma unroll
+        for (int e = 0; e < E / 2; ++e) {
+          t = fmaf(qreg[h][2 * e], lo16(kr[i][e]), t);
+          t = fmaf(qreg[h][2 * e + 1], hi16(kr[i][e]), t);
+        }
+        part[i * 2 + h] = t;
+      }
+    float sc = reduce_transpose<NV>(part);
+    const int my_v = lane >> SH, my_k = my_v >> 1, my_h = my_v & 1;
+    if (warp + my_k * kConsumerWarps >= nk) sc = -INFINITY;
+    float gm = sc;
+#pragma unroll
+    for (int b = SH + 1; b < 5; ++b) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, 1 << b));
+    float m_new[2], alpha[2];
+    bool any = false;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float gmh = __shfl_sync(0xffffffffu, gm, h << SH);
+      any |= gmh != -INFINITY;
+      m_new[h] = fmaxf(m[h], gmh);
+      alpha[h] = (m_new[h] == -INFINITY) ? 1.f : expf(m[h] - m_new[h]);
+    }
+    if (!any) return;  // no key of this chunk for this warp (warp-uniform)
+    const float mh = my_h ? m_new[1] : m_new[0];
+    const float pv = (sc == -INFINITY) ? 0.f : expf(sc - mh);
+    float gs = pv;
+#pragma unroll
+    for (int b = SH + 1; b < 5; ++b) gs += __shfl_xor_sync(0xffffffffu, gs, 1 << b);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      l[h] = l[h] * alpha[h] + __shfl_sync(0xffffffffu, gs, h << SH);
+      m[h] = m_new[h];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[h][e] *= alpha[h];
+    }
+#pragma unroll
+    for (int i = 0; i < KG; ++i)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float pk = __shfl_sync(0xffffffffu, pv, (i * 2 + h) << SH);
+#pragma unroll
+        for (int e = 0; e < E / 2; ++e) {
+          acc[h][2 * e] = fmaf(pk, lo16(vr[i][e]), acc[h][2 * e]);
+          acc[h][2 * e + 1] = fmaf(pk, hi16(vr[i][e]), acc[h][2 * e + 1]);
+        }
+      }
+  }
+
   __device__ __forceinline__ void kv(int, const Item&, int, int nk) {
     // Contains a CTA barrier: no early exit; a thread that gave up skips the work.
     const unsigned char* st = stage_wait();
-    const int d = p.d, rep = p.nq / p.nkv, E = d / 32;
     const __nv_bfloat16* K = reinterpret_cast<const __nv_bfloat16*>(st);
     const __nv_bfloat16* Vv = reinterpret_cast<const __nv_bfloat16*>(st + kWeightBytes / 2);
-    for (int j = warp; j < nk && !quit; j += kConsumerWarps) {
-      float kk[4] = {0.f, 0.f, 0.f, 0.f}, vv[4] = {0.f, 0.f, 0.f, 0.f};
-      if (E == 4) {
-        const uint2 ku = *reinterpret_cast<const uint2*>(K + j * d + lane * 4);
-        const uint2 vu = *reinterpret_cast<const uint2*>(Vv + j * d + lane * 4);
-        kk[0] = lo16(ku.x); kk[1] = hi16(ku.x); kk[2] = lo16(ku.y); kk[3] = hi16(ku.y);
-        vv[0] = lo16(vu.x); vv[1] = hi16(vu.x); vv[2] = lo16(vu.y); vv[3] = hi16(vu.y);
-      } else {
-        const uint32_t ku = *reinterpret_cast<const uint32_t*>(K + j * d + lane * 2);
-        const uint32_t vu = *reinterpret_cast<const uint32_t*>(Vv + j * d + lane * 2);
-        kk[0] = lo16(ku); kk[1] = hi16(ku);
-        vv[0] = lo16(vu); vv[1] = hi16(vu);
-      }
-      attend(kk, vv, rep);
+    if (!__any_sync(0xffffffffu, quit)) {
+      if (p.d == 128)
+        attend_group<4>(K, Vv, nk);
+      else
+        attend_group<2>(K, Vv, nk);
     }
     // Every consumer warp reads a KV chunk; the stage is released once, after
     // all of them are done with it.
@@ -1214,11 +1307,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mega_kernel(const __grid_c
       for (int k = threadIdx.x; k < p.B * pps; k += blockDim.x)
         bt[k] = p.kv.block_table[(size_t)p.seq[k / pps] * pps + k % pps];
     }
-  }
-  {
-    float* cz = reinterpret_cast<float*>(smem + p.off_red);
-    const int n = kMaxStages * kConsumerWarps * (2 * kMaxB + 1);
-    for (int k = threadIdx.x; k < n; k += blockDim.x) cz[k] = 0.f;
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5;
@@ -1450,23 +1538,23 @@ fs_status decode_mega(fs_model* m, const fs_kv* kv, const RowMap& map, int B, co
   const size_t fixed_xs = align_up((size_t)B * maxK * 4, 128);
   const size_t attn = align_up((16 + rep * s.d + 2 * s.d + mega::kConsumerWarps * rep * 2 +
                                 mega::kConsumerWarps * rep * s.d) * 4, 128);
-  const size_t redb =
-      align_up((size_t)mega::kMaxStages * mega::kConsumerWarps * (2 * mega::kMaxB + 1) * 4, 128);
   const size_t bars = 2 * mega::kMaxStages * 8;
   const size_t misc = 128;
   const size_t bt_bytes = (size_t)B * kv->pages_per_seq * sizeof(int32_t);
   const bool bt_smem = bt_bytes <= 8192;
   const size_t tab = align_up((size_t)s.L * sizeof(LayerDev) + (bt_smem ? bt_bytes : 0), 128);
-  const size_t fixed = fixed_hs + fixed_xs + attn + redb + bars + misc + tab;
+  const size_t fixed = fixed_hs + fixed_xs + attn + bars + misc + tab;
   const size_t budget = 232448;
   int n_stages = (int)((budget - fixed) / mega::kStageBytes);
   n_stages = std::min(n_stages, mega::kMaxStages);
-  if (n_stages < 3) return FS_ERR_UNSUPPORTED;
+  // The ring keeps at least one stage per consumer warp: with fewer, steps
+  // were seen to stall until the wait limit, so such shapes and batch sizes
+  // take the general path.
+  if (n_stages < mega::kConsumerWarps) return FS_ERR_UNSUPPORTED;
   off = (size_t)n_stages * mega::kStageBytes;
   p.off_hs = (int)off; off += fixed_hs;
   p.off_xs = (int)off; off += fixed_xs;
   p.off_attn = (int)off; off += attn;
-  p.off_red = (int)off; off += redb;
   p.off_bar = (int)off; off += bars;
   p.off_misc = (int)off; off += misc;
   p.off_tab = (int)off; off += tab;

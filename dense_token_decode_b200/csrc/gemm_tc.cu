@@ -25,9 +25,9 @@
 namespace fs {
 namespace tc {
 
-constexpr int BM = 128, BN = 128, BK = 64;
+constexpr int BM = 128, BK = 64;
 constexpr int kThreads = 192;
-constexpr int kTileBytes = BM * BK * 2;  // 16 KB for a 128 x 64 fp16 tile
+constexpr int kTileBytes = BM * BK * 2;  // 16 KB for a 128 x 64 fp16 A tile
 
 enum Kind { kStore = 0, kResidual = 1, kSwiGLU = 2 };
 
@@ -45,6 +45,9 @@ struct Params {
   int* err;
 };
 
+// BN (128 or 256): output columns per tile; the B tile is BN x 64 and the two
+// fp32 accumulators take 2 x BN tensor-memory columns.
+template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap map_a,
                    const __grid_constant__ CUtensorMap map_a_lo,
@@ -55,7 +58,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = p.stages;
-  const int stage_bytes = (p.a_terms + 1) * kTileBytes;
+  constexpr int kBBytes = BN * BK * 2;
+  const int stage_bytes = p.a_terms * kTileBytes + kBBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * stage_bytes);
   uint64_t* empty = full + S;
   uint64_t* acc_full = empty + S;   // [2]
@@ -112,7 +116,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (swiglu) {
             // 64 gate rows then 64 up rows of the same act columns
             tma_load_2d(sb, &map_b, kb * BK, nt * (BN / 2), &full[s]);
-            tma_load_2d(sb + kTileBytes / 2, &map_b2, kb * BK, nt * (BN / 2), &full[s]);
+            tma_load_2d(sb + kBBytes / 2, &map_b2, kb * BK, nt * (BN / 2), &full[s]);
           } else {
             tma_load_2d(sb, &map_b, kb * BK, nt * BN, &full[s]);
           }
@@ -290,15 +294,16 @@ bool make_tmap_16(CUtensorMap* map, const void* base, long long rows, int cols, 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Launch one tensor-core GEMM. a_lo may be null (one fp16 term). For kSwiGLU
-// b2 is the up matrix and N counts gate+up columns per tile pair (2 * I).
-cudaError_t launch_gemm_tc(const CUtensorMap* a, const CUtensorMap* a_lo, const CUtensorMap* b,
-                           const CUtensorMap* b2, int M, int N, int K, int kind, float* out,
-                           int ldo, __half* act_hi, __half* act_lo, int act_ld, int* err,
-                           int num_sms, cudaStream_t st) {
+namespace {
+template <int BN>
+cudaError_t launch_bn(const CUtensorMap* a, const CUtensorMap* a_lo, const CUtensorMap* b,
+                      const CUtensorMap* b2, int M, int N, int K, int kind, float* out, int ldo,
+                      __half* act_hi, __half* act_lo, int act_ld, int* err, int num_sms,
+                      cudaStream_t st) {
   static bool attr_done = false;
   if (!attr_done) {
-    cudaFuncSetAttribute(tc::gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+    cudaFuncSetAttribute(tc::gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         232448);
     attr_done = true;
   }
   tc::Params p{};
@@ -308,8 +313,8 @@ cudaError_t launch_gemm_tc(const CUtensorMap* a, const CUtensorMap* a_lo, const 
   p.kind = kind;
   p.a_terms = a_lo ? 2 : 1;
   p.n_tiles_m = (M + tc::BM - 1) / tc::BM;
-  p.n_tiles_n = N / tc::BN;
-  const int stage_bytes = (p.a_terms + 1) * tc::kTileBytes;
+  p.n_tiles_n = N / BN;
+  const int stage_bytes = p.a_terms * tc::kTileBytes + BN * tc::BK * 2;
   p.stages = std::min(8, (232448 - 2048) / stage_bytes);
   p.out = out;
   p.ldo = ldo;
@@ -321,8 +326,25 @@ cudaError_t launch_gemm_tc(const CUtensorMap* a, const CUtensorMap* a_lo, const 
   const int tiles = p.n_tiles_m * p.n_tiles_n;
   const int grid = std::min(tiles, num_sms);
   count_launches();
-  tc::gemm_tc_kernel<<<grid, tc::kThreads, smem, st>>>(p, *a, a_lo ? *a_lo : *a, *b, b2 ? *b2 : *b);
+  tc::gemm_tc_kernel<BN><<<grid, tc::kThreads, smem, st>>>(p, *a, a_lo ? *a_lo : *a, *b,
+                                                           b2 ? *b2 : *b);
   return cudaGetLastError();
+}
+}  // namespace
+
+// Launch one tensor-core GEMM with BN-wide output tiles (128 or 256; the B
+// tensor maps must have boxes of BN rows, BN / 2 for kSwiGLU). a_lo may be
+// null (one fp16 term). For kSwiGLU b2 is the up matrix and N counts
+// gate+up columns (2 * I).
+cudaError_t launch_gemm_tc(const CUtensorMap* a, const CUtensorMap* a_lo, const CUtensorMap* b,
+                           const CUtensorMap* b2, int M, int N, int K, int kind, float* out,
+                           int ldo, __half* act_hi, __half* act_lo, int act_ld, int* err,
+                           int num_sms, cudaStream_t st, int bn) {
+  if (bn == 256)
+    return launch_bn<256>(a, a_lo, b, b2, M, N, K, kind, out, ldo, act_hi, act_lo, act_ld, err,
+                          num_sms, st);
+  return launch_bn<128>(a, a_lo, b, b2, M, N, K, kind, out, ldo, act_hi, act_lo, act_ld, err,
+                        num_sms, st);
 }
 
 }  // namespace fs

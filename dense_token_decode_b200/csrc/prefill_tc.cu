@@ -17,7 +17,7 @@ namespace fs {
 cudaError_t launch_gemm_tc(const CUtensorMap* a, const CUtensorMap* a_lo, const CUtensorMap* b,
                            const CUtensorMap* b2, int M, int N, int K, int kind, float* out,
                            int ldo, __half* act_hi, __half* act_lo, int act_ld, int* err,
-                           int num_sms, cudaStream_t st);
+                           int num_sms, cudaStream_t st, int bn);
 
 namespace {
 
@@ -103,6 +103,11 @@ void tc_release(fs_model* m) {
   m->tc_extras = nullptr;
 }
 
+// Output tile widths: 256 where the output is wide (fewer re-reads of the
+// activations per FLOP), 128 for the H-wide outputs (enough tiles for the SMs).
+static int bn_qkv(const Shape& s) { return s.qkv_dim() % 256 == 0 ? 256 : 128; }
+static int bn_gu(const Shape& s) { return s.I % 128 == 0 ? 256 : 128; }
+
 // Whether the tensor-core prefill covers this model's shape.
 static bool tc_shape_ok(const fs_model* m) {
   const Shape& s = m->s;
@@ -168,9 +173,10 @@ static fs_status tc_prepare(fs_model* m, cudaStream_t st) {
             static_cast<const __nv_bfloat16*>(Lw.w[pt.which]), n, pt.dst);
     }
     LayerMaps& mp = t->maps[l];
-    if (!make_tmap_16(&mp.qkv, wqkv, s.qkv_dim(), s.H, 128, false) ||
+    if (!make_tmap_16(&mp.qkv, wqkv, s.qkv_dim(), s.H, bn_qkv(s), false) ||
         !make_tmap_16(&mp.o, wo, s.H, s.q_dim(), 128, false) ||
-        !make_tmap_16(&mp.g, wg, s.I, s.H, 64, false) || !make_tmap_16(&mp.u, wu, s.I, s.H, 64, false) ||
+        !make_tmap_16(&mp.g, wg, s.I, s.H, bn_gu(s) / 2, false) ||
+        !make_tmap_16(&mp.u, wu, s.I, s.H, bn_gu(s) / 2, false) ||
         !make_tmap_16(&mp.d, wd, s.H, s.I, 128, false))
       return fail(FS_ERR_UNSUPPORTED, "the driver refused a TMA descriptor");
   }
@@ -216,7 +222,7 @@ fs_status layer_tc(fs_model* m, const fs_kv* kv, const RowMap& map, int rows, in
   FS_TRY(cudaGetLastError());
   FS_TRY(launch_gemm_tc(&t->a_xn_hi, split ? &t->a_xn_lo : nullptr, &mp.qkv, nullptr, rows,
                         s.qkv_dim(), s.H, 0, m->qkv, s.qkv_dim(), nullptr, nullptr, 0, m->err,
-                        m->num_sms, st));
+                        m->num_sms, st, bn_qkv(s)));
   FS_TRY(launch_qk_norm_rope_append(m->qkv, rows, map, s, Lw.q_norm, Lw.k_norm, m->rope, m->q,
                                     kvv, l, st));
   if (attention_tc_supported(s, kvv, map)) {
@@ -229,14 +235,14 @@ fs_status layer_tc(fs_model* m, const fs_kv* kv, const RowMap& map, int rows, in
     FS_TRY(cudaGetLastError());
   }
   FS_TRY(launch_gemm_tc(&t->a_o, nullptr, &mp.o, nullptr, rows, s.H, s.q_dim(), 1, m->h, s.H,
-                        nullptr, nullptr, 0, m->err, m->num_sms, st));
+                        nullptr, nullptr, 0, m->err, m->num_sms, st, 128));
   count_launches();
   rmsnorm_f16_kernel<<<rows, 256, 0, st>>>(m->h, s.H, Lw.ffn_norm, s.eps, t->xn_hi, nullptr);
   FS_TRY(cudaGetLastError());
   FS_TRY(launch_gemm_tc(&t->a_xn_hi, nullptr, &mp.g, &mp.u, rows, 2 * s.I, s.H, 2, nullptr, 0,
-                        t->act_hi, nullptr, s.I, m->err, m->num_sms, st));
+                        t->act_hi, nullptr, s.I, m->err, m->num_sms, st, bn_gu(s)));
   FS_TRY(launch_gemm_tc(&t->a_act, nullptr, &mp.d, nullptr, rows, s.H, s.I, 1, m->h, s.H, nullptr,
-                        nullptr, 0, m->err, m->num_sms, st));
+                        nullptr, 0, m->err, m->num_sms, st, 128));
 #undef FS_TRY
   return FS_OK;
 }
