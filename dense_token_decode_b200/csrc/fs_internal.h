@@ -103,6 +103,13 @@ cudaError_t launch_gemv(const float* x, int rows, int K, const void* W, const __
 cudaError_t launch_gemv_swiglu(const float* x, int rows, int K, const void* Wg, const __half* sg,
                                const void* Wu, const __half* su, int N, float* act,
                                cudaStream_t st);
+// Split-K weight streaming for 5..16 rows of bf16 weights (gemv_splitk.cu).
+bool gemv_splitk_ok(int rows, int K, const __half* scales);
+cudaError_t launch_gemv_splitk(const float* x, int rows, int K, const __nv_bfloat16* W, int N,
+                               float* out, int ldo, bool accumulate, cudaStream_t st);
+// Greedy id per row of fp32 logits [rows][V] (lowest id on exact ties).
+cudaError_t launch_argmax_rows(const float* logits, int rows, int V, int32_t* argmax,
+                               cudaStream_t st);
 cudaError_t launch_gemm_simt(const float* A, int M, int K, const void* W, const __half* scales,
                              int N, float* C, int ldc, bool accumulate, cudaStream_t st);
 cudaError_t launch_swiglu(const float* gu, int rows, int I, float* act, cudaStream_t st);

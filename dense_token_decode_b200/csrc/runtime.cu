@@ -69,7 +69,7 @@ namespace fs {
 void model_free_buffers(fs_model* m) {
   void* bufs[] = {m->rope, m->h,   m->xn,  m->qkv,     m->q,   m->o,       m->gu,
                   m->act,  m->xf,  m->tok, m->partial, m->err, m->gen_tok, m->scratch,
-                  m->attn_part};
+                  m->attn_part, m->lm_scratch};
   for (void* b : bufs)
     if (b) cudaFree(b);
   release_extras(m);
@@ -178,6 +178,7 @@ extern "C" fs_status fs_model_create(const fs_config* cfg, const fs_weights* w, 
       (st = dev_alloc(&m->q, R * s.q_dim(), "workspace")) != FS_OK ||
       (st = dev_alloc(&m->o, R * s.q_dim(), "workspace")) != FS_OK ||
       (st = dev_alloc(&m->attn_part, fs::attention_decode_part_floats(s), "workspace")) != FS_OK ||
+      (st = dev_alloc(&m->lm_scratch, (size_t)16 * s.V, "workspace")) != FS_OK ||
       (st = dev_alloc(&m->gu, R * 2 * s.I, "workspace")) != FS_OK ||
       (st = dev_alloc(&m->act, R * s.I, "workspace")) != FS_OK ||
       (st = dev_alloc(&m->xf, (size_t)fs::kMaxBatch * s.H, "workspace")) != FS_OK ||
@@ -363,6 +364,9 @@ namespace fs {
 static cudaError_t linear(const fs_model* m, const float* x, int rows, int K, int layer, Lin which,
                           int N, float* out, int ldo, bool acc, cudaStream_t st) {
   const LayerDev& L = m->layers[layer];
+  if (rows > 4 && gemv_splitk_ok(rows, K, L.s[which]))
+    return launch_gemv_splitk(x, rows, K, static_cast<const __nv_bfloat16*>(L.w[which]), N, out,
+                              ldo, acc, st);
   if (rows <= 16) return launch_gemv(x, rows, K, L.w[which], L.s[which], N, out, ldo, acc, st);
   return launch_gemm_simt(x, rows, K, L.w[which], L.s[which], N, out, ldo, acc, st);
 }
@@ -391,7 +395,7 @@ fs_status layer_general(fs_model* m, const fs_kv* kv, const RowMap& map, int row
   }
   FS_CUDA(linear(m, m->o, rows, qd, l, kWo, H, m->h, H, true, st));
   FS_CUDA(launch_rmsnorm(m->h, rows, H, Lw.ffn_norm, s.eps, m->xn, st));
-  if (rows <= 16) {
+  if (rows <= 16 && !(rows > 4 && gemv_splitk_ok(rows, H, Lw.s[kWg]))) {
     FS_CUDA(launch_gemv_swiglu(m->xn, rows, H, Lw.w[kWg], Lw.s[kWg], Lw.w[kWu], Lw.s[kWu], s.I,
                                m->act, st));
   } else {
@@ -430,8 +434,16 @@ fs_status forward_general(fs_model* m, const fs_kv* kv, const RowMap& map, int r
   const int nh = rows - head_first;
   if (nh > 0 && (logits || argmax)) {
     FS_CUDA(launch_rmsnorm(m->h + (size_t)head_first * H, nh, H, m->final_norm, s.eps, m->xf, st));
-    FS_CUDA(launch_lm_head(m->xf, nh, s, m->embed, logits, argmax, m->partial, m->n_part, m->err,
-                           st));
+    if (nh > 4 && gemv_splitk_ok(nh, H, nullptr)) {
+      // 5..16 rows: split-K streaming of the tied embedding into the logits
+      // (the caller's, or the model's scratch), then the greedy pass.
+      float* lg = logits ? logits : m->lm_scratch;
+      FS_CUDA(launch_gemv_splitk(m->xf, nh, H, m->embed, s.V, lg, s.V, false, st));
+      if (argmax) FS_CUDA(launch_argmax_rows(lg, nh, s.V, argmax, st));
+    } else {
+      FS_CUDA(launch_lm_head(m->xf, nh, s, m->embed, logits, argmax, m->partial, m->n_part,
+                             m->err, st));
+    }
   }
   return FS_OK;
 }

@@ -25,6 +25,7 @@ struct fs_model {
   float* q = nullptr;      // rotated queries [max_rows, nq*d]
   float* o = nullptr;      // attention output [max_rows, nq*d]
   float* attn_part = nullptr;  // split-KV attention partials (attention_decode.cu)
+  float* lm_scratch = nullptr; // logits of 5..16 rows when the caller passes none [16, V]
   float* gu = nullptr;     // gate||up [max_rows, 2I]
   float* act = nullptr;    // SwiGLU output [max_rows, I]
   float* xf = nullptr;     // final-normed rows [64, H]
