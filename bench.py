@@ -47,6 +47,12 @@ DECODE_STEPS = 256
 PREFILL_S = 2048
 SEED = 1
 
+# DRAM bytes (read + write) of one decode-kernel launch, from the ncu capture
+# in profiles/decode_mega_qwen3_0p6b_bs1.md (batch 1, context of 53 positions).
+# Re-take it whenever the decode kernel changes.
+DECODE_TRAFFIC_BYTES = 1_198_254_000 + 3_646_720
+DECODE_TRAFFIC_CONTEXT = 53
+
 
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -288,6 +294,10 @@ def run_ours(args, world, rank, local):
     per_step, weight_bytes = decode_bytes(shape, ctx)
     step_s = dec_ms / 1e3 / DECODE_STEPS
     achieved = statistics.mean(per_step) / step_s / 1e9
+    # the captured launch's traffic, moved to the job's mean context (KV grows by
+    # one position's K and V per step)
+    kv_tok = shape.n_layers * 2 * shape.n_kv_heads * shape.head_dim * 2
+    traffic = DECODE_TRAFFIC_BYTES + kv_tok * (statistics.mean(ctx) - DECODE_TRAFFIC_CONTEXT)
 
     # End to end: fs_greedy with host buffers (prompt H2D, ids D2H inside the call).
     host_prompt = prompt.cpu().pin_memory()
@@ -408,7 +418,8 @@ def run_ours(args, world, rank, local):
             "dtype": "bf16 weights, fp32 activations", "data": "synthetic",
             "config": workload_config(),
             "roofline": {"bound": "hbm", "kernel": "decode forward step", "achieved": achieved,
-                         "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                         "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                         "traffic": traffic,
                          "bytes_per_step": statistics.mean(per_step),
                          "weight_bytes": weight_bytes, "step_us": step_s * 1e6,
                          "peak_source": peak_src},

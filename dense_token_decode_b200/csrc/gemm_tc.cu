@@ -35,6 +35,7 @@ struct Params {
   int M, N, K;       // N = output columns of D (SwiGLU: 2 x act columns per tile)
   int kind;
   int a_terms;       // 1 or 2
+  int lo_col0;       // with 2 terms: only output tiles from this column on use A_lo
   int n_tiles_m, n_tiles_n;
   int stages;
   float* out;        // kStore: fp32 [M, ldo]; kResidual: fp32 [M, ldo] (+=)
@@ -109,9 +110,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait(&empty[s], ph ^ 1, p.err);
           if (!ok) break;
           unsigned char* st = smem + s * stage_bytes;
-          mbar_expect_tx(&full[s], stage_bytes);
+          const bool two = p.a_terms == 2 && nt * BN >= p.lo_col0;
+          mbar_expect_tx(&full[s], stage_bytes - (p.a_terms == 2 && !two ? kTileBytes : 0));
           tma_load_2d(st, &map_a, kb * BK, mt * BM, &full[s]);
-          if (p.a_terms == 2) tma_load_2d(st + kTileBytes, &map_a_lo, kb * BK, mt * BM, &full[s]);
+          if (two) tma_load_2d(st + kTileBytes, &map_a_lo, kb * BK, mt * BM, &full[s]);
           unsigned char* sb = st + p.a_terms * kTileBytes;
           if (swiglu) {
             // 64 gate rows then 64 up rows of the same act columns
@@ -142,6 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const uint32_t d_tmem = tmem + abuf * BN;
+        const bool two = p.a_terms == 2 && (t / p.n_tiles_m) * BN >= p.lo_col0;
         for (int kb = 0; kb < kblocks && ok; ++kb) {
           ok = mbar_wait(&full[s], ph, p.err);
           if (!ok) break;
@@ -152,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t bdesc = smem_desc(sb + k * 32);
             mma_f16(d_tmem, smem_desc(st + k * 32), bdesc, idesc, (kb > 0 || k > 0) ? 1u : 0u);
-            if (p.a_terms == 2) mma_f16(d_tmem, smem_desc(st + kTileBytes + k * 32), bdesc, idesc, 1u);
+            if (two) mma_f16(d_tmem, smem_desc(st + kTileBytes + k * 32), bdesc, idesc, 1u);
           }
           mma_commit(&empty[s]);  // the stage is free once these MMAs have read it
           ++counts[1];
@@ -299,7 +302,7 @@ template <int BN>
 cudaError_t launch_bn(const CUtensorMap* a, const CUtensorMap* a_lo, const CUtensorMap* b,
                       const CUtensorMap* b2, int M, int N, int K, int kind, float* out, int ldo,
                       __half* act_hi, __half* act_lo, int act_ld, int* err, int num_sms,
-                      cudaStream_t st) {
+                      cudaStream_t st, int lo_col0) {
   static bool attr_done = false;
   if (!attr_done) {
     cudaFuncSetAttribute(tc::gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -312,6 +315,7 @@ cudaError_t launch_bn(const CUtensorMap* a, const CUtensorMap* a_lo, const CUten
   p.K = K;
   p.kind = kind;
   p.a_terms = a_lo ? 2 : 1;
+  p.lo_col0 = lo_col0;
   p.n_tiles_m = (M + tc::BM - 1) / tc::BM;
   p.n_tiles_n = N / BN;
   const int stage_bytes = p.a_terms * tc::kTileBytes + BN * tc::BK * 2;
@@ -335,16 +339,17 @@ cudaError_t launch_bn(const CUtensorMap* a, const CUtensorMap* a_lo, const CUten
 // Launch one tensor-core GEMM with BN-wide output tiles (128 or 256; the B
 // tensor maps must have boxes of BN rows, BN / 2 for kSwiGLU). a_lo may be
 // null (one fp16 term). For kSwiGLU b2 is the up matrix and N counts
-// gate+up columns (2 * I).
+// gate+up columns (2 * I). With a_lo, output tiles from column lo_col0 on
+// add the second term (0: all tiles).
 cudaError_t launch_gemm_tc(const CUtensorMap* a, const CUtensorMap* a_lo, const CUtensorMap* b,
                            const CUtensorMap* b2, int M, int N, int K, int kind, float* out,
                            int ldo, __half* act_hi, __half* act_lo, int act_ld, int* err,
-                           int num_sms, cudaStream_t st, int bn) {
+                           int num_sms, cudaStream_t st, int bn, int lo_col0) {
   if (bn == 256)
     return launch_bn<256>(a, a_lo, b, b2, M, N, K, kind, out, ldo, act_hi, act_lo, act_ld, err,
-                          num_sms, st);
+                          num_sms, st, lo_col0);
   return launch_bn<128>(a, a_lo, b, b2, M, N, K, kind, out, ldo, act_hi, act_lo, act_ld, err,
-                        num_sms, st);
+                        num_sms, st, lo_col0);
 }
 
 }  // namespace fs

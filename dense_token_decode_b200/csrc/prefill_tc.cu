@@ -17,7 +17,7 @@ namespace fs {
 cudaError_t launch_gemm_tc(const CUtensorMap* a, const CUtensorMap* a_lo, const CUtensorMap* b,
                            const CUtensorMap* b2, int M, int N, int K, int kind, float* out,
                            int ldo, __half* act_hi, __half* act_lo, int act_ld, int* err,
-                           int num_sms, cudaStream_t st, int bn);
+                           int num_sms, cudaStream_t st, int bn, int lo_col0 = 0);
 
 namespace {
 
@@ -207,6 +207,9 @@ fs_status layer_tc(fs_model* m, const fs_kv* kv, const RowMap& map, int rows, in
   const LayerMaps& mp = t->maps[l];
   const KVView kvv = kv_view(kv);
   const bool split = m->prefill_split != 0;
+  // The second operand term matters where the output is rounded to bf16 in
+  // the cache (the K and V columns); the Q columns use one fp16 term.
+  const int split_from = s.q_dim() % bn_qkv(s) == 0 ? s.q_dim() : 0;
   cudaError_t e;
 #define FS_TRY(x)                                                     \
   do {                                                                \
@@ -222,7 +225,7 @@ fs_status layer_tc(fs_model* m, const fs_kv* kv, const RowMap& map, int rows, in
   FS_TRY(cudaGetLastError());
   FS_TRY(launch_gemm_tc(&t->a_xn_hi, split ? &t->a_xn_lo : nullptr, &mp.qkv, nullptr, rows,
                         s.qkv_dim(), s.H, 0, m->qkv, s.qkv_dim(), nullptr, nullptr, 0, m->err,
-                        m->num_sms, st, bn_qkv(s)));
+                        m->num_sms, st, bn_qkv(s), split_from));
   FS_TRY(launch_qk_norm_rope_append(m->qkv, rows, map, s, Lw.q_norm, Lw.k_norm, m->rope, m->q,
                                     kvv, l, st));
   if (attention_tc_supported(s, kvv, map)) {
