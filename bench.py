@@ -162,12 +162,22 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The slowest rank's time (the job's time): an all-reduce MAX over the
+    process group (on the GPU under NCCL, on the host under gloo)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, world: int, ms_this_rank: float) -> tuple[float, float]:
+    """Whole-job tokens/s of N independent replicas: every rank's tokens over
+    the slowest rank's time. Returns (value, max ms)."""
+    ms_max = max_over_ranks(ms_this_rank, world)
+    return tokens_per_rank * world / (ms_max / 1e3), ms_max
 
 
 # --------------------------------------------------------------------------- CPU oracle
@@ -284,10 +294,8 @@ def run_ours(args, world, rank, local):
     launches = abi.fs_debug_kernel_launches() - l0
     barrier(world)
     ms = t0.elapsed_time(t1)
-    ms_max = max_over_ranks(ms, world)
+    value, ms_max = job_throughput(DECODE_STEPS * args.steps, world, ms)
     dec_ms = sum(a.elapsed_time(b) for a, b in dec_ev) / args.steps
-    tokens_all = DECODE_STEPS * args.steps * world
-    value = tokens_all / (ms_max / 1e3)
 
     hbm, bf16, bf16_s, peak_src = peaks()
     ctx = [PROMPT + i + 1 for i in range(DECODE_STEPS)]  # context incl. the new position
@@ -321,8 +329,7 @@ def run_ours(args, world, rank, local):
         e2e_job()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_val = DECODE_STEPS * args.steps * world / (e2e_ms / 1e3)
+    e2e_val, _ = job_throughput(DECODE_STEPS * args.steps, world, e0.elapsed_time(e1))
     assert n_out.value == DECODE_STEPS
 
     # Prefill of 2048 tokens.

@@ -269,9 +269,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int c = un >> 3, u = un & 7;
         float x[8];
         if (live) {
+          // the softmax scale (log2 e / sqrt d) is folded into Q
           const float4 a = src[un * 2], b4 = src[un * 2 + 1];
-          x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-          x[4] = b4.x; x[5] = b4.y; x[6] = b4.z; x[7] = b4.w;
+          const float sc = p.scale_log2;
+          x[0] = a.x * sc; x[1] = a.y * sc; x[2] = a.z * sc; x[3] = a.w * sc;
+          x[4] = b4.x * sc; x[5] = b4.y * sc; x[6] = b4.z * sc; x[7] = b4.w * sc;
         } else {
 #pragma unroll
           for (int i = 0; i < 8; ++i) x[i] = 0.f;
@@ -302,9 +304,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_before();
         mbar_arrive(&s_free[b]);
         const int lim = qp - j * kKTile - half * 32;  // columns c <= lim are visible
+        if (__all_sync(0xffffffffu, lim >= 31)) {  // below the diagonal: nothing masked
 #pragma unroll
-        for (int c = 0; c < 32; ++c)
-          x[c] = c <= lim ? __uint_as_float(ra[c]) * p.scale_log2 : -INFINITY;
+          for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(ra[c]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) x[c] = c <= lim ? __uint_as_float(ra[c]) : -INFINITY;
+        }
         float mx4[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
         for (int c = 4; c < 32; c += 4)

@@ -36,6 +36,7 @@ struct Params {
   int kind;
   int a_terms;       // 1 or 2
   int lo_col0;       // with 2 terms: only output tiles from this column on use A_lo
+  int ksplit;        // K split into this many parts per tile (kResidual only: atomic adds)
   int n_tiles_m, n_tiles_n;
   int stages;
   float* out;        // kStore: fp32 [M, ldo]; kResidual: fp32 [M, ldo] (+=)
@@ -96,6 +97,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_base_s;
 
   const int n_tiles = p.n_tiles_m * p.n_tiles_n;
+  const int n_units = n_tiles * p.ksplit;  // (tile, K part) work units
   const int kblocks = p.K / BK;
   const bool swiglu = p.kind == kSwiGLU;
 
@@ -104,9 +106,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const int t = u / p.ksplit, kp = u % p.ksplit;
         const int mt = t % p.n_tiles_m, nt = t / p.n_tiles_m;
-        for (int kb = 0; kb < kblocks && ok; ++kb) {
+        const int kb0 = kblocks * kp / p.ksplit, kb1 = kblocks * (kp + 1) / p.ksplit;
+        for (int kb = kb0; kb < kb1 && ok; ++kb) {
           ok = mbar_wait(&empty[s], ph ^ 1, p.err);
           if (!ok) break;
           unsigned char* st = smem + s * stage_bytes;
@@ -137,7 +141,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t ph = 0;
       int tcount = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tcount) {
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++tcount) {
+        const int t = u / p.ksplit, kp = u % p.ksplit;
+        const int kb0 = kblocks * kp / p.ksplit, kb1 = kblocks * (kp + 1) / p.ksplit;
         const int abuf = tcount & 1;
         const uint32_t aph = (tcount >> 1) & 1;
         ok = mbar_wait(&acc_empty[abuf], aph ^ 1, p.err);
@@ -145,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const uint32_t d_tmem = tmem + abuf * BN;
         const bool two = p.a_terms == 2 && (t / p.n_tiles_m) * BN >= p.lo_col0;
-        for (int kb = 0; kb < kblocks && ok; ++kb) {
+        for (int kb = kb0; kb < kb1 && ok; ++kb) {
           ok = mbar_wait(&full[s], ph, p.err);
           if (!ok) break;
           asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -154,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t bdesc = smem_desc(sb + k * 32);
-            mma_f16(d_tmem, smem_desc(st + k * 32), bdesc, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+            mma_f16(d_tmem, smem_desc(st + k * 32), bdesc, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
             if (two) mma_f16(d_tmem, smem_desc(st + kTileBytes + k * 32), bdesc, idesc, 1u);
           }
           mma_commit(&empty[s]);  // the stage is free once these MMAs have read it
@@ -177,7 +183,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;
     const int row_in_tile = quad * 32 + lane;
     int tcount = 0;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tcount) {
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++tcount) {
+      const int t = u / p.ksplit;
       const int mt = t % p.n_tiles_m, nt = t / p.n_tiles_m;
       const int abuf = tcount & 1;
       const uint32_t aph = (tcount >> 1) & 1;
@@ -192,7 +199,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(taddr + c0, r);
           if (!live) continue;
           float* o = p.out + (size_t)m * p.ldo + nt * BN + c0;
-          if (p.kind == kResidual) {
+          if (p.kind == kResidual && p.ksplit > 1) {
+            // several K parts add into the same rows: vector atomics
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+              atomicAdd(reinterpret_cast<float4*>(o + j),
+                        make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                                    __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3])));
+          } else if (p.kind == kResidual) {
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
               float4 h = *reinterpret_cast<float4*>(o + j);
@@ -318,6 +332,9 @@ cudaError_t launch_bn(const CUtensorMap* a, const CUtensorMap* a_lo, const CUten
   p.lo_col0 = lo_col0;
   p.n_tiles_m = (M + tc::BM - 1) / tc::BM;
   p.n_tiles_n = N / BN;
+  // Residual GEMMs with fewer tiles than SMs split K in two (atomic adds).
+  p.ksplit = (kind == tc::kResidual && p.n_tiles_m * p.n_tiles_n < num_sms && (K / tc::BK) >= 8)
+                 ? 2 : 1;
   const int stage_bytes = p.a_terms * tc::kTileBytes + BN * tc::BK * 2;
   p.stages = std::min(8, (232448 - 2048) / stage_bytes);
   p.out = out;
@@ -327,8 +344,8 @@ cudaError_t launch_bn(const CUtensorMap* a, const CUtensorMap* a_lo, const CUten
   p.act_ld = act_ld;
   p.err = err;
   const size_t smem = 1024 + (size_t)p.stages * stage_bytes + 1024;
-  const int tiles = p.n_tiles_m * p.n_tiles_n;
-  const int grid = std::min(tiles, num_sms);
+  const int units = p.n_tiles_m * p.n_tiles_n * p.ksplit;
+  const int grid = std::min(units, num_sms);
   count_launches();
   tc::gemm_tc_kernel<BN><<<grid, tc::kThreads, smem, st>>>(p, *a, a_lo ? *a_lo : *a, *b,
                                                            b2 ? *b2 : *b);
