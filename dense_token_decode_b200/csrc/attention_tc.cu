@@ -15,10 +15,10 @@
 // updated lazily (only when it grows by more than 2^8 in the exp2 domain),
 // which keeps every P below 256 and the final O / l exact up to rounding.
 //
-// Warp roles (320 threads): warp 0 TMA producer; warp 1 TMEM owner and MMA
-// issuer (one lane); warps 2-9 softmax, two warps per TMEM lane quadrant
-// (= warp % 4): each thread owns one query row and half of the columns, then
-// the epilogue writes its half of O / l as fp16.
+// Warp roles (576 threads): warp 0 TMA producer; warp 1 TMEM owner and MMA
+// issuer (one lane); warps 2-17 softmax, four warps per TMEM lane quadrant
+// (= warp % 4): each thread owns one query row and a quarter of the score
+// and O columns, then the epilogue writes its quarter of O / l as fp16.
 //
 // Requirement: KV slots past a sequence's length hold finite values (they are
 // multiplied by exact zeros); the cache is zeroed when allocated and only ever
@@ -33,7 +33,9 @@ namespace attn_tc {
 
 using namespace tc;
 
-constexpr int kSoftWarps = 8;
+constexpr int kSoftWarps = 16;
+constexpr int kGroups = kSoftWarps / 4;  // warps sharing a TMEM lane quadrant
+constexpr int kSCols = 64 / kGroups;     // score columns of a page per warp
 constexpr int kSoft = kSoftWarps * 32;
 constexpr int kThreads = 64 + kSoft;
 constexpr int kQTile = 128;
@@ -58,7 +60,7 @@ struct Layout {
   static constexpr int kPageBytes = kChunks * 8192;  // one K or V page: 64 rows x 128 B per chunk
   static constexpr int kNK = 3, kNV = 2;              // K and V ring stages
   static constexpr int kKVBytes = (kNK + kNV) * kPageBytes;
-  static constexpr int kMiscBytes = 256 + 3 * 2 * kQTile * 4;  // barriers, row max / sum
+  static constexpr int kMiscBytes = 256 + 3 * kGroups * kQTile * 4;  // barriers, row max / sum
   static constexpr int kSmemBytes = 1024 + kQBytes + kPBytes + kKVBytes + kMiscBytes;
   static constexpr int kTmemCols = 256;                // S[2] (64 cols each) + O (d cols)
   static constexpr int kOCol = 128;
@@ -112,9 +114,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = o_full + 1;
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(drain + 1);
   uint32_t* counts = tmem_base_s + 1;  // K pages loaded / waited, V pages loaded / waited
-  float(*red_max)[2][kQTile] = reinterpret_cast<float(*)[2][kQTile]>(
-      reinterpret_cast<unsigned char*>(k_full) + 256);  // [page parity][half][row]
-  float(*red_sum)[kQTile] = reinterpret_cast<float(*)[kQTile]>(red_max + 2);  // [half][row]
+  float(*red_max)[kGroups][kQTile] = reinterpret_cast<float(*)[kGroups][kQTile]>(
+      reinterpret_cast<unsigned char*>(k_full) + 256);  // [page parity][group][row]
+  float(*red_sum)[kQTile] = reinterpret_cast<float(*)[kQTile]>(red_max + 2);  // [group][row]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = p.n_qt - 1 - (int)blockIdx.x / p.nq;
@@ -153,7 +155,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
-    if (lane == 0) {
+    // Lane 0 streams the K pages, lane 1 the V pages, each at the pace of its
+    // own ring: the next K page never waits for a V slot.
+    if (lane < 2) {
+      const bool is_k = lane == 0;
+      const int NS = is_k ? NK : NV;
+      uint64_t* fullb = is_k ? k_full : v_full;
+      uint64_t* emptyb = is_k ? k_empty : v_empty;
+      unsigned char* ring = is_k ? sK : sV;
+      const CUtensorMap* map = is_k ? &map_k : &map_v;
       for (int j = 0; j < nt; ++j) {
         int page = p.block_table[(size_t)p.seq * p.pages_per_seq + j];
         if (page < 0 || page >= p.n_pages) {
@@ -161,19 +171,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           page = 0;
         }
         const int row = ((p.layer * p.n_pages + page) * p.nkv + g) * kKTile;
-        const int sk = j % NK, sv = j % NV;
-        if (!mbar_wait(&k_empty[sk], ((j / NK) & 1) ^ 1, p.err)) break;
-        mbar_expect_tx(&k_full[sk], Lay::kPageBytes);
+        const int st = j % NS;
+        if (!mbar_wait(&emptyb[st], ((j / NS) & 1) ^ 1, p.err)) break;
+        mbar_expect_tx(&fullb[st], Lay::kPageBytes);
 #pragma unroll
         for (int c = 0; c < Lay::kChunks; ++c)
-          tma_load_2d(sK + sk * Lay::kPageBytes + c * 8192, &map_k, c * 64, row, &k_full[sk]);
-        ++counts[0];
-        if (!mbar_wait(&v_empty[sv], ((j / NV) & 1) ^ 1, p.err)) break;
-        mbar_expect_tx(&v_full[sv], Lay::kPageBytes);
-#pragma unroll
-        for (int c = 0; c < Lay::kChunks; ++c)
-          tma_load_2d(sV + sv * Lay::kPageBytes + c * 8192, &map_v, c * 64, row, &v_full[sv]);
-        ++counts[2];
+          tma_load_2d(ring + st * Lay::kPageBytes + c * 8192, map, c * 64, row, &fullb[st]);
+        ++counts[is_k ? 0 : 2];
       }
     }
   } else if (warp == 1) {
@@ -234,38 +238,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------------- softmax warps
-    // Two warps per TMEM lane quadrant: `half` 0 owns score columns 0..31 of
-    // each page and O columns 0..d/2-1, `half` 1 the rest. The row maximum is
-    // combined through shared memory (one named barrier per quadrant pair).
+    // kGroups warps per TMEM lane quadrant: warp group g owns score columns
+    // [g * kSCols, (g + 1) * kSCols) of each page and the same share of the O
+    // columns. The row maximum is combined through shared memory (one reducing
+    // barrier of the quadrant's warps per page).
     const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int grp = (warp - 2) >> 2;
     const int row = quad * 32 + lane;
     const int r = q0 + row;
     const bool live = r < p.rows;
     const int qp = p.pos0 + (live ? r : p.rows - 1);  // position of this query
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    constexpr int kOHalf = D / 2;
+    constexpr int kOCols = D / kGroups;           // O columns per warp
+    constexpr int kOC = kOCols < 32 ? kOCols : 32;  // TMEM columns per load
     auto pair_sync = [&]() {
-      asm volatile("bar.sync %0, 64;" ::"r"(1 + quad) : "memory");
+      asm volatile("bar.sync %0, %1;" ::"r"(1 + quad), "n"(32 * kGroups) : "memory");
     };
     auto pair_or = [&](int id, bool v) -> bool {
       uint32_t r;
       asm volatile(
-          "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, 64, p;\n"
+          "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, %3, p;\n"
           " selp.u32 %0, 1, 0, q;\n}\n"
           : "=r"(r)
-          : "r"((uint32_t)v), "r"(id)
+          : "r"((uint32_t)v), "r"(id), "n"(32 * kGroups)
           : "memory");
       return r != 0;
     };
 
-    // Q row -> two bf16 terms in swizzled K-major layout (this warp's half of the units).
+    // Q row -> two bf16 terms in swizzled K-major layout (this warp's share of the units).
     {
       const float4* src = reinterpret_cast<const float4*>(p.q + ((size_t)r * p.nq + h) * D);
       constexpr int kUnits = Lay::kChunks * 8;  // 16-byte units of a row
 #pragma unroll
-      for (int uu = 0; uu < kUnits / 2; ++uu) {
-        const int un = half * (kUnits / 2) + uu;
+      for (int uu = 0; uu < kUnits / kGroups; ++uu) {
+        const int un = grp * (kUnits / kGroups) + uu;
         const int c = un >> 3, u = un & 7;
         float x[8];
         if (live) {
@@ -294,41 +300,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     // warp skips the work but still takes part).
     for (int j = 0; j < nt; ++j) {
       const int b = j & 1;
-      float x[32];
+      float x[kSCols];
       float mx = -INFINITY;
       if (ok) ok = mbar_wait_warp(&s_full[b], (j >> 1) & 1, p.err);
       if (ok) {
         fence_after();
-        uint32_t ra[32];
-        tmem_ld32(tmem + lane_off + b * kKTile + half * 32, ra);
+        uint32_t ra[kSCols];
+        tmem_ld(tmem + lane_off + b * kKTile + grp * kSCols, ra);
         fence_before();
         mbar_arrive(&s_free[b]);
-        const int lim = qp - j * kKTile - half * 32;  // columns c <= lim are visible
-        if (__all_sync(0xffffffffu, lim >= 31)) {  // below the diagonal: nothing masked
+        const int lim = qp - j * kKTile - grp * kSCols;  // columns c <= lim are visible
+        if (__all_sync(0xffffffffu, lim >= kSCols - 1)) {  // below the diagonal: nothing masked
 #pragma unroll
-          for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(ra[c]);
+          for (int c = 0; c < kSCols; ++c) x[c] = __uint_as_float(ra[c]);
         } else {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) x[c] = c <= lim ? __uint_as_float(ra[c]) : -INFINITY;
+          for (int c = 0; c < kSCols; ++c) x[c] = c <= lim ? __uint_as_float(ra[c]) : -INFINITY;
         }
         float mx4[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-        for (int c = 4; c < 32; c += 4)
+        for (int c = 4; c < kSCols; c += 4)
 #pragma unroll
           for (int i = 0; i < 4; ++i) mx4[i] = fmaxf(mx4[i], x[c + i]);
         mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       }
-      red_max[b][half][row] = mx;
+      red_max[b][grp][row] = mx;
       if (pair_or(1 + quad, !ok)) {
         ok = false;
         break;
       }
-      mx = fmaxf(mx, red_max[b][half ^ 1][row]);
+#pragma unroll
+      for (int g2 = 0; g2 < kGroups; ++g2) mx = fmaxf(mx, red_max[b][g2][row]);
       const float m_new = fmaxf(m, mx);
       if (j == 0) {
         m = m_new;  // key 0 is visible to every row: finite
       } else if (__any_sync(0xffffffffu, m_new > m + kRescaleLog2)) {
-        // Both warps of the pair see the same rows and maxima: same decision.
+        // The quadrant's warps see the same rows and maxima: same decision.
         const float alpha = exp2f(m - m_new);
         // O may only be rescaled once the previous P V has landed in it.
         if (!mbar_wait_warp(&p_free[(j - 1) & 1], ((j - 1) >> 1) & 1, p.err)) {
@@ -337,19 +344,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_after();
 #pragma unroll 1
-        for (int c0 = half * kOHalf; c0 < (half + 1) * kOHalf; c0 += 32) {
-          uint32_t o[32];
-          tmem_ld32(tmem + lane_off + Lay::kOCol + c0, o);
+        for (int c0 = grp * kOCols; c0 < (grp + 1) * kOCols; c0 += kOC) {
+          uint32_t o[kOC];
+          tmem_ld(tmem + lane_off + Lay::kOCol + c0, o);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-          tmem_st32(tmem + lane_off + Lay::kOCol + c0, o);
+          for (int c = 0; c < kOC; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+          tmem_st(tmem + lane_off + Lay::kOCol + c0, o);
         }
         l *= alpha;
         m = m_new;
       }
       float sm4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 32; c += 4)
+      for (int c = 0; c < kSCols; c += 4)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           x[c + i] = exp2f(x[c + i] - m);
@@ -363,11 +370,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       unsigned char* pb = sP + b * 2 * 16384;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < kSCols / 8; ++u) {
         uint4 hi, lo;
         split8(x + u * 8, hi, lo);
-        *reinterpret_cast<uint4*>(pb + swz(row, half * 4 + u)) = hi;
-        *reinterpret_cast<uint4*>(pb + 16384 + swz(row, half * 4 + u)) = lo;
+        *reinterpret_cast<uint4*>(pb + swz(row, grp * (kSCols / 8) + u)) = hi;
+        *reinterpret_cast<uint4*>(pb + 16384 + swz(row, grp * (kSCols / 8) + u)) = lo;
       }
       fence_proxy_async();
       fence_before();
@@ -375,21 +382,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // Full row sum from the two halves (uniform control flow for the barrier:
     // a timed-out warp still takes part).
-    red_sum[half][row] = l;
+    red_sum[grp][row] = l;
     pair_sync();
-    const float l_row = l + red_sum[half ^ 1][row];
+    float l_row = 0.f;
+#pragma unroll
+    for (int g2 = 0; g2 < kGroups; ++g2) l_row += red_sum[g2][row];
     if (ok) ok = mbar_wait_warp(o_full, 0, p.err);
     if (ok) {
       fence_after();
       const float inv = 1.f / l_row;
       __half* dst = p.o + ((size_t)r * p.nq + h) * D;
 #pragma unroll 1
-      for (int c0 = half * kOHalf; c0 < (half + 1) * kOHalf; c0 += 32) {
-        uint32_t o[32];
-        tmem_ld32(tmem + lane_off + Lay::kOCol + c0, o);
+      for (int c0 = grp * kOCols; c0 < (grp + 1) * kOCols; c0 += kOC) {
+        uint32_t o[kOC];
+        tmem_ld(tmem + lane_off + Lay::kOCol + c0, o);
         if (live) {
 #pragma unroll
-          for (int c = 0; c < 32; c += 8) {
+          for (int c = 0; c < kOC; c += 8) {
             __align__(16) __half v[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) v[i] = __float2half_rn(__uint_as_float(o[c + i]) * inv);
