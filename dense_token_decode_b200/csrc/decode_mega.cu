@@ -132,19 +132,6 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// As mbar_test, but a thread whose phase is not complete sleeps (up to
-// hint_ns) instead of returning at once, so waiting warps leave the issue
-// slots to the warps that compute; it wakes when the phase completes.
-__device__ __forceinline__ bool mbar_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(su32(bar)), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
 __device__ __forceinline__ uint64_t evict_first_policy() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -396,7 +383,7 @@ struct Producer {
     const int s = stage;
     unsigned long long t0 = 0;
     int spins = 0;
-    while (!mbar_wait_hint(&r.empty[s], parity, 20000)) {
+    while (!mbar_test(&r.empty[s], parity)) {
       // The clock only starts after many failed polls: reading it is not free.
       if ((++spins & 15) == 0) {
         if (t0 == 0) t0 = now_ns();
@@ -531,7 +518,7 @@ struct Consumer {
     // copy's bytes visible to it); the give-up decision is lane 0's, so the
     // warp stays converged for the shuffles that follow.
     while (true) {
-      const bool ok = quit || mbar_wait_hint(&r.full[s], parity, 20000);
+      const bool ok = quit || mbar_test(&r.full[s], parity);
       if (__all_sync(0xffffffffu, ok)) break;
       if ((++spins & 15) == 0) {
         int bad = 0;
