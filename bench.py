@@ -14,6 +14,8 @@ Also reported:
 * ``prefill``: a 2048-token prefill, tokens/s and TFLOP/s against bf16 peak;
 * ``batched_decode``: batch 16 with 8192 pre-filled KV positions per sequence,
   tokens/s against HBM bandwidth (weights + KV bytes per step);
+* ``q8_0_decode``: batch-1 decode with Q8_0 linear weights, tokens/s against
+  HBM bandwidth (34 bytes per 32 linear weights);
 * ``e2e``: the same job through ``fs_greedy`` with host buffers (prompt in,
   ids out, copies inside the timed region);
 * ``cpu_baseline``: the CPU oracle on a bounded sample of the same job.
@@ -62,12 +64,14 @@ def peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def decode_bytes(shape, ctx_lens):
+def decode_bytes(shape, ctx_lens, q8=False):
     """Algorithmic HBM bytes of one batch-1 decode step at each context length:
     every weight once (linear + tied embedding/LM head + norms) + the KV read
-    (all positions incl. the new one) + the KV write of the new position."""
+    (all positions incl. the new one) + the KV write of the new position.
+    Q8_0 linear weights take 34 bytes per 32 (int8 codes + one fp16 scale)."""
     from dense_token_decode_b200.synth import LINEAR_NAMES, linear_shape
-    lin = sum(a * b for a, b in (linear_shape(shape, n) for n in LINEAR_NAMES)) * 2
+    n_lin = sum(a * b for a, b in (linear_shape(shape, n) for n in LINEAR_NAMES))
+    lin = n_lin * 34 // 32 if q8 else n_lin * 2
     norms = (2 * shape.hidden + 2 * shape.head_dim) * 2
     weights = shape.n_layers * (lin + norms) + shape.vocab * shape.hidden * 2 + shape.hidden * 2
     kv_tok = shape.n_layers * 2 * shape.n_kv_heads * shape.head_dim * 2
@@ -363,6 +367,47 @@ def run_ours(args, world, rank, local):
                                           "flops": flops, "peak_source": peak_src}}
         kvp.close()
 
+    # Q8_0 decode at batch 1: the same job shape with Q8_0 linear weights
+    # (embedding / LM head bf16), 64 greedy steps after the 8-token prompt.
+    q8r = None
+    if not args.no_q8:
+        wq = synth.model_weights(shape, 4, "q8_0")
+        mq = Model(shape, wq, dev, max_pos=1024)
+        del wq
+        kvq = mq.kv(1, PROMPT + 80)
+        qgen = torch.zeros(72, dtype=torch.int32, device=dev)
+        qprompt = synth.token_ids(PROMPT, shape.vocab, seed=4).to(dev)
+
+        def qjob(n):
+            kvq.set_length(0, 0)
+            mq.prefill(kvq, 0, qprompt, None, qgen[0:1])
+            for i in range(n):
+                mq.decode_step(kvq, [0], qgen[i:i + 1], None, qgen[i + 1:i + 2])
+
+        qjob(8)
+        qjob(8)
+        torch.cuda.synchronize(dev)
+        kvq.set_length(0, 0)
+        mq.prefill(kvq, 0, qprompt, None, qgen[0:1])
+        q0 = torch.cuda.Event(enable_timing=True)
+        q1 = torch.cuda.Event(enable_timing=True)
+        QSTEPS = 64
+        q0.record(stream)
+        for i in range(QSTEPS):
+            mq.decode_step(kvq, [0], qgen[i:i + 1], None, qgen[i + 1:i + 2])
+        q1.record(stream)
+        torch.cuda.synchronize(dev)
+        qms = q0.elapsed_time(q1) / QSTEPS
+        qbytes, _ = decode_bytes(shape, [PROMPT + i + 1 for i in range(QSTEPS)], q8=True)
+        qach = statistics.mean(qbytes) / (qms / 1e3) / 1e9
+        q8r = {"value": 1e3 / qms, "unit": "tok/s", "ms_per_step": qms,
+               "workload": f"batch 1, Q8_0 linear weights, 8-token prompt + {QSTEPS} decode steps",
+               "roofline": {"bound": "hbm", "achieved": qach, "peak": hbm, "unit": "GB/s",
+                            "frac": qach / hbm, "bytes_per_step": statistics.mean(qbytes),
+                            "peak_source": peak_src}}
+        kvq.close()
+        mq.close()
+
     # Batched decode: 16 sequences, each with 8192 pre-filled N(0,1) bf16 K/V
     # positions, 32 greedy steps (ids stay on the device).
     bat = None
@@ -436,6 +481,7 @@ def run_ours(args, world, rank, local):
             "clocks": clocks.summary(),
             "prefill": pre,
             "batched_decode": bat,
+            "q8_0_decode": q8r,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line))
@@ -452,6 +498,7 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-batched", action="store_true")
+    ap.add_argument("--no-q8", action="store_true")
     ap.add_argument("--cpu-steps", type=int, default=16)
     args = ap.parse_args()
     world, rank, local = dist_setup(args)

@@ -28,3 +28,12 @@ def test_prefill_flops_2048():
     attn = s.n_layers * s.n_q_heads * 4 * s.head_dim * S * (S + 1) // 2
     head = 2 * s.hidden * s.vocab
     assert bench.prefill_flops(s, S) == lin + attn + head == 2_285_468_647_424
+
+
+def test_q8_0_decode_bytes():
+    s = synth.QWEN3_0P6B
+    _, weights = bench.decode_bytes(s, [1], q8=True)
+    n_lin = s.n_layers * 15_728_640
+    # 32 int8 codes + one fp16 scale per 32 weights; the tied embedding stays bf16
+    assert weights == n_lin * 34 // 32 + s.vocab * s.hidden * 2 + (s.n_layers * 2304 + s.hidden) * 2
+    assert weights == 779_223_040
