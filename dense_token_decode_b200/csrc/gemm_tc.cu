@@ -29,7 +29,22 @@ constexpr int BM = 128, BK = 64;
 constexpr int kThreads = 192;
 constexpr int kTileBytes = BM * BK * 2;  // 16 KB for a 128 x 64 fp16 A tile
 
-enum Kind { kStore = 0, kResidual = 1, kSwiGLU = 2 };
+enum Kind { kStore = 0, kResidual = 1, kSwiGLU = 2, kQKVHead = 3 };
+
+// kQKVHead epilogue: the QKV projection of consecutive positions pos0 + m of
+// one sequence, finished per head in the epilogue: q and k heads RMSNorm'ed
+// (gains over the head) and rotated (rotate-half RoPE at the row's position);
+// q written fp32 [M][nq * d], k and v rounded to bf16 into the paged cache.
+struct HeadEpi {
+  const float2* rope;  // [max_pos][d/2] (cos, sin)
+  const __nv_bfloat16* q_norm;
+  const __nv_bfloat16* k_norm;
+  float eps;
+  int nq, nkv, d;
+  KVView kv;
+  int layer, seq, pos0;
+  float* q_out;
+};
 
 struct Params {
   int M, N, K;       // N = output columns of D (SwiGLU: 2 x act columns per tile)
@@ -37,6 +52,7 @@ struct Params {
   int a_terms;       // 1 or 2
   int lo_col0;       // with 2 terms: only output tiles from this column on use A_lo
   int ksplit;        // K split into this many parts per tile (kResidual only: atomic adds)
+  HeadEpi he;        // kQKVHead only
   int n_tiles_m, n_tiles_n;
   int stages;
   float* out;        // kStore: fp32 [M, ldo]; kResidual: fp32 [M, ldo] (+=)
@@ -46,6 +62,88 @@ struct Params {
   int act_ld;
   int* err;
 };
+
+// Epilogue of a QKV tile (columns [col0, col0 + BN) of the projection, whole
+// heads since BN is a multiple of d) for this thread's row m. All lanes take
+// part in the tensor-memory loads; only live rows store.
+template <int BN>
+__device__ __forceinline__ void qkv_head_epilogue(const HeadEpi& e, uint32_t taddr, int col0,
+                                                  int m, bool live) {
+  const int d = e.d, half = d / 2;
+  const int pos = e.pos0 + m;
+  for (int cb = 0; cb < BN; cb += d) {
+    const int gh = (col0 + cb) / d;  // head index over q | k | v
+    if (gh >= e.nq + e.nkv) {
+      // v head: bf16 into the cache
+      const int g = gh - e.nq - e.nkv;
+      const size_t off = live ? e.kv.offset(e.layer, e.seq, pos, g) : 0;
+      for (int c0 = 0; c0 < d; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(taddr + cb + c0, r);
+        if (!live) continue;
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+          __align__(16) __nv_bfloat16 v[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) v[i] = __float2bfloat16_rn(__uint_as_float(r[j + i]));
+          *reinterpret_cast<uint4*>(e.kv.v + off + c0 + j) = *reinterpret_cast<uint4*>(v);
+        }
+      }
+      continue;
+    }
+    const bool is_q = gh < e.nq;
+    const __nv_bfloat16* gain = is_q ? e.q_norm : e.k_norm;
+    float ss = 0.f;
+    for (int c0 = 0; c0 < d; c0 += 32) {
+      uint32_t r[32];
+      tmem_ld32(taddr + cb + c0, r);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) ss = fmaf(__uint_as_float(r[j]), __uint_as_float(r[j]), ss);
+    }
+    const float inv = rsqrtf(ss / (float)d + e.eps);
+    const float2* cs = e.rope + (size_t)(live ? pos : 0) * half;
+    float* qdst = e.q_out + (size_t)m * e.nq * d + (size_t)gh * d;
+    const size_t koff = (!is_q && live) ? e.kv.offset(e.layer, e.seq, pos, gh - e.nq) : 0;
+    // pairs (i, i + d/2): columns c0 .. c0+31 of the first half with the
+    // same columns of the second half
+    for (int c0 = 0; c0 < half; c0 += 32) {
+      uint32_t lo[32], hi[32];
+      tmem_ld32(taddr + cb + c0, lo);
+      tmem_ld32(taddr + cb + half + c0, hi);
+      if (!live) continue;
+#pragma unroll
+      for (int j = 0; j < 32; j += 8) {
+        float olo[8], ohi[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int i = c0 + j + q;
+          const float a = __uint_as_float(lo[j + q]) * inv * __bfloat162float(gain[i]);
+          const float b = __uint_as_float(hi[j + q]) * inv * __bfloat162float(gain[half + i]);
+          const float2 t = cs[i];
+          olo[q] = a * t.x - b * t.y;
+          ohi[q] = b * t.x + a * t.y;
+        }
+        if (is_q) {
+          float* dl = qdst + c0 + j;
+          float* dh = qdst + half + c0 + j;
+          *reinterpret_cast<float4*>(dl) = make_float4(olo[0], olo[1], olo[2], olo[3]);
+          *reinterpret_cast<float4*>(dl + 4) = make_float4(olo[4], olo[5], olo[6], olo[7]);
+          *reinterpret_cast<float4*>(dh) = make_float4(ohi[0], ohi[1], ohi[2], ohi[3]);
+          *reinterpret_cast<float4*>(dh + 4) = make_float4(ohi[4], ohi[5], ohi[6], ohi[7]);
+        } else {
+          __align__(16) __nv_bfloat16 kl[8], kh[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            kl[q] = __float2bfloat16_rn(olo[q]);
+            kh[q] = __float2bfloat16_rn(ohi[q]);
+          }
+          *reinterpret_cast<uint4*>(e.kv.k + koff + c0 + j) = *reinterpret_cast<uint4*>(kl);
+          *reinterpret_cast<uint4*>(e.kv.k + koff + half + c0 + j) = *reinterpret_cast<uint4*>(kh);
+        }
+      }
+    }
+  }
+}
 
 // BN (128 or 256): output columns per tile; the B tile is BN x 64 and the two
 // fp32 accumulators take 2 x BN tensor-memory columns.
@@ -193,7 +291,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + abuf * BN;
       const int m = mt * BM + row_in_tile;
       const bool live = m < p.M;
-      if (!swiglu) {
+      if (p.kind == kQKVHead) {
+        qkv_head_epilogue<BN>(p.he, taddr, nt * BN, m, live);
+      } else if (!swiglu) {
         for (int c0 = 0; c0 < BN; c0 += 32) {
           uint32_t r[32];
           tmem_ld32(taddr + c0, r);
@@ -316,7 +416,7 @@ template <int BN>
 cudaError_t launch_bn(const CUtensorMap* a, const CUtensorMap* a_lo, const CUtensorMap* b,
                       const CUtensorMap* b2, int M, int N, int K, int kind, float* out, int ldo,
                       __half* act_hi, __half* act_lo, int act_ld, int* err, int num_sms,
-                      cudaStream_t st, int lo_col0) {
+                      cudaStream_t st, int lo_col0, const tc::HeadEpi* he) {
   static bool attr_done = false;
   if (!attr_done) {
     cudaFuncSetAttribute(tc::gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -330,6 +430,7 @@ cudaError_t launch_bn(const CUtensorMap* a, const CUtensorMap* a_lo, const CUten
   p.kind = kind;
   p.a_terms = a_lo ? 2 : 1;
   p.lo_col0 = lo_col0;
+  if (he) p.he = *he;
   p.n_tiles_m = (M + tc::BM - 1) / tc::BM;
   p.n_tiles_n = N / BN;
   // Residual GEMMs with fewer tiles than SMs split K in two (atomic adds).
@@ -364,9 +465,27 @@ cudaError_t launch_gemm_tc(const CUtensorMap* a, const CUtensorMap* a_lo, const 
                            int num_sms, cudaStream_t st, int bn, int lo_col0) {
   if (bn == 256)
     return launch_bn<256>(a, a_lo, b, b2, M, N, K, kind, out, ldo, act_hi, act_lo, act_ld, err,
-                          num_sms, st, lo_col0);
+                          num_sms, st, lo_col0, nullptr);
   return launch_bn<128>(a, a_lo, b, b2, M, N, K, kind, out, ldo, act_hi, act_lo, act_ld, err,
-                        num_sms, st, lo_col0);
+                        num_sms, st, lo_col0, nullptr);
+}
+
+// The QKV GEMM of a prefill chunk with the per-head epilogue (see HeadEpi):
+// rows map to positions pos0.. of sequence seq; q goes to q_out, k and v to
+// the cache. bn must be a multiple of d.
+cudaError_t launch_gemm_tc_qkv_heads(const CUtensorMap* a, const CUtensorMap* a_lo,
+                                     const CUtensorMap* b, int M, int N, int K, int* err,
+                                     int num_sms, cudaStream_t st, int bn, int lo_col0,
+                                     const float2* rope, const __nv_bfloat16* q_norm,
+                                     const __nv_bfloat16* k_norm, float eps, int nq, int nkv,
+                                     int d, const KVView& kv, int layer, int seq, int pos0,
+                                     float* q_out) {
+  tc::HeadEpi he{rope, q_norm, k_norm, eps, nq, nkv, d, kv, layer, seq, pos0, q_out};
+  if (bn == 256)
+    return launch_bn<256>(a, a_lo, b, nullptr, M, N, K, tc::kQKVHead, nullptr, 0, nullptr,
+                          nullptr, 0, err, num_sms, st, lo_col0, &he);
+  return launch_bn<128>(a, a_lo, b, nullptr, M, N, K, tc::kQKVHead, nullptr, 0, nullptr, nullptr,
+                        0, err, num_sms, st, lo_col0, &he);
 }
 
 }  // namespace fs

@@ -1,8 +1,8 @@
 // Prefill blocks on the tensor cores: the state the tcgen05 GEMMs need (fp16
 // copies of the weights, fp16 activation operands, TMA descriptors) and the
 // per-block kernel sequence
-//   RMSNorm -> fp16 operand (two terms when split) -> QKV GEMM (fp32 out)
-//   -> q/k head norm + RoPE + KV append -> tensor-core attention (fp16 out)
+//   RMSNorm -> fp16 operand (two terms when split) -> QKV GEMM whose epilogue
+//   does the q/k head norm + RoPE + KV append -> tensor-core attention (fp16 out)
 //   -> O GEMM (+= residual) -> RMSNorm -> fp16 operand
 //   -> gate/up GEMM with SwiGLU epilogue (fp16 act) -> down GEMM (+= residual).
 #include <cuda.h>
@@ -18,6 +18,13 @@ cudaError_t launch_gemm_tc(const CUtensorMap* a, const CUtensorMap* a_lo, const 
                            const CUtensorMap* b2, int M, int N, int K, int kind, float* out,
                            int ldo, __half* act_hi, __half* act_lo, int act_ld, int* err,
                            int num_sms, cudaStream_t st, int bn, int lo_col0 = 0);
+cudaError_t launch_gemm_tc_qkv_heads(const CUtensorMap* a, const CUtensorMap* a_lo,
+                                     const CUtensorMap* b, int M, int N, int K, int* err,
+                                     int num_sms, cudaStream_t st, int bn, int lo_col0,
+                                     const float2* rope, const __nv_bfloat16* q_norm,
+                                     const __nv_bfloat16* k_norm, float eps, int nq, int nkv,
+                                     int d, const KVView& kv, int layer, int seq, int pos0,
+                                     float* q_out);
 
 namespace {
 
@@ -223,11 +230,19 @@ fs_status layer_tc(fs_model* m, const fs_kv* kv, const RowMap& map, int rows, in
   rmsnorm_f16_kernel<<<rows, 256, 0, st>>>(m->h, s.H, Lw.attn_norm, s.eps, t->xn_hi,
                                            split ? t->xn_lo : nullptr);
   FS_TRY(cudaGetLastError());
-  FS_TRY(launch_gemm_tc(&t->a_xn_hi, split ? &t->a_xn_lo : nullptr, &mp.qkv, nullptr, rows,
-                        s.qkv_dim(), s.H, 0, m->qkv, s.qkv_dim(), nullptr, nullptr, 0, m->err,
-                        m->num_sms, st, bn_qkv(s), split_from));
-  FS_TRY(launch_qk_norm_rope_append(m->qkv, rows, map, s, Lw.q_norm, Lw.k_norm, m->rope, m->q,
-                                    kvv, l, st));
+  if (map.n_list == 0 && bn_qkv(s) % s.d == 0 && s.d % 64 == 0) {
+    // the per-head RMSNorm, RoPE and the K/V append run in the GEMM epilogue
+    FS_TRY(launch_gemm_tc_qkv_heads(&t->a_xn_hi, split ? &t->a_xn_lo : nullptr, &mp.qkv, rows,
+                                    s.qkv_dim(), s.H, m->err, m->num_sms, st, bn_qkv(s),
+                                    split_from, m->rope, Lw.q_norm, Lw.k_norm, s.eps, s.nq,
+                                    s.nkv, s.d, kvv, l, map.seq0, map.pos0, m->q));
+  } else {
+    FS_TRY(launch_gemm_tc(&t->a_xn_hi, split ? &t->a_xn_lo : nullptr, &mp.qkv, nullptr, rows,
+                          s.qkv_dim(), s.H, 0, m->qkv, s.qkv_dim(), nullptr, nullptr, 0, m->err,
+                          m->num_sms, st, bn_qkv(s), split_from));
+    FS_TRY(launch_qk_norm_rope_append(m->qkv, rows, map, s, Lw.q_norm, Lw.k_norm, m->rope, m->q,
+                                      kvv, l, st));
+  }
   if (attention_tc_supported(s, kvv, map)) {
     FS_TRY(launch_attention_tc(m->q, rows, map, s, kvv, l, t->o_hi, m->err, st));
   } else {

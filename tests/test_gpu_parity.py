@@ -333,6 +333,32 @@ def test_tiny_split_kv_decode_batch_of_seven(tiny):
         assert kv.length(q) == lens[q] + 1
 
 
+def test_tiny_decode_largest_batch(tiny):
+    """The largest decode batch the boundary accepts (64 rows): the tiled
+    CUDA-core GEMMs, split-KV attention over 64 rows and the LM head for 64
+    rows, sequences of different lengths in one step."""
+    s = tiny.shape
+    B = 64
+    lens = [1 + (7 * i) % 37 for i in range(B)]
+    prompts = [synth.token_ids(n, s.vocab, seed=100 + i).tolist() for i, n in enumerate(lens)]
+    kv = tiny.model.kv(B, 48)
+    for i, p in enumerate(prompts):
+        tiny.model.prefill(kv, i, _dev_i32(p))
+    nxt = synth.token_ids(B, s.vocab, seed=99).tolist()
+    order = list(range(B - 1, -1, -1))
+    logits = torch.empty((B, s.vocab), device=DEV)
+    am = torch.empty(B, dtype=torch.int32, device=DEV)
+    tiny.model.decode_step(kv, order, _dev_i32([nxt[q] for q in order]), logits, am)
+    torch.cuda.synchronize()
+    for b in (0, 1, 17, 40, 63):
+        q = order[b]
+        cache = tiny.oracle.forward(prompts[q])[2]
+        rl = tiny.oracle.forward([nxt[q]], cache)[0]
+        assert_logits_close(oracle_tensor(logits[b]), rl, what=f"batch row {b} (len {lens[q]})")
+        check_greedy_step(int(am[b]), oracle_tensor(logits[b]), rl)
+    assert all(kv.length(q) == lens[q] + 1 for q in range(B))
+
+
 def test_tiny_errors_are_reported_not_faulted(tiny):
     m, s = tiny.model, tiny.shape
     kv = m.kv(2, 16)
