@@ -811,19 +811,27 @@ struct Consumer {
               const uint4 u = *reinterpret_cast<const uint4*>(st + srow[r] * rb + k0 * 2);
               w[0] = lo16(u.x); w[1] = hi16(u.x); w[2] = lo16(u.y); w[3] = hi16(u.y);
               w[4] = lo16(u.z); w[5] = hi16(u.z); w[6] = lo16(u.w); w[7] = hi16(u.w);
+#pragma unroll
+              for (int bb = 0; bb < NBT; ++bb)
+#pragma unroll
+                for (int q = 0; q < 8; ++q) acc[r][bb] = fmaf(w[q], x8[bb][q], acc[r][bb]);
             } else {
+              // the lane's 8 codes share one block scale: dot the codes, scale once
               const uint2 u = *reinterpret_cast<const uint2*>(st + srow[r] * rb + k0);
               const float sc = __half2float(sbase[srow[r] * (K / 32) + k0 / 32]);
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
-                w[q] = (float)(int8_t)((u.x >> (8 * q)) & 0xff) * sc;
-                w[4 + q] = (float)(int8_t)((u.y >> (8 * q)) & 0xff) * sc;
+                w[q] = (float)(int8_t)((u.x >> (8 * q)) & 0xff);
+                w[4 + q] = (float)(int8_t)((u.y >> (8 * q)) & 0xff);
+              }
+#pragma unroll
+              for (int bb = 0; bb < NBT; ++bb) {
+                float t = 0.f;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) t = fmaf(w[q], x8[bb][q], t);
+                acc[r][bb] = fmaf(sc, t, acc[r][bb]);
               }
             }
-#pragma unroll
-            for (int bb = 0; bb < NBT; ++bb)
-#pragma unroll
-              for (int q = 0; q < 8; ++q) acc[r][bb] = fmaf(w[q], x8[bb][q], acc[r][bb]);
           }
         }
         stage_release();
