@@ -139,6 +139,9 @@ void fs_model_destroy(fs_model* model);
  * layer so decode does one token of work). Pages hold 64 positions; each
  * sequence owns ceil(max_tokens_per_seq/64) pages reached through a block
  * table. K is stored after q/k-norm and RoPE. Every sequence starts empty.
+ * The pages are zeroed: slots past a sequence's length always hold finite
+ * values (the attention kernels read whole pages and weight those slots by
+ * exact zeros; values imported with fs_kv_import must be finite too).
  * Errors: FS_ERR_NULL, FS_ERR_INVALID, FS_ERR_OOM. */
 fs_status fs_kv_alloc(const fs_model* model, int32_t max_seqs, int32_t max_tokens_per_seq,
                       fs_kv** out);
