@@ -52,7 +52,7 @@ SEED = 1
 # DRAM bytes (read + write) of one decode-kernel launch, from the ncu capture
 # in profiles/decode_mega_qwen3_0p6b_bs1.md (batch 1, context of 53 positions).
 # Re-take it whenever the decode kernel changes.
-DECODE_TRAFFIC_BYTES = 1_198_254_000 + 3_646_720
+DECODE_TRAFFIC_BYTES = 1_198_240_000 + 3_810_048
 DECODE_TRAFFIC_CONTEXT = 53
 
 
