@@ -1,5 +1,6 @@
 // Persistent decode forward: one cooperative launch runs every block and the
-// LM head of one decode step for a batch of up to 4 sequences.
+// LM head of one decode step for a batch of up to 4 sequences (as many as
+// leave the weight ring one stage per consumer warp).
 //
 // Layout of the work. Each CTA (one per SM) owns a contiguous slice of the
 // rows of every weight matrix. A producer warp streams the CTA's slices —
@@ -9,7 +10,8 @@
 // Weights do not depend on activations, so the producer runs ahead across
 // phase and layer boundaries and HBM never waits for the dependency chain.
 //
-// Eight consumer warps compute. Activations move between CTAs as 64-bit
+// Eleven consumer warps compute: weight chunk i belongs to warp i mod 11;
+// KV chunks are shared by all of them. Activations move between CTAs as 64-bit
 // words (fp32 value | 32-bit tag): a consumer polls the words it needs until
 // their tag is the one of the current phase, so there is no grid barrier and
 // no separate flag. Tags grow monotonically across steps; nothing is reset.
@@ -1464,7 +1466,8 @@ void mega_reset(fs_model* m) {
 
 // Runs layers [l0, l1) (and the LM head if run_head) of one decode step for
 // B <= 4 rows. Returns FS_ERR_UNSUPPORTED when the shape or batch is not
-// covered (the caller then uses the general path).
+// covered or the ring would get fewer stages than consumer warps (the caller
+// then uses the general path).
 fs_status decode_mega(fs_model* m, const fs_kv* kv, const RowMap& map, int B, const int32_t* tok,
                       const float* h_in, float* h_out, int l0, int l1, bool run_head,
                       float* logits, int32_t* argmax, cudaStream_t stream) {
