@@ -1,8 +1,8 @@
 // Causal GQA attention over the paged bf16 KV cache, one CTA per (row, query
 // head), CUDA cores, online softmax in fp32. Row r at position p attends keys
-// 0..p of its sequence; query head h reads kv head h / (nq / nkv). This is the
-// general path (any row count, any position mix) and the unfused reference
-// the specialised decode / prefill attention kernels are checked against.
+// 0..p of its sequence; query head h reads kv head h / (nq / nkv). It takes
+// what the specialised kernels do not cover (any row count, any position mix,
+// head sizes or GQA groups outside their templates).
 #include "fs_internal.h"
 
 namespace fs {

@@ -1,7 +1,8 @@
 // Plain shared-memory tiled GEMM on the CUDA cores (fp32 arithmetic):
 // C[m, n] (+)= sum_k A[m, k] W[n, k], A fp32 [M, K], W bf16 or Q8_0 [N, K].
-// It is the general many-row path and the unfused reference the tensor-core
-// prefill GEMM is checked against; it makes no attempt at peak throughput.
+// It serves the general path for 17..127 rows (decode batches above 16, short
+// prefill chunks) and shapes the tensor-core GEMM does not cover; it makes no
+// attempt at peak throughput.
 #include "fs_internal.h"
 
 namespace fs {
