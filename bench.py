@@ -471,7 +471,10 @@ def run_ours(args, world, rank, local):
             "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16 weights, fp32 activations", "data": "synthetic",
+            "dtype": "f32", "data": "synthetic",
+            "precision": "decode: bf16 (or Q8_0) weights widened in registers, fp32 FMA; "
+                         "prefill: fp16 tensor-core operands (two terms where K/V are "
+                         "rounded), fp32 accumulation; KV cache bf16",
             "config": workload_config(),
             "roofline": {"bound": "hbm", "kernel": "decode forward step", "achieved": achieved,
                          "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
