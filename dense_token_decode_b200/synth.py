@@ -11,7 +11,10 @@ regenerated alone):
 
 * linear weights and the (tied) embedding: fp32 N(0, 0.02) draws rounded to
   bf16 with round-to-nearest-even (torch's ``.to(torch.bfloat16)``);
-* RMSNorm gains: exactly 1.0 (bf16);
+* RMSNorm gains: exactly 1.0 (bf16) for the benchmark configurations; with
+  ``gains="random"`` every gain vector (each layer's attn/ffn/q/k norm and the
+  final norm) is its own fp32 N(1, 0.3) draw rounded to bf16, so a kernel that
+  reads one gain in place of another gives a different result;
 * Q8_0 linear weights: blocks of 32 consecutive weights along the input
   (dot-product) axis; int8 codes uniform in [-127, 127]; one fp16 scale per
   block, ``0.02 * sqrt(3) / 127 * u`` with ``u ~ U[0.5, 1.5]`` (weight standard
@@ -111,8 +114,15 @@ def q8_0_blocks(rows: int, cols: int, seed: int) -> tuple[torch.Tensor, torch.Te
     return codes, scales
 
 
+def _gain(n: int, gains: str, seed: int) -> torch.Tensor:
+    if gains == "ones":
+        return torch.ones(n, dtype=torch.bfloat16)
+    g = _gen(seed)
+    return (1.0 + 0.3 * torch.randn(n, generator=g, dtype=torch.float32)).to(torch.bfloat16)
+
+
 def model_weights(shape: ModelShape, seed: int, weight_format: str = "bf16",
-                  layers: range | None = None) -> dict:
+                  layers: range | None = None, gains: str = "ones") -> dict:
     """Random-init weights as CPU tensors.
 
     Returns ``{"embed": bf16 [V,H], "final_norm": bf16 [H], "layers": [...]}``
@@ -120,12 +130,16 @@ def model_weights(shape: ModelShape, seed: int, weight_format: str = "bf16",
     ``weight_format="q8_0"``, to a ``(codes, scales)`` pair) and the norm names
     to bf16 gains. ``layers`` restricts which layers are drawn (the others are
     ``None``); the draws of a layer do not depend on which others are drawn.
+    ``gains`` is ``"ones"`` (every RMSNorm gain 1.0) or ``"random"`` (each gain
+    vector an independent N(1, 0.3) draw); the linear weights do not depend on it.
     """
     if weight_format not in ("bf16", "q8_0"):
         raise ValueError(weight_format)
+    if gains not in ("ones", "random"):
+        raise ValueError(gains)
     out = {
         "embed": normal_bf16(shape.vocab, shape.hidden, 0.02, _sub_seed(seed, 0)),
-        "final_norm": torch.ones(shape.hidden, dtype=torch.bfloat16),
+        "final_norm": _gain(shape.hidden, gains, _sub_seed(seed, 4999)),
         "layers": [],
     }
     want = set(range(shape.n_layers) if layers is None else layers)
@@ -141,8 +155,8 @@ def model_weights(shape: ModelShape, seed: int, weight_format: str = "bf16",
                 lw[name] = normal_bf16(n, k, 0.02, s)
             else:
                 lw[name] = q8_0_blocks(n, k, s)
-        for name in NORM_NAMES:
-            lw[name] = torch.ones(norm_len(shape, name), dtype=torch.bfloat16)
+        for j, name in enumerate(NORM_NAMES):
+            lw[name] = _gain(norm_len(shape, name), gains, _sub_seed(seed, 5000 + l, j))
         out["layers"].append(lw)
     return out
 

@@ -292,16 +292,10 @@ def test_q8_0_model_runs_on_dequantised_weights():
     assert np.all(np.isfinite(logits))
 
 
-@pytest.mark.parametrize("kv_bf16", [False, True])
-def test_forward_matches_transformers_qwen3(kv_bf16):
-    """The whole block structure (norm forms and order, q/k-norm before RoPE,
-    rotate-half pairs, GQA grouping, scale, SwiGLU, tied head) against the
-    Qwen3 implementation in ``transformers`` in fp64. Its RoPE tables are
-    built in fp32, which bounds the agreement near 1e-6."""
+def _transformers_run(shape, w, toks):
+    """Logits [S, V] and hidden states of the ``transformers`` Qwen3 model in
+    fp64 over the same bf16 weights (gains included)."""
     transformers = pytest.importorskip("transformers")
-    shape = synth.TINY
-    w = synth.model_weights(shape, 0)
-    orc = oracle.Qwen3Oracle(shape, oracle_weights(w), kv_bf16=kv_bf16)
     cfg = transformers.Qwen3Config(
         vocab_size=shape.vocab, hidden_size=shape.hidden, intermediate_size=shape.ffn,
         num_hidden_layers=shape.n_layers, num_attention_heads=shape.n_q_heads,
@@ -320,15 +314,61 @@ def test_forward_matches_transformers_qwen3(kv_bf16):
         for k, v in lw.items():
             sd[f"model.layers.{l}.{names[k]}.weight"] = v
     m.load_state_dict({k: v.double() for k, v in sd.items()}, strict=True)
-    toks = synth.token_ids(16, shape.vocab, seed=0)
     with torch.no_grad():
         out = m(toks[None].long(), output_hidden_states=True)
-    ref_logits = out.logits[0].numpy()
+    return out.logits[0].numpy(), [h[0].numpy() for h in out.hidden_states]
+
+
+def _transformers_gap(orc, ref, toks):
+    """Worst relative difference of the oracle against the transformers run:
+    the hidden states before each block and the logits of every row."""
+    ref_logits, ref_hidden = ref
     ours, hidden, _ = orc.forward(toks.tolist(), all_logits=True)
-    tol = 2e-3 if kv_bf16 else 2e-6
-    for l in range(shape.n_layers):
-        a, b = hidden[l], out.hidden_states[l][0].numpy()
-        assert np.linalg.norm(a - b) / np.linalg.norm(b) < tol
-    assert np.max(np.abs(ours - ref_logits)) < tol * np.max(np.abs(ref_logits))
+    gaps = [np.linalg.norm(hidden[l] - ref_hidden[l]) / np.linalg.norm(ref_hidden[l])
+            for l in range(orc.cfg.n_layers)]
+    gaps.append(np.max(np.abs(ours - ref_logits)) / np.max(np.abs(ref_logits)))
+    return max(gaps), ours
+
+
+@pytest.mark.parametrize("gains", ["ones", "random"])
+@pytest.mark.parametrize("kv_bf16", [False, True])
+def test_forward_matches_transformers_qwen3(kv_bf16, gains):
+    """The whole block structure (norm forms and order, q/k-norm before RoPE,
+    rotate-half pairs, GQA grouping, scale, SwiGLU, tied head) against the
+    Qwen3 implementation in ``transformers`` in fp64. With ``gains="random"``
+    every RMSNorm gain vector is its own draw, which pins which gain each norm
+    applies (attention vs MLP norm, q vs k norm, final norm). The library's
+    RoPE tables are built in fp32, which bounds the agreement near 1e-6; the
+    bf16 K/V rounding of the cache bounds it near 1e-3."""
+    shape = synth.TINY
+    w = synth.model_weights(shape, 0, gains=gains)
+    toks = synth.token_ids(16, shape.vocab, seed=0)
+    ref = _transformers_run(shape, w, toks)
+    orc = oracle.Qwen3Oracle(shape, oracle_weights(w), kv_bf16=kv_bf16)
+    gap, ours = _transformers_gap(orc, ref, toks)
+    # transformers keeps K/V unrounded; the bf16 cache rounds each stored
+    # element by up to 2^-9 relative, so that mode agrees to about 2^-8
+    tol = 2.0 ** -8 if kv_bf16 else 2e-6
+    assert gap < tol, gap
     if not kv_bf16:
-        assert [oracle.greedy_select(r) for r in ours] == ref_logits.argmax(-1).tolist()
+        assert [oracle.greedy_select(r) for r in ours] == ref[0].argmax(-1).tolist()
+
+
+@pytest.mark.parametrize("swap", [("q_norm", "k_norm"), ("attn_norm", "ffn_norm"), "final"])
+def test_transformers_pin_catches_misplaced_gains(swap):
+    """The random-gain comparison above fails for an oracle that applies one
+    gain in place of another: the mistake is planted in a copy of the oracle
+    (CPU only) and the gap must exceed the tolerance by orders of magnitude."""
+    shape = synth.TINY
+    w = synth.model_weights(shape, 0, gains="random")
+    toks = synth.token_ids(16, shape.vocab, seed=0)
+    ref = _transformers_run(shape, w, toks)
+    orc = oracle.Qwen3Oracle(shape, oracle_weights(w), kv_bf16=False)
+    if swap == "final":
+        orc.final_norm = orc.layers[0]["attn_norm"].copy()
+    else:
+        a, b = swap
+        for layer in orc.layers:
+            layer[a], layer[b] = layer[b], layer[a]
+    gap, _ = _transformers_gap(orc, ref, toks)
+    assert gap > 1e-2, gap
