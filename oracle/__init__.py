@@ -27,3 +27,10 @@ from .qwen3 import (  # noqa: F401
     round_to_bf16,
     silu,
 )
+from .sampling import (  # noqa: F401
+    filtered_distribution,
+    philox4x32_10,
+    ranking,
+    sample,
+    uniform,
+)
