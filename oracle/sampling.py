@@ -26,9 +26,9 @@ taken here:
 
 The uniform comes from a counter-based generator so that the GPU and this
 oracle draw the same numbers: Philox4x32-10 (Salmon, Moraes, Dror and Shaw,
-"Parallel random numbers: as easy as 1, 2, 3", SC'11), key = the 64-bit seed,
-counter = (step, row, 0, 0); ``u`` = the top 24 bits of the first output word
-times 2^-24, exact in fp32.
+"Parallel random numbers: as easy as 1, 2, 3", SC'11), key = the 64-bit seed
+(low word first), counter = (step low word, row, step high word, 0); ``u`` =
+the top 24 bits of the first output word times 2^-24, exact in fp32.
 """
 
 from __future__ import annotations
@@ -64,7 +64,8 @@ def philox4x32_10(counter, key):
 
 def uniform(seed: int, step: int, row: int) -> float:
     """The draw's uniform in [0, 1): 24 bits of Philox4x32-10 output."""
-    x = philox4x32_10((step, row, 0, 0), (seed & _MASK, (seed >> 32) & _MASK))[0]
+    x = philox4x32_10((step & _MASK, row, (step >> 32) & _MASK, 0),
+                      (seed & _MASK, (seed >> 32) & _MASK))[0]
     return (x >> 8) * 2.0 ** -24
 
 
