@@ -49,11 +49,10 @@ DECODE_STEPS = 256
 PREFILL_S = 2048
 SEED = 1
 
-# DRAM bytes (read + write) of one decode-kernel launch, from the ncu capture
-# in profiles/decode_mega_qwen3_0p6b_bs1.md (batch 1, context of 53 positions).
-# Re-take it whenever the decode kernel changes.
-DECODE_TRAFFIC_BYTES = 1_198_240_000 + 3_810_048
-DECODE_TRAFFIC_CONTEXT = 53
+# DRAM bytes (read + write) of one decode-kernel launch as an ncu capture
+# measured them, with the capture's context length and date; None until the
+# current decode kernel has been captured (the JSON line then reports null).
+DECODE_TRAFFIC = None  # {"bytes": ..., "context": ..., "taken": "YYYY-MM-DD"}
 
 
 def peaks():
@@ -186,6 +185,20 @@ def job_throughput(tokens_per_rank: int, world: int, ms_this_rank: float) -> tup
 
 # --------------------------------------------------------------------------- CPU oracle
 
+def host_cpu():
+    """The host's logical core count and CPU model (for the CPU baseline)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return os.cpu_count(), model
+
+
 def oracle_decode_sample(shape, n_decode: int, n_warm: int = 0):
     """The CPU oracle (single BLAS thread) on the head of the same job: the
     8-token prompt prefill, n_warm untimed greedy decode steps, then n_decode
@@ -235,6 +248,7 @@ def run_reference(args, world, rank):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(),
         "cpu_baseline": {"value": value, "unit": "tok/s", "cores": cores, "kind": "oracle",
+                         "host_cores": host_cpu()[0], "cpu_model": host_cpu()[1],
                          "sample": f"{args.steps} timed greedy decode steps after the 8-token "
                                    f"prompt and {args.warmup} untimed ones (fp64 numpy, one "
                                    f"BLAS thread)"},
@@ -313,7 +327,10 @@ def run_ours(args, world, rank, local):
     # the captured launch's traffic, moved to the job's mean context (KV grows by
     # one position's K and V per step)
     kv_tok = shape.n_layers * 2 * shape.n_kv_heads * shape.head_dim * 2
-    traffic = DECODE_TRAFFIC_BYTES + kv_tok * (statistics.mean(ctx) - DECODE_TRAFFIC_CONTEXT)
+    traffic = None
+    if DECODE_TRAFFIC is not None:
+        traffic = DECODE_TRAFFIC["bytes"] + kv_tok * (statistics.mean(ctx)
+                                                      - DECODE_TRAFFIC["context"])
 
     # End to end: fs_greedy with host buffers (prompt H2D, ids D2H inside the call).
     host_prompt = prompt.cpu().pin_memory()
@@ -372,14 +389,15 @@ def run_ours(args, world, rank, local):
         kvp.close()
 
     # Q8_0 decode at batch 1: the same job shape with Q8_0 linear weights
-    # (embedding / LM head bf16), 64 greedy steps after the 8-token prompt.
+    # (embedding / LM head bf16), 256 greedy steps after the 8-token prompt.
     q8r = None
     if not args.no_q8:
         wq = synth.model_weights(shape, 4, "q8_0")
         mq = Model(shape, wq, dev, max_pos=1024)
         del wq
-        kvq = mq.kv(1, PROMPT + 80)
-        qgen = torch.zeros(72, dtype=torch.int32, device=dev)
+        QSTEPS = DECODE_STEPS
+        kvq = mq.kv(1, PROMPT + QSTEPS + 16)
+        qgen = torch.zeros(QSTEPS + 8, dtype=torch.int32, device=dev)
         qprompt = synth.token_ids(PROMPT, shape.vocab, seed=4).to(dev)
 
         def qjob(n):
@@ -395,7 +413,6 @@ def run_ours(args, world, rank, local):
         mq.prefill(kvq, 0, qprompt, None, qgen[0:1])
         q0 = torch.cuda.Event(enable_timing=True)
         q1 = torch.cuda.Event(enable_timing=True)
-        QSTEPS = 64
         q0.record(stream)
         for i in range(QSTEPS):
             mq.decode_step(kvq, [0], qgen[i:i + 1], None, qgen[i + 1:i + 2])
@@ -413,10 +430,10 @@ def run_ours(args, world, rank, local):
         mq.close()
 
     # Batched decode: 16 sequences, each with 8192 pre-filled N(0,1) bf16 K/V
-    # positions, 32 greedy steps (ids stay on the device).
+    # positions, 64 greedy steps (ids stay on the device).
     bat = None
     if not args.no_batched:
-        B, CTX, BSTEPS = 16, 8192, 32
+        B, CTX, BSTEPS = 16, 8192, 64
         kvb = model.kv(B, CTX + BSTEPS + 8)
         for q in range(B):
             for l in range(shape.n_layers):
@@ -463,6 +480,7 @@ def run_ours(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         sec, cores = oracle_decode_sample(shape, args.cpu_steps)
         cpu = {"value": 1.0 / sec, "unit": "tok/s", "cores": cores, "kind": "oracle",
+               "host_cores": host_cpu()[0], "cpu_model": host_cpu()[1],
                "sample": f"{args.cpu_steps} greedy decode steps after the 8-token prompt of "
                          f"the same job (fp64 numpy oracle, one BLAS thread)"}
 
@@ -479,6 +497,11 @@ def run_ours(args, world, rank, local):
             "roofline": {"bound": "hbm", "kernel": "decode forward step", "achieved": achieved,
                          "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                          "traffic": traffic,
+                         "traffic_source": (None if DECODE_TRAFFIC is None else
+                                            f"ncu dram bytes of one launch at context "
+                                            f"{DECODE_TRAFFIC['context']}, taken "
+                                            f"{DECODE_TRAFFIC['taken']}, moved to the mean "
+                                            f"context"),
                          "bytes_per_step": statistics.mean(per_step),
                          "weight_bytes": weight_bytes, "step_us": step_s * 1e6,
                          "peak_source": peak_src},

@@ -78,10 +78,14 @@ SIGNATURES = {
     "fs_prefill": (_I, [_P, _P, _I, _P, _I, _P, _P, _P]),
     "fs_decode_step": (_I, [_P, _P, _P, _P, _I, _P, _P, _P]),
     "fs_greedy": (_I, [_P, _P, _I, _P, _I, _I, _P, _I, _P, _PI, _PI, _P]),
+    "fs_sample": (_I, [_P, _P, _I, C.c_float, _I, C.c_float, C.c_uint64, C.c_uint64, _P, _P]),
+    "fs_generate": (_I, [_P, _P, _I, _P, _I, _I, _P, _I, C.c_float, _I, C.c_float, C.c_uint64,
+                         _P, _PI, _PI, _P]),
     "fs_debug_capture": (_I, [_P, _P, _I]),
     "fs_debug_block": (_I, [_P, _P, _I, _I, _P, _I, _P, _P]),
     "fs_debug_dequant_q8_0": (_I, [_P, _P, _I, _I, _P, _P]),
     "fs_debug_trace": (_I, [_P, _P]),
+    "fs_debug_wait_limit": (_I, [_P, C.c_uint64, _I]),
     "fs_debug_lm_head": (_I, [_P, _P, _I, _P, _P, _P]),
     "fs_device_error": (_I, [_P, _PI]),
     "fs_set_prefill_split": (_I, [_P, _I]),
@@ -149,10 +153,13 @@ fs_kv_set_length = _wrap("fs_kv_set_length")
 fs_prefill = _wrap("fs_prefill")
 fs_decode_step = _wrap("fs_decode_step")
 fs_greedy = _wrap("fs_greedy")
+fs_sample = _wrap("fs_sample")
+fs_generate = _wrap("fs_generate")
 fs_debug_capture = _wrap("fs_debug_capture")
 fs_debug_block = _wrap("fs_debug_block")
 fs_debug_dequant_q8_0 = _wrap("fs_debug_dequant_q8_0")
 fs_debug_trace = _wrap("fs_debug_trace")
+fs_debug_wait_limit = _wrap("fs_debug_wait_limit")
 fs_debug_lm_head = _wrap("fs_debug_lm_head")
 fs_device_error = _wrap("fs_device_error")
 fs_set_prefill_split = _wrap("fs_set_prefill_split")

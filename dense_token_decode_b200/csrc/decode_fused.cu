@@ -1,0 +1,1828 @@
+// Persistent decode forward for batches of 1..4 sequences: one cooperative
+// launch (one CTA per SM) runs every block, the final norm, the tied LM head
+// and the greedy argmax of one decode step.
+//
+// Work split of a block (G CTAs, CTA c):
+//   A  RMSNorm + QKV projection, row split: CTA c owns rows [a_c, b_c) of
+//      Wq|Wk|Wv. Outputs go out as tagged 64-bit words (fp32 value | tag).
+//   B  attention fused with the output projection, split by (kv head g,
+//      8-wide slice j of the head dimension): the unit normalises and rotates
+//      the group's q heads and k (the j = 0 unit appends k, v to the cache),
+//      runs the causal softmax over every key of the group, keeps the output
+//      o[h][8j .. 8j+8) of each of the group's query heads exactly (no split
+//      merge) and multiplies it by the matching 8 rows of Wo^T (a transposed
+//      copy made at model creation), adding its share of the O projection to
+//      the residual.
+//   C  RMSNorm + gate/up + SwiGLU + down, split by intermediate columns: CTA c
+//      owns columns [a_c, b_c) of Wg, Wu and the matching rows of Wd^T, so its
+//      SwiGLU outputs feed its own share of the down projection, added to the
+//      residual.
+// Three hand-offs per block: A -> B (tagged words), B -> C and C -> next A
+// (the residual sums).
+//
+// Residual sums. Every contribution is added with one 64-bit integer atomic
+// per element, the value in fixed point (2^-32 units), so the sum does not
+// depend on the order of arrival (the step is bit-for-bit reproducible).
+// Contributions are spread over P copies of each accumulator (contributor k
+// adds into copy k % P) to spread the atomics over more L2 lines; readers
+// add the copies. After its atomics a contributing CTA passes a barrier and
+// one thread publishes them with a release fence and an increment of the
+// copy's arrival counter; a reader's first thread acquires the counters, the
+// CTA passes a barrier, and every thread then loads its words once.
+// Accumulators of a step live in one of two sets; each step clears the other
+// set for the step after it.
+//
+// Weight stream. A producer warp (one lane) copies the CTA's weights, the
+// group's K/V pages and, for the LM head, its rows of the embedding into a
+// ring of shared-memory stages with cp.async.bulk, in the order the consumers
+// use them; it runs ahead across phase and block boundaries, since weights do
+// not depend on activations. Every consumer warp waits on every chunk and
+// arrives on its release barrier (arrival count = consumer warps), so no warp
+// can get a full ring ahead of another and a parity wait always refers to the
+// chunk it means.
+//
+// Every wait is bounded by %globaltimer (limit set per launch); on timeout
+// the CTA records kErrTimeout, raises the abort flag that every wait checks,
+// drains its own bulk copies and returns.
+#include <algorithm>
+
+#include "runtime.h"
+
+namespace fs {
+namespace fused {
+
+constexpr int kConsumerWarps = 11;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kThreads = kConsumers + 32;  // + producer warp
+constexpr int kMaxB = 4;
+constexpr int kData = 16384;   // main area of a stage
+constexpr int kExtra = 2048;   // Q8_0 scale area after it
+constexpr int kStageBytes = kData + kExtra;
+constexpr int kMaxStages = 16;
+constexpr int kSlice = 8;      // head-dimension slice of one attention unit
+constexpr int kMaxCopies = 4;  // copies of each residual accumulator
+constexpr float kFix = 4294967296.0f;       // 2^32
+constexpr float kUnfix = 2.3283064365386963e-10f;  // 2^-32
+constexpr int kMaxRep = 2;     // query heads per kv head
+constexpr int kTraceSlots = 16;
+
+enum { kQ8 = 1 };
+
+struct TLayer {
+  const void* wo_t;    // Wo^T [nq*d][H] (bf16, or int8 codes)
+  const __half* so_t;  // Q8_0: scales of Wo^T rows, [nq*d/32][H]
+  const void* wd_t;    // Wd^T [I][H]
+  const __half* sd_t;  // Q8_0: [I/32][H]
+};
+
+struct Params {
+  int L, H, nq, nkv, d, I, V;
+  float eps;
+  int q8;
+  const LayerDev* layers;
+  const TLayer* tl;
+  const __nv_bfloat16* embed;
+  const __nv_bfloat16* final_norm;
+  const float2* rope;
+  KVView kv;
+  int B;
+  int seq[kMaxB];
+  int pos[kMaxB];
+  const int32_t* tokens;
+  unsigned long long* xq;    // [B][(nq+2nkv)d] tagged words
+  unsigned long long* acc;   // this step's accumulators [2L][P][B][H]
+  unsigned long long* cnt;   // their arrival counters [2L][kMaxCopies]
+  unsigned long long* clear; // the other set, cleared by this step
+  long long clear_words;     // words of the other set to clear
+  int P;                     // copies per accumulator
+  int n_units;               // attention units nkv * d/8
+  int c_ctas;                // CTAs with intermediate columns
+  uint32_t tag0;
+  int l0, l1;
+  const float* h_in;
+  float* h_out;
+  int run_head;
+  float* logits;
+  int32_t* argmax;
+  unsigned long long* am_key;
+  unsigned int* am_cnt;
+  float* capture;
+  int capture_stride;
+  int* err;
+  int* abort_flag;
+  unsigned long long wait_ns;
+  int withhold_layer;  // debug: phase-A outputs of this layer are never published
+  unsigned long long* trace;
+  int n_stages;
+  int off_r, off_z, off_misc, off_attn, off_tab, off_bar;
+  int bt_in_smem;
+  int lm_owner;  // LM-head chunks each consumed by one warp (ring of >= 11 stages)
+  int lm_rows;   // rows per LM-head chunk
+};
+
+// ---------------------------------------------------------------------------
+// Small helpers
+
+__device__ __forceinline__ uint32_t su32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(su32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(su32(dst)),
+      "l"(src), "r"(bytes), "r"(su32(bar)), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_word(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_tag(unsigned long long* p, float v, uint32_t tag) {
+  const unsigned long long w = ((unsigned long long)tag << 32) | __float_as_uint(v);
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+__device__ __forceinline__ void red_add(unsigned long long* p, unsigned long long v) {
+  asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+// Publishes the CTA's earlier atomics (ordered before this thread by a CTA
+// barrier) and counts one arrival.
+__device__ __forceinline__ void release_count(unsigned long long* c) {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+  asm volatile("red.relaxed.gpu.global.add.u64 [%0], 1;" ::"l"(c) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_acquire(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void mbar_arrive_n(uint64_t* bar, uint32_t n) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(su32(bar)), "r"(n) : "memory");
+}
+__device__ __forceinline__ unsigned long long now_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void consumer_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory");
+}
+// Barrier of the consumer warps that also ORs a flag over them, so that a
+// decision to stop (a timeout seen by one thread) is taken by all at once.
+__device__ __forceinline__ bool __syncthreads_or_consumers(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, %2, p;\n"
+      " selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(kConsumers)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ bool aborted(const int* flag) {
+  return *reinterpret_cast<const volatile int*>(flag) != 0;
+}
+__device__ __forceinline__ float lo16(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float hi16(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+// One contribution to an accumulator word: the value in fixed point.
+__device__ __forceinline__ unsigned long long fix_word(float x) {
+  return (unsigned long long)__float2ll_rn(x * kFix);
+}
+__device__ __forceinline__ long long word_value(unsigned long long w) { return (long long)w; }
+
+__host__ __device__ inline void slice(int N, int G, int c, int& a, int& b) {
+  a = (int)((long long)N * c / G);
+  b = (int)((long long)N * (c + 1) / G);
+}
+
+// Rows per chunk of each kind (the consumers and the producer agree on them).
+__host__ __device__ inline int rows_cap(int H, bool q8) {  // rows of K = H
+  const int r = q8 ? kData / H : kData / (2 * H);
+  return r < 16 ? r : 16;
+}
+__host__ __device__ inline int pairs_cap(int H, bool q8) {
+  const int r = q8 ? kData / (2 * H) : kData / (4 * H);
+  return r < 8 ? r : 8;
+}
+// End of the QKV chunk from row n (never across the wq|wk|wv boundaries).
+__host__ __device__ inline int qkv_chunk_end(int n, int b, int cap, int qd, int kvd) {
+  int e = n + cap < b ? n + cap : b;
+  if (n < qd) e = e < qd ? e : qd;
+  else if (n < qd + kvd) e = e < qd + kvd ? e : qd + kvd;
+  return e;
+}
+// End of the Wd^T chunk from row n: Q8_0 chunks stay within one 32-row block
+// (one row of transposed scales).
+__host__ __device__ inline int down_chunk_end(int n, int b, int cap, bool q8) {
+  int e = n + cap < b ? n + cap : b;
+  if (q8) {
+    const int blk = (n / 32 + 1) * 32;
+    e = e < blk ? e : blk;
+  }
+  return e;
+}
+
+struct Ring {
+  unsigned char* stages;
+  uint64_t* full;
+  uint64_t* empty;
+  int n;
+};
+
+// Shared-memory copies of the per-layer pointers and the batch's block-table rows.
+__device__ __forceinline__ const LayerDev& layer_s(const Params& p, int l) {
+  extern __shared__ __align__(1024) unsigned char smem_base[];
+  return reinterpret_cast<const LayerDev*>(smem_base + p.off_tab)[l];
+}
+__device__ __forceinline__ const TLayer& tlayer_s(const Params& p, int l) {
+  extern __shared__ __align__(1024) unsigned char smem_base[];
+  return reinterpret_cast<const TLayer*>(smem_base + p.off_tab + (size_t)p.L * sizeof(LayerDev))[l];
+}
+__device__ __forceinline__ size_t kv_off(const Params& p, int layer, int b, int pos, int g) {
+  extern __shared__ __align__(1024) unsigned char smem_base[];
+  int page;
+  if (p.bt_in_smem) {
+    const int32_t* bt = reinterpret_cast<const int32_t*>(
+        smem_base + p.off_tab + (size_t)p.L * (sizeof(LayerDev) + sizeof(TLayer)));
+    page = bt[b * p.kv.pages_per_seq + pos / kPage];
+  } else {
+    page = p.kv.block_table[(size_t)p.seq[b] * p.kv.pages_per_seq + pos / kPage];
+  }
+  return (size_t)layer * p.kv.layer_elems() +
+         (((size_t)page * p.kv.n_kv_heads + g) * kPage + (pos % kPage)) * p.kv.head_dim;
+}
+
+// Accumulator words of version v (2l: after the attention half of block l,
+// 2l+1: after block l), copy q, row b. A launch uses the first 2L*P*B*H words
+// of its set.
+__device__ __forceinline__ unsigned long long* acc_row(const Params& p, int v, int q, int b) {
+  return p.acc + (((size_t)v * p.P + q) * p.B + b) * p.H;
+}
+
+// ---------------------------------------------------------------------------
+// Producer: issues the bulk copies of every chunk, in consumption order.
+
+struct Producer {
+  const Params& p;
+  Ring r;
+  uint64_t policy;
+  unsigned int i = 0;   // chunks issued
+  int stage = 0;
+  uint32_t parity = 1;  // the first pass over the ring finds every stage free
+  bool quit = false;
+
+  __device__ Producer(const Params& pp, Ring rr) : p(pp), r(rr) { policy = evict_first_policy(); }
+
+  __device__ unsigned char* acquire(uint32_t bytes) {
+    if (quit) return nullptr;
+    const int s = stage;
+    unsigned long long t0 = 0;
+    int spins = 0;
+    while (!mbar_test(&r.empty[s], parity)) {
+      if ((++spins & 15) == 0) {
+        if (t0 == 0) t0 = now_ns();
+        if (aborted(p.abort_flag) || now_ns() - t0 > p.wait_ns) {
+          if (!aborted(p.abort_flag)) {
+            atomicExch(p.abort_flag, 1);
+            atomicCAS(p.err, 0, kErrTimeout);
+          }
+          quit = true;
+          return nullptr;
+        }
+      }
+    }
+    mbar_expect_tx(&r.full[s], bytes);
+    return r.stages + (size_t)s * kStageBytes;
+  }
+  __device__ __forceinline__ uint64_t* bar() { return &r.full[stage]; }
+  __device__ __forceinline__ void advance() {
+    ++i;
+    if (++stage == r.n) {
+      stage = 0;
+      parity ^= 1u;
+    }
+  }
+
+  // Rows [n, e) of a [N][K = H] matrix (bf16, or Q8_0 codes + scales).
+  __device__ void rows(const void* w, const __half* s, int n, int e, bool q8) {
+    const int H = p.H, nr = e - n;
+    const uint32_t rb = q8 ? H : 2 * H;
+    const uint32_t sb = q8 ? H / 16 : 0;
+    unsigned char* st = acquire(nr * (rb + sb));
+    if (!st) return;
+    bulk_load(st, static_cast<const unsigned char*>(w) + (size_t)n * rb, nr * rb, bar(), policy);
+    if (q8)
+      bulk_load(st + kData, reinterpret_cast<const unsigned char*>(s) + (size_t)n * sb, nr * sb,
+                bar(), policy);
+    advance();
+  }
+
+  __device__ void phase_a(int l, int a, int b) {
+    const LayerDev& Lw = layer_s(p, l);
+    const bool q8 = p.q8;
+    const int qd = p.nq * p.d, kvd = p.nkv * p.d, cap = rows_cap(p.H, q8);
+    for (int n = a; n < b && !quit;) {
+      const int e = qkv_chunk_end(n, b, cap, qd, kvd);
+      const int which = n < qd ? kWq : (n < qd + kvd ? kWk : kWv);
+      const int base = which == kWq ? 0 : (which == kWk ? qd : qd + kvd);
+      rows(Lw.w[which], Lw.s[which], n - base, e - base, q8);
+      n = e;
+    }
+  }
+
+  __device__ void phase_b(int l, int c, int G) {
+    const TLayer& T = tlayer_s(p, l);
+    const int H = p.H, d = p.d, ds = d / kSlice, rep = p.nq / p.nkv;
+    for (int u = c; u < p.n_units && !quit; u += G) {
+      const int g = u / ds, j = u % ds;
+      for (int b = 0; b < p.B && !quit; ++b) {
+        const int old = p.pos[b];
+        for (int j0 = 0; j0 < old && !quit; j0 += kPage) {
+          const int nk = min(kPage, old - j0);
+          const size_t off = kv_off(p, l, b, j0, g);
+          unsigned char* st = acquire(nk * d * 2);
+          if (!st) return;
+          bulk_load(st, p.kv.k + off, nk * d * 2, bar(), policy);
+          advance();
+          st = acquire(nk * d * 2);
+          if (!st) return;
+          bulk_load(st, p.kv.v + off, nk * d * 2, bar(), policy);
+          advance();
+        }
+      }
+      for (int h = 0; h < rep && !quit; ++h) {
+        const int c0 = (g * rep + h) * d + j * kSlice;
+        if (p.q8) {
+          unsigned char* st = acquire(kSlice * H + 2 * H);
+          if (!st) return;
+          bulk_load(st, static_cast<const int8_t*>(T.wo_t) + (size_t)c0 * H, kSlice * H, bar(),
+                    policy);
+          bulk_load(st + kData, T.so_t + (size_t)(c0 / 32) * H, 2 * H, bar(), policy);
+        } else {
+          unsigned char* st = acquire(kSlice * 2 * H);
+          if (!st) return;
+          bulk_load(st, static_cast<const __nv_bfloat16*>(T.wo_t) + (size_t)c0 * H,
+                    kSlice * 2 * H, bar(), policy);
+        }
+        advance();
+      }
+    }
+  }
+
+  __device__ void phase_c(int l, int a, int b) {
+    const LayerDev& Lw = layer_s(p, l);
+    const TLayer& T = tlayer_s(p, l);
+    const bool q8 = p.q8;
+    const int H = p.H, pc = pairs_cap(H, q8);
+    const uint32_t rb = q8 ? H : 2 * H;
+    const uint32_t sb = q8 ? H / 16 : 0;
+    for (int n = a; n < b && !quit;) {
+      const int e = min(b, n + pc), nr = e - n;
+      unsigned char* st = acquire(2 * nr * (rb + sb));
+      if (!st) return;
+      bulk_load(st, static_cast<const unsigned char*>(Lw.w[kWg]) + (size_t)n * rb, nr * rb, bar(),
+                policy);
+      bulk_load(st + pc * rb, static_cast<const unsigned char*>(Lw.w[kWu]) + (size_t)n * rb,
+                nr * rb, bar(), policy);
+      if (q8) {
+        bulk_load(st + kData, reinterpret_cast<const unsigned char*>(Lw.s[kWg]) + (size_t)n * sb,
+                  nr * sb, bar(), policy);
+        bulk_load(st + kData + pc * sb,
+                  reinterpret_cast<const unsigned char*>(Lw.s[kWu]) + (size_t)n * sb, nr * sb,
+                  bar(), policy);
+      }
+      advance();
+      n = e;
+    }
+    const int rc = rows_cap(H, q8);
+    for (int n = a; n < b && !quit;) {
+      const int e = down_chunk_end(n, b, rc, q8), nr = e - n;
+      unsigned char* st = acquire(nr * rb + (q8 ? 2 * H : 0));
+      if (!st) return;
+      bulk_load(st, static_cast<const unsigned char*>(T.wd_t) + (size_t)n * rb, nr * rb, bar(),
+                policy);
+      if (q8) bulk_load(st + kData, T.sd_t + (size_t)(n / 32) * H, 2 * H, bar(), policy);
+      advance();
+      n = e;
+    }
+  }
+
+  __device__ void tail(int a, int b) {
+    if (!p.run_head) return;
+    const int cap = p.lm_rows;
+    for (int n = a; n < b && !quit;) {
+      const int e = min(b, n + cap);
+      rows(p.embed, nullptr, n, e, false);
+      n = e;
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Consumers
+
+template <int NB, bool Q8W, int IT>
+struct Consumer {
+  const Params& p;
+  Ring r;
+  float* rs;    // [B][H] raw residual rows of the current phase input
+  float* zs;    // [B][H] gain * residual (the GEMV operand before 1/rms)
+  float* zs_base;  // two buffers of zs: phase A / LM head, and phase C
+  float* misc;  // ss partials [2][64] | act [kMaxB][128] | o [kMaxB][2][8]
+  float* attn;  // q [rep][d] | k [d] | v [d] | warp states
+  unsigned long long* best;  // [kMaxB] greedy keys of this CTA
+  int* flag;
+  unsigned long long wbest[kMaxB] = {0ull, 0ull, 0ull, 0ull};
+  unsigned int i = 0;
+  int stage = 0;
+  uint32_t parity = 0;
+  bool quit = false;
+  int tid, warp, lane, G, cta;
+
+  __device__ Consumer(const Params& pp, Ring rr, unsigned char* sm) : p(pp), r(rr) {
+    rs = reinterpret_cast<float*>(sm + p.off_r);
+    zs_base = reinterpret_cast<float*>(sm + p.off_z);
+    zs = zs_base;
+    misc = reinterpret_cast<float*>(sm + p.off_misc);
+    attn = reinterpret_cast<float*>(sm + p.off_attn);
+    best = reinterpret_cast<unsigned long long*>(sm + p.off_misc + 4096);
+    flag = reinterpret_cast<int*>(sm + p.off_misc + 4096 + 8 * kMaxB);
+    tid = threadIdx.x;
+    warp = tid >> 5;
+    lane = tid & 31;
+    G = gridDim.x;
+    cta = blockIdx.x;
+  }
+  float* ss_s = nullptr;                                 // [11][kMaxB] of the current slot
+  __device__ float* act_s() { return misc + 128; }       // [kMaxB][128]
+  __device__ float* o_s() { return misc + 128 + 512; }   // [kMaxB][kMaxRep][kSlice]
+
+  __device__ void tr(int layer, int k) {
+    if (p.trace && tid == 0) p.trace[((size_t)cta * (p.L + 1) + layer) * kTraceSlots + k] = now_ns();
+  }
+  __device__ void give_up() {
+    if (!aborted(p.abort_flag)) {
+      atomicExch(p.abort_flag, 1);
+      atomicCAS(p.err, 0, kErrTimeout);
+    }
+    quit = true;
+  }
+
+  // Wait (whole warp) for the chunk `ahead` places after the oldest one this
+  // warp has not released; returns its stage. Every chunk before it has been
+  // waited for by this warp, so the stage's full barrier is in this chunk's
+  // phase or the one before it.
+  __device__ const unsigned char* chunk_wait(int ahead = 0) {
+    int s = stage + ahead;
+    uint32_t par = parity;
+    if (s >= r.n) {
+      s -= r.n;
+      par ^= 1u;
+    }
+    unsigned long long t0 = 0;
+    int spins = 0;
+    while (true) {
+      const bool ok = quit || mbar_test(&r.full[s], par);
+      if (__all_sync(0xffffffffu, ok)) break;
+      if ((++spins & 15) == 0) {
+        int bad = 0;
+        if (lane == 0) {
+          if (t0 == 0) t0 = now_ns();
+          bad = aborted(p.abort_flag) || now_ns() - t0 > p.wait_ns;
+        }
+        if (__shfl_sync(0xffffffffu, bad, 0)) give_up();
+      }
+    }
+    return r.stages + (size_t)s * kStageBytes;
+  }
+  __device__ void cursor_advance() {
+    ++i;
+    if (++stage == r.n) {
+      stage = 0;
+      parity ^= 1u;
+    }
+  }
+  __device__ void chunk_release() {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&r.empty[stage]);
+    cursor_advance();
+  }
+  // Wait (whole warp) for the next chunk when this warp alone consumes it and
+  // skips the chunks of other warps (ring of at least kConsumerWarps stages):
+  // first the release of the chunk n places earlier in the same stage, then
+  // the chunk itself. With n >= kConsumerWarps the release test cannot see an
+  // older phase: this warp waited on a chunk at most kConsumerWarps places
+  // back, so every chunk 2n places back has been released.
+  __device__ const unsigned char* chunk_wait_owned() {
+    const int s = stage;
+    unsigned long long t0 = 0;
+    int spins = 0;
+    while (true) {
+      const bool ok =
+          quit || (mbar_test(&r.empty[s], parity ^ 1u) && mbar_test(&r.full[s], parity));
+      if (__all_sync(0xffffffffu, ok)) break;
+      if ((++spins & 15) == 0) {
+        int bad = 0;
+        if (lane == 0) {
+          if (t0 == 0) t0 = now_ns();
+          bad = aborted(p.abort_flag) || now_ns() - t0 > p.wait_ns;
+        }
+        if (__shfl_sync(0xffffffffu, bad, 0)) give_up();
+      }
+    }
+    return r.stages + (size_t)s * kStageBytes;
+  }
+
+  // ---- residual input of a phase -----------------------------------------
+
+  static constexpr int kEPT = (NB * IT * 256 + kConsumers - 1) / kConsumers;  // elements / thread
+  float inv[NB];
+
+  // Gains of this thread's elements (k = tid + 352 e of the [B][H] rows),
+  // fetched before the wait for the residual so their latency overlaps it.
+  __device__ __forceinline__ void load_gains(const __nv_bfloat16* g, float (&gr)[kEPT]) {
+#pragma unroll
+    for (int e = 0; e < kEPT; ++e) {
+      const int k = tid + e * kConsumers;
+      gr[e] = k < p.B * p.H ? __bfloat162float(g[k % p.H]) : 0.f;
+    }
+  }
+
+  // Thread 0 waits until every copy of accumulator version v has all of its
+  // `contrib` contributors (contributor c counts in copy c % P); the caller's
+  // barrier then orders every thread's loads after it.
+  __device__ void wait_counts(int v, int contrib) {
+    if (tid != 0 || quit) return;
+    const int P = p.P;
+    unsigned long long t0 = 0;
+    int spins = 0;
+    for (int q = 0; q < P; ++q) {
+      const unsigned long long want = (unsigned long long)((contrib - q + P - 1) / P);
+      const unsigned long long* c = p.cnt + (size_t)v * kMaxCopies + q;
+      while (ld_acquire(c) < want) {
+        __nanosleep(32);
+        if ((++spins & 63) == 0) {
+          if (t0 == 0) t0 = now_ns();
+          if (aborted(p.abort_flag) || now_ns() - t0 > p.wait_ns) {
+            give_up();
+            return;
+          }
+        }
+      }
+    }
+  }
+
+  // The phase input rows into rs (source: v >= 0 an accumulator version, -1
+  // the embedding rows of the tokens or h_in), zs = gain * rs, and 1/rms of
+  // each row into inv. Ends on a barrier.
+  // `slot` (0: phase A and the LM head, 1: phase C) picks the buffers of zs and
+  // of the partial sums, so a warp that runs ahead into the next phase never
+  // writes what a slower warp still reads.
+  __device__ void gather_norm(int v, int contrib, const float (&gr)[kEPT], int slot) {
+    const int H = p.H, n = p.B * H;
+    zs = zs_base + (size_t)slot * p.B * H;
+    ss_s = misc + slot * 64;
+    float ss[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) ss[b] = 0.f;
+    long long sum[kEPT];
+    if (v >= 0) {
+      wait_counts(v, contrib);
+      if (__syncthreads_or_consumers(quit)) quit = true;
+      // every word of every copy of this thread's elements, loads issued together
+#pragma unroll
+      for (int e = 0; e < kEPT; ++e) sum[e] = 0;
+      for (int q = 0; q < p.P; ++q) {
+        unsigned long long w[kEPT];
+#pragma unroll
+        for (int e = 0; e < kEPT; ++e) {
+          const int k = tid + e * kConsumers;
+          w[e] = k < n ? ld_word(acc_row(p, v, q, k / H) + k % H) : 0ull;
+        }
+#pragma unroll
+        for (int e = 0; e < kEPT; ++e) sum[e] += word_value(w[e]);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < kEPT; ++e) {
+      const int k = tid + e * kConsumers;
+      if (k >= n) break;
+      const int b = k / H;
+      float x;
+      if (v >= 0) {
+        x = __ll2float_rn(sum[e]) * kUnfix;
+      } else if (p.h_in) {
+        x = p.h_in[k];
+      } else {
+        int t = p.tokens[b];
+        if (t < 0 || t >= p.V) {
+          if (k % H == 0) atomicCAS(p.err, 0, kErrToken);
+          t = 0;
+        }
+        x = __bfloat162float(p.embed[(size_t)t * H + k % H]);
+      }
+      rs[k] = x;
+      zs[k] = x * gr[e];
+#pragma unroll
+      for (int bb = 0; bb < NB; ++bb)
+        if (bb == b) ss[bb] += x * x;
+    }
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      const float t = warp_sum(ss[b]);
+      if (lane == 0) ss_s[warp * kMaxB + b] = t;
+    }
+    consumer_sync();
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      float t = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) t += ss_s[w * kMaxB + b];
+      inv[b] = rsqrtf(t / (float)H + p.eps);
+    }
+  }
+
+  // Dot products of one weight row (K = H) with every batch row of zs.
+  __device__ __forceinline__ void row_dot(const unsigned char* row, const __half* srow,
+                                          float (&acc)[NB]) {
+    const int H = p.H;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) acc[b] = 0.f;
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+      const int k = lane * 8 + it * 256;
+      float w[8];
+      float sc = 1.f;
+      if (!Q8W) {
+        const uint4 u = *reinterpret_cast<const uint4*>(row + 2 * k);
+        w[0] = lo16(u.x); w[1] = hi16(u.x); w[2] = lo16(u.y); w[3] = hi16(u.y);
+        w[4] = lo16(u.z); w[5] = hi16(u.z); w[6] = lo16(u.w); w[7] = hi16(u.w);
+      } else {
+        const uint2 u = *reinterpret_cast<const uint2*>(row + k);
+        sc = __half2float(srow[k / 32]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          w[q] = (float)(int8_t)((u.x >> (8 * q)) & 0xff);
+          w[4 + q] = (float)(int8_t)((u.y >> (8 * q)) & 0xff);
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        if (b < p.B) {
+          const float4 z0 = *reinterpret_cast<const float4*>(zs + b * H + k);
+          const float4 z1 = *reinterpret_cast<const float4*>(zs + b * H + k + 4);
+          float t = 0.f;
+          t = fmaf(w[0], z0.x, t); t = fmaf(w[1], z0.y, t); t = fmaf(w[2], z0.z, t);
+          t = fmaf(w[3], z0.w, t); t = fmaf(w[4], z1.x, t); t = fmaf(w[5], z1.y, t);
+          t = fmaf(w[6], z1.z, t); t = fmaf(w[7], z1.w, t);
+          acc[b] = Q8W ? fmaf(sc, t, acc[b]) : acc[b] + t;
+        }
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < NB; ++b) acc[b] = warp_sum(acc[b]);
+  }
+
+  // ---- phase A: RMSNorm + QKV rows --------------------------------------
+
+  __device__ void capture_rows(int slot) {
+    if (!p.capture || cta != 0) return;
+    for (int k = tid; k < p.B * p.H; k += kConsumers) {
+      const int b = k / p.H, e = k % p.H;
+      p.capture[((size_t)slot * p.capture_stride + b) * p.H + e] = rs[k];
+    }
+  }
+
+  __device__ void phase_a(int l, int a, int b) {
+    tr(l, 0);
+    const LayerDev& Lw = layer_s(p, l);
+    float gr[kEPT];
+    load_gains(Lw.attn_norm, gr);
+    gather_norm(l == p.l0 ? -1 : 2 * (l - 1) + 1, p.c_ctas, gr, 0);
+    tr(l, 1);
+    capture_rows(l);
+    const int qkvd = (p.nq + 2 * p.nkv) * p.d;
+    const int qd = p.nq * p.d, kvd = p.nkv * p.d, cap = rows_cap(p.H, Q8W);
+    const uint32_t tag = p.tag0 + (uint32_t)(l - p.l0);
+    const bool publish = l != p.withhold_layer;
+    const int rb = Q8W ? p.H : 2 * p.H;
+    for (int n = a; n < b;) {
+      const int e = qkv_chunk_end(n, b, cap, qd, kvd), nr = e - n;
+      const unsigned char* st = chunk_wait();
+      int r0 = (warp - (n - a)) % kConsumerWarps;
+      if (r0 < 0) r0 += kConsumerWarps;
+      if (!quit) {
+        for (int rr = r0; rr < nr; rr += kConsumerWarps) {
+          float acc[NB];
+          row_dot(st + rr * rb,
+                  reinterpret_cast<const __half*>(st + kData) + rr * (p.H / 32), acc);
+          if (lane == 0 && publish) {
+#pragma unroll
+            for (int bb = 0; bb < NB; ++bb)
+              if (bb < p.B) st_tag(p.xq + (size_t)bb * qkvd + n + rr, acc[bb] * inv[bb], tag);
+          }
+        }
+      }
+      chunk_release();
+      n = e;
+    }
+    tr(l, 2);
+  }
+
+  // ---- phase B: attention units with their share of the O projection ------
+
+  // Per-lane constants of one head's RMSNorm + RoPE (elements lane*E + e of
+  // both halves, E = d/64).
+  struct HeadConst {
+    float g_lo[2], g_hi[2];
+    float2 cs[2];
+  };
+  __device__ __forceinline__ void head_const(const __nv_bfloat16* gain, int pos, HeadConst& hc) {
+    const int half = p.d / 2, E = p.d / 64;
+    const float2* rp = p.rope + (size_t)pos * half;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int i = lane * E + e;
+      const bool ok = e < E;
+      hc.g_lo[e] = ok ? __bfloat162float(gain[i]) : 0.f;
+      hc.g_hi[e] = ok ? __bfloat162float(gain[half + i]) : 0.f;
+      hc.cs[e] = ok ? rp[i] : make_float2(0.f, 0.f);
+    }
+  }
+  // Poll one head's d tagged words of xq into x_lo/x_hi (elements lane*E+e).
+  __device__ __forceinline__ void poll_head(const unsigned long long* src, uint32_t want,
+                                            float (&lo)[2], float (&hi)[2]) {
+    const int half = p.d / 2, E = p.d / 64;
+    unsigned long long xs[2][2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+#pragma unroll
+      for (int part = 0; part < 2; ++part)
+        xs[e][part] = e < E ? ld_word(src + lane * E + e + part * half) : 0ull;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      lo[e] = hi[e] = 0.f;
+      if (e >= E) continue;
+      const int i = lane * E + e;
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        const unsigned long long* w = src + i + part * half;
+        unsigned long long x = xs[e][part];
+        if ((uint32_t)(x >> 32) != want && !quit) {
+          unsigned long long t0 = 0;
+          int spins = 0;
+          do {
+            __nanosleep(20);
+            x = ld_word(w);
+            if ((++spins & 63) == 0) {
+              if (t0 == 0) t0 = now_ns();
+              if (aborted(p.abort_flag) || now_ns() - t0 > p.wait_ns) {
+                give_up();
+                break;
+              }
+            }
+          } while ((uint32_t)(x >> 32) != want);
+        }
+        (part ? hi[e] : lo[e]) = __uint_as_float((uint32_t)x);
+      }
+    }
+  }
+  // RMSNorm over the head (warp) + rotate-half RoPE; writes the d values.
+  __device__ __forceinline__ void head_norm_rope(float (&lo)[2], float (&hi)[2],
+                                                 const HeadConst& hc, float scale, float* out) {
+    const int half = p.d / 2, E = p.d / 64;
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+      if (e < E) ss += lo[e] * lo[e] + hi[e] * hi[e];
+    ss = warp_sum(ss);
+    const float inv = rsqrtf(ss / (float)p.d + p.eps);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      if (e >= E) break;
+      const int i = lane * E + e;
+      const float a = lo[e] * inv * hc.g_lo[e];
+      const float c = hi[e] * inv * hc.g_hi[e];
+      out[i] = (a * hc.cs[e].x - c * hc.cs[e].y) * scale;
+      out[half + i] = (c * hc.cs[e].x + a * hc.cs[e].y) * scale;
+    }
+  }
+
+  __device__ float* q_sm() { return attn; }                         // [rep][d]
+  __device__ float* k_sm() { return attn + kMaxRep * 128; }         // [d]
+  __device__ float* v_sm() { return attn + kMaxRep * 128 + 128; }   // [d]
+  __device__ float* st_sm() { return attn + kMaxRep * 128 + 256; }  // [11][rep][2 + 8]
+
+  // q heads, k and v of (row b, group g) into shared memory; the j = 0 unit
+  // also appends k and v (bf16) to the cache. Ends on a barrier.
+  __device__ void attn_prep(int l, int b, int g, int j) {
+    const int d = p.d, rep = p.nq / p.nkv, qd = p.nq * d, kvd = p.nkv * d;
+    const int qkvd = qd + 2 * kvd, pos = p.pos[b];
+    const LayerDev& Lw = layer_s(p, l);
+    const unsigned long long* row = p.xq + (size_t)b * qkvd;
+    const uint32_t want = p.tag0 + (uint32_t)(l - p.l0);
+    if (warp < rep) {
+      HeadConst hc;
+      head_const(Lw.q_norm, pos, hc);
+      float lo[2], hi[2];
+      poll_head(row + (g * rep + warp) * d, want, lo, hi);
+      head_norm_rope(lo, hi, hc, rsqrtf((float)d), q_sm() + warp * d);
+    } else if (warp == rep) {
+      HeadConst hc;
+      head_const(Lw.k_norm, pos, hc);
+      float lo[2], hi[2];
+      poll_head(row + qd + g * d, want, lo, hi);
+      head_norm_rope(lo, hi, hc, 1.f, k_sm());
+      __syncwarp();
+      const size_t off = kv_off(p, l, b, pos, g);
+      for (int i2 = lane; i2 < d; i2 += 32) {
+        const __nv_bfloat16 kb = __float2bfloat16_rn(k_sm()[i2]);
+        if (j == 0 && !quit) p.kv.k[off + i2] = kb;
+        k_sm()[i2] = __bfloat162float(kb);
+      }
+    } else if (warp == rep + 1) {
+      float lo[2], hi[2];
+      poll_head(row + qd + kvd + g * d, want, lo, hi);
+      const int half = d / 2, E = d / 64;
+      const size_t off = kv_off(p, l, b, pos, g);
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        if (e >= E) break;
+        const int i2 = lane * E + e;
+        const __nv_bfloat16 vl = __float2bfloat16_rn(lo[e]);
+        const __nv_bfloat16 vh = __float2bfloat16_rn(hi[e]);
+        if (j == 0 && !quit) {
+          p.kv.v[off + i2] = vl;
+          p.kv.v[off + half + i2] = vh;
+        }
+        v_sm()[i2] = __bfloat162float(vl);
+        v_sm()[half + i2] = __bfloat162float(vh);
+      }
+    }
+    consumer_sync();
+  }
+
+  // Online-softmax state of this lane: lane = (key kk = lane >> 2, quarter
+  // qq = lane & 3); the quarter holds dims [qq*d/4, (qq+1)*d/4) of the score
+  // dot products and dims 8j + 2qq, 8j + 2qq + 1 of the output slice.
+  struct AttnState {
+    float m[kMaxRep], l[kMaxRep], o[kMaxRep][2];
+  };
+
+  // One group of 8 keys (kk valid iff kk < nk): scores, update, P*V.
+  // q holds the lane's quarter of each head in rotated 8-element blocks:
+  // block c of the registers is block (c + kk) % (DQ/8) of the quarter, so
+  // the 8 key lanes of one quarter read different bank groups of their keys.
+  template <int DQ>
+  __device__ __forceinline__ void attend8(const float (&q)[kMaxRep][DQ], const __nv_bfloat16* Kp,
+                                          const __nv_bfloat16* Vp, int nk, int vcol, int rep,
+                                          AttnState& S) {
+    constexpr int NC = DQ / 8;
+    const int kk = lane >> 2, qq = lane & 3, d = 4 * DQ;
+    const bool valid = kk < nk;
+    float s[kMaxRep];
+#pragma unroll
+    for (int h = 0; h < kMaxRep; ++h) s[h] = 0.f;
+    if (valid) {
+      const __nv_bfloat16* krow = Kp + kk * d + qq * DQ;
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        const uint4 u = *reinterpret_cast<const uint4*>(krow + ((c + kk) % NC) * 8);
+        const float kf[8] = {lo16(u.x), hi16(u.x), lo16(u.y), hi16(u.y),
+                             lo16(u.z), hi16(u.z), lo16(u.w), hi16(u.w)};
+#pragma unroll
+        for (int h = 0; h < kMaxRep; ++h)
+#pragma unroll
+          for (int t = 0; t < 8; ++t) s[h] = fmaf(q[h][c * 8 + t], kf[t], s[h]);
+      }
+    }
+    float vv[2] = {0.f, 0.f};
+    if (valid) {
+      const uint32_t u = *reinterpret_cast<const uint32_t*>(Vp + kk * d + vcol + 2 * qq);
+      vv[0] = lo16(u);
+      vv[1] = hi16(u);
+    }
+#pragma unroll
+    for (int h = 0; h < kMaxRep; ++h) {
+      if (h >= rep) break;
+      float t = s[h];
+      t += __shfl_xor_sync(0xffffffffu, t, 1);
+      t += __shfl_xor_sync(0xffffffffu, t, 2);
+      t = valid ? t : -INFINITY;
+      float mx = t;
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const float mn = fmaxf(S.m[h], mx);
+      const float alpha = (S.m[h] == -INFINITY) ? 0.f : expf(S.m[h] - mn);
+      const float pr = valid ? expf(t - mn) : 0.f;
+      S.m[h] = mn;
+      // l: one copy per key lane (summed over keys at the end); quarters
+      // other than 0 keep l at zero.
+      S.l[h] = S.l[h] * alpha + (qq == 0 ? pr : 0.f);
+      S.o[h][0] = fmaf(pr, vv[0], S.o[h][0] * alpha);
+      S.o[h][1] = fmaf(pr, vv[1], S.o[h][1] * alpha);
+    }
+  }
+
+  template <int DQ>
+  __device__ void attn_keys(int l, int b, int g, int j, AttnState& S) {
+    const int rep = p.nq / p.nkv, old = p.pos[b];
+    float q[kMaxRep][DQ];
+    const int qq = lane & 3;
+    constexpr int NC = DQ / 8;
+    const int kk = lane >> 2;
+#pragma unroll
+    for (int h = 0; h < kMaxRep; ++h)
+#pragma unroll
+      for (int c = 0; c < NC; ++c)
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+          q[h][c * 8 + t] = h < rep ? q_sm()[h * 4 * DQ + qq * DQ + ((c + kk) % NC) * 8 + t] : 0.f;
+#pragma unroll
+    for (int h = 0; h < kMaxRep; ++h) {
+      S.m[h] = -INFINITY;
+      S.l[h] = 0.f;
+      S.o[h][0] = S.o[h][1] = 0.f;
+    }
+    const int vcol = j * kSlice;
+    // groups of 8 keys: group gi covers keys [8 gi, 8 gi + 8); warp w takes
+    // groups w, w + 11, ...; a page holds 8 groups.
+    for (int j0 = 0; j0 < old; j0 += kPage) {
+      const int nk = min(kPage, old - j0);
+      const __nv_bfloat16* Kp = reinterpret_cast<const __nv_bfloat16*>(chunk_wait(0));
+      const __nv_bfloat16* Vp = reinterpret_cast<const __nv_bfloat16*>(chunk_wait(1));
+      if (!quit) {
+        const int g0 = j0 / 8, g1 = (j0 + nk + 7) / 8;
+        int gi = g0 + ((warp - g0) % kConsumerWarps + kConsumerWarps) % kConsumerWarps;
+        for (; gi < g1; gi += kConsumerWarps) {
+          const int kbase = gi * 8 - j0;
+          attend8<DQ>(q, Kp + (size_t)kbase * 4 * DQ, Vp + (size_t)kbase * 4 * DQ,
+                      min(8, nk - kbase), vcol, rep, S);
+        }
+      }
+      chunk_release();  // K
+      chunk_release();  // V
+    }
+    (void)l;
+    (void)g;
+  }
+
+  // The new key (position pos, from k_sm / v_sm) on warp 0, then the merge of
+  // the warps' states into o_s[b][h][t]. Ends on a barrier.
+  template <int DQ>
+  __device__ void attn_finish(int b, int j, AttnState& S) {
+    const int rep = p.nq / p.nkv, d = 4 * DQ, qq = lane & 3, kk = lane >> 2;
+    if (warp == 0 && !quit) {
+      float s[kMaxRep];
+#pragma unroll
+      for (int h = 0; h < kMaxRep; ++h) {
+        float t = 0.f;
+        if (kk == 0 && h < rep)
+#pragma unroll
+          for (int c = 0; c < DQ; ++c) t = fmaf(q_sm()[h * d + qq * DQ + c], k_sm()[qq * DQ + c], t);
+        t += __shfl_xor_sync(0xffffffffu, t, 1);
+        t += __shfl_xor_sync(0xffffffffu, t, 2);
+        s[h] = __shfl_sync(0xffffffffu, t, 0);
+      }
+#pragma unroll
+      for (int h = 0; h < kMaxRep; ++h) {
+        if (h >= rep) break;
+        const float mn = fmaxf(S.m[h], s[h]);
+        const float alpha = (S.m[h] == -INFINITY) ? 0.f : expf(S.m[h] - mn);
+        const float pr = (kk == 0) ? expf(s[h] - mn) : 0.f;
+        S.m[h] = mn;
+        S.l[h] = S.l[h] * alpha + (qq == 0 ? pr : 0.f);
+        const float v0 = v_sm()[j * kSlice + 2 * qq], v1 = v_sm()[j * kSlice + 2 * qq + 1];
+        S.o[h][0] = fmaf(pr, v0, S.o[h][0] * alpha);
+        S.o[h][1] = fmaf(pr, v1, S.o[h][1] * alpha);
+      }
+    }
+    // reduce over the 8 key lanes (same quarter): lanes qq = 0..3 keep the sums
+#pragma unroll
+    for (int h = 0; h < kMaxRep; ++h) {
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        S.l[h] += __shfl_xor_sync(0xffffffffu, S.l[h], o);
+        S.o[h][0] += __shfl_xor_sync(0xffffffffu, S.o[h][0], o);
+        S.o[h][1] += __shfl_xor_sync(0xffffffffu, S.o[h][1], o);
+      }
+    }
+    float* ws = st_sm();  // [warp][h][0: m, 1: l, 2..9: o]
+    if (lane < 4) {
+#pragma unroll
+      for (int h = 0; h < kMaxRep; ++h) {
+        if (h >= rep) break;
+        float* e = ws + (warp * kMaxRep + h) * 10;
+        if (lane == 0) {
+          e[0] = S.m[h];
+          e[1] = S.l[h];
+        }
+        e[2 + 2 * lane] = S.o[h][0];
+        e[3 + 2 * lane] = S.o[h][1];
+      }
+    }
+    consumer_sync();
+    if (tid < rep * kSlice) {
+      const int h = tid / kSlice, t = tid % kSlice;
+      float M = -INFINITY;
+      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ws[(w * kMaxRep + h) * 10]);
+      float Lsum = 0.f, O = 0.f;
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float* e = ws + (w * kMaxRep + h) * 10;
+        const float f = (e[0] == -INFINITY) ? 0.f : expf(e[0] - M);
+        Lsum += e[1] * f;
+        O += e[2 + t] * f;
+      }
+      o_s()[(b * kMaxRep + h) * kSlice + t] = O / Lsum;
+    }
+    consumer_sync();
+  }
+
+  // Adds one contribution (per batch row: 4 consecutive elements from n4*4)
+  // to copy `copy` of accumulator version v; `with_input` adds the rows of rs.
+  __device__ __forceinline__ void contribute(int v, int copy, int n4, const float (&a)[NB][4],
+                                             bool with_input) {
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (b >= p.B) break;
+      unsigned long long* dst = acc_row(p, v, copy, b) + 4 * n4;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float x = a[b][e];
+        if (with_input) x += rs[b * p.H + 4 * n4 + e];
+        red_add(dst + e, fix_word(x));
+      }
+    }
+  }
+
+  // acc4[b][0..3] += s[b] * W[row][4 n4 .. 4 n4 + 4) for one row of a
+  // transposed matrix in shared memory (bf16, or Q8_0 codes with a scale row).
+  __device__ __forceinline__ void axpy_row(const unsigned char* row, const __half* srow, int n4,
+                                           const float (&s)[NB], float (&acc4)[NB][4]) {
+    float w[4];
+    if (!Q8W) {
+      const uint2 u = *reinterpret_cast<const uint2*>(row + 8 * n4);
+      w[0] = lo16(u.x); w[1] = hi16(u.x); w[2] = lo16(u.y); w[3] = hi16(u.y);
+    } else {
+      const uint32_t u = *reinterpret_cast<const uint32_t*>(row + 4 * n4);
+      const uint2 sv = *reinterpret_cast<const uint2*>(srow + 4 * n4);
+      const float s0 = __half2float(__ushort_as_half((unsigned short)(sv.x & 0xffff)));
+      const float s1 = __half2float(__ushort_as_half((unsigned short)(sv.x >> 16)));
+      const float s2 = __half2float(__ushort_as_half((unsigned short)(sv.y & 0xffff)));
+      const float s3 = __half2float(__ushort_as_half((unsigned short)(sv.y >> 16)));
+      w[0] = (float)(int8_t)(u & 0xff) * s0;
+      w[1] = (float)(int8_t)((u >> 8) & 0xff) * s1;
+      w[2] = (float)(int8_t)((u >> 16) & 0xff) * s2;
+      w[3] = (float)(int8_t)((u >> 24) & 0xff) * s3;
+    }
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc4[b][e] = fmaf(s[b], w[e], acc4[b][e]);
+  }
+
+  __device__ void phase_b(int l) {
+    tr(l, 3);
+    const int d = p.d, ds = d / kSlice, rep = p.nq / p.nkv, H = p.H;
+    for (int u = cta; u < p.n_units; u += G) {
+      const int g = u / ds, j = u % ds;
+      for (int b = 0; b < p.B; ++b) {
+        attn_prep(l, b, g, j);
+        if (b == 0) tr(l, 4);
+        AttnState S;
+        if (d == 128) {
+          attn_keys<32>(l, b, g, j, S);
+          attn_finish<32>(b, j, S);
+        } else {
+          attn_keys<16>(l, b, g, j, S);
+          attn_finish<16>(b, j, S);
+        }
+      }
+      tr(l, 5);
+      // O projection share: Wo^T rows (g*rep + h)*d + 8j + t
+      const int n4 = tid;
+      float acc4[NB][4];
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc4[b][e] = 0.f;
+      for (int h = 0; h < rep; ++h) {
+        const unsigned char* st = chunk_wait();
+        if (!quit && n4 < H / 4) {
+          const int rb = Q8W ? H : 2 * H;
+          const __half* srow = reinterpret_cast<const __half*>(st + kData);
+#pragma unroll 4
+          for (int t = 0; t < kSlice; ++t) {
+            float s[NB];
+#pragma unroll
+            for (int b = 0; b < NB; ++b) s[b] = o_s()[(b * kMaxRep + h) * kSlice + t];
+            axpy_row(st + t * rb, srow, n4, s, acc4);
+          }
+        }
+        chunk_release();
+      }
+      if (!quit && n4 < H / 4) contribute(2 * l, u % p.P, n4, acc4, u == 0);
+      consumer_sync();
+      if (tid == 0) release_count(p.cnt + (size_t)(2 * l) * kMaxCopies + u % p.P);
+    }
+    tr(l, 6);
+  }
+
+  // ---- phase C: RMSNorm + gate/up + SwiGLU + down share ------------------
+
+  __device__ void phase_c(int l, int a, int b) {
+    tr(l, 7);
+    const LayerDev& Lw = layer_s(p, l);
+    float gr[kEPT];
+    load_gains(Lw.ffn_norm, gr);
+    gather_norm(2 * l, p.n_units, gr, 1);
+    tr(l, 8);
+    const int H = p.H, pc = pairs_cap(H, Q8W), rb = Q8W ? H : 2 * H, sb = Q8W ? H / 32 : 0;
+    for (int n = a; n < b;) {
+      const int e = min(b, n + pc), nr = e - n;
+      const unsigned char* st = chunk_wait();
+      int r0 = (warp - (n - a)) % kConsumerWarps;
+      if (r0 < 0) r0 += kConsumerWarps;
+      if (!quit) {
+        for (int rr = r0; rr < nr; rr += kConsumerWarps) {
+          float gv[NB], uv[NB];
+          const __half* sg = reinterpret_cast<const __half*>(st + kData) + rr * sb;
+          const __half* su = reinterpret_cast<const __half*>(st + kData) + (pc + rr) * sb;
+          row_dot(st + rr * rb, sg, gv);
+          row_dot(st + (pc + rr) * rb, su, uv);
+          if (lane == 0) {
+#pragma unroll
+            for (int bb = 0; bb < NB; ++bb) {
+              if (bb >= p.B) break;
+              const float y = gv[bb] * inv[bb], z = uv[bb] * inv[bb];
+              act_s()[bb * 128 + (n - a) + rr] = y / (1.f + expf(-y)) * z;
+            }
+          }
+        }
+      }
+      chunk_release();
+      n = e;
+    }
+    consumer_sync();
+    tr(l, 9);
+    const int n4 = tid, rc = rows_cap(H, Q8W);
+    float acc4[NB][4];
+#pragma unroll
+    for (int bb = 0; bb < NB; ++bb)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc4[bb][e] = 0.f;
+    for (int n = a; n < b;) {
+      const int e = down_chunk_end(n, b, rc, Q8W), nr = e - n;
+      const unsigned char* st = chunk_wait();
+      if (!quit && n4 < H / 4) {
+        const __half* srow = reinterpret_cast<const __half*>(st + kData);
+        for (int t = 0; t < nr; ++t) {
+          float s[NB];
+#pragma unroll
+          for (int bb = 0; bb < NB; ++bb) s[bb] = act_s()[bb * 128 + (n - a) + t];
+          axpy_row(st + t * rb, srow, n4, s, acc4);
+        }
+      }
+      chunk_release();
+      n = e;
+    }
+    if (!quit && a < b && n4 < H / 4) contribute(2 * l + 1, cta % p.P, n4, acc4, cta == 0);
+    consumer_sync();
+    if (tid == 0 && a < b) release_count(p.cnt + (size_t)(2 * l + 1) * kMaxCopies + cta % p.P);
+    tr(l, 10);
+  }
+
+  // ---- tail: final norm + LM head + greedy, or the block output -----------
+
+  __device__ void tail(int a, int b) {
+    const int L = p.L;
+    tr(L, 0);
+    float gr[kEPT];
+    load_gains(p.final_norm, gr);
+    if (!p.run_head) {
+      // the block output: only CTA 0 waits for it (gather_norm's barrier is
+      // CTA-local)
+      if (cta == 0) {
+        gather_norm(2 * (p.l1 - 1) + 1, p.c_ctas, gr, 0);
+        capture_rows(p.l1);
+        if (p.h_out)
+          for (int k = tid; k < p.B * p.H; k += kConsumers) p.h_out[k] = rs[k];
+      }
+      return;
+    }
+    gather_norm(2 * (p.l1 - 1) + 1, p.c_ctas, gr, 0);
+    tr(L, 1);
+    consumer_sync();  // rs complete before CTA 0 copies it out
+    capture_rows(p.l1);
+    if (cta == 0 && p.h_out)
+      for (int k = tid; k < p.B * p.H; k += kConsumers) p.h_out[k] = rs[k];
+    const int cap = p.lm_rows, rb = 2 * p.H;
+    for (int n = a; n < b && p.lm_owner;) {
+      const int e = min(b, n + cap), nr = e - n;
+      if ((int)(i % kConsumerWarps) == warp) {
+        const unsigned char* st = chunk_wait_owned();
+        if (!quit) lm_rows_owned(st, n, nr);
+        __syncwarp();
+        if (lane == 0) mbar_arrive_n(&r.empty[stage], kConsumerWarps);
+      }
+      cursor_advance();
+      n = e;
+    }
+    for (int n = a; n < b && !p.lm_owner;) {
+      const int e = min(b, n + cap), nr = e - n;
+      const unsigned char* st = chunk_wait();
+      int r0 = (warp - (n - a)) % kConsumerWarps;
+      if (r0 < 0) r0 += kConsumerWarps;
+      if (!quit) {
+        for (int rr = r0; rr < nr; rr += kConsumerWarps) {
+          float acc[NB];
+          lm_dot(st + rr * rb, acc);
+          if (lane == 0) {
+#pragma unroll
+            for (int bb = 0; bb < NB; ++bb) {
+              if (bb >= p.B) break;
+              fold_logit(bb, n + rr, acc[bb] * inv[bb]);
+            }
+          }
+        }
+      }
+      chunk_release();
+      n = e;
+    }
+    tr(L, 2);
+    finish_head();
+  }
+
+  // Sum of 8 per-lane values over the warp in 9 shuffles: each step halves
+  // the values a lane keeps. Lane l ends with the total of value
+  // 4*bit4(l) + 2*bit3(l) + bit2(l).
+  __device__ __forceinline__ float reduce8(const float (&v)[8]) {
+    const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4;
+    float a4[4], c2[2];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float keep = h16 ? v[r + 4] : v[r], send = h16 ? v[r] : v[r + 4];
+      a4[r] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const float keep = h8 ? a4[r + 2] : a4[r], send = h8 ? a4[r] : a4[r + 2];
+      c2[r] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    const float keep = h4 ? c2[1] : c2[0], send = h4 ? c2[0] : c2[1];
+    float t = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    t += __shfl_xor_sync(0xffffffffu, t, 2);
+    t += __shfl_xor_sync(0xffffffffu, t, 1);
+    return t;
+  }
+
+  // Greedy key of logit y at vocabulary id `id`: order-preserving in y (+0 and
+  // -0 equal), and on equal y the lower id is the larger key.
+  __device__ __forceinline__ void fold_logit(int bb, int id, float y) {
+    if (p.logits) p.logits[(size_t)bb * p.V + id] = y;
+    if (isfinite(y)) {
+      const uint32_t uu = (y == 0.f) ? 0u : __float_as_uint(y);
+      const uint32_t ord = (uu & 0x80000000u) ? ~uu : (uu | 0x80000000u);
+      const unsigned long long key = ((unsigned long long)ord << 32) | (0xffffffffu - (uint32_t)id);
+#pragma unroll
+      for (int b2 = 0; b2 < kMaxB; ++b2)
+        if (b2 == bb && key > wbest[b2]) wbest[b2] = key;
+    }
+  }
+
+  // All rows (up to 8) of an LM-head chunk on this warp: the lane's 8-element
+  // blocks of every row with shared activation loads, one transposing
+  // reduction per batch row.
+  __device__ __forceinline__ void lm_rows_owned(const unsigned char* st, int n0, int nr) {
+    const int H = p.H;
+    float acc[8][NB];
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+      for (int b = 0; b < NB; ++b) acc[r][b] = 0.f;
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+      const int k = lane * 8 + it * 256;
+      float z[NB][8];
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        if (b < p.B) {
+          const float4 z0 = *reinterpret_cast<const float4*>(zs + b * H + k);
+          const float4 z1 = *reinterpret_cast<const float4*>(zs + b * H + k + 4);
+          z[b][0] = z0.x; z[b][1] = z0.y; z[b][2] = z0.z; z[b][3] = z0.w;
+          z[b][4] = z1.x; z[b][5] = z1.y; z[b][6] = z1.z; z[b][7] = z1.w;
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) z[b][q] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        if (r >= nr) break;
+        const uint4 u = *reinterpret_cast<const uint4*>(st + r * 2 * H + 2 * k);
+        const float w[8] = {lo16(u.x), hi16(u.x), lo16(u.y), hi16(u.y),
+                            lo16(u.z), hi16(u.z), lo16(u.w), hi16(u.w)};
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) acc[r][b] = fmaf(w[q], z[b][q], acc[r][b]);
+      }
+    }
+    const int my_r = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      float col[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) col[r] = acc[r][b];
+      const float tot = reduce8(col);
+      if (b < p.B && (lane & 3) == 0 && my_r < nr) fold_logit(b, n0 + my_r, tot * inv[b]);
+    }
+  }
+
+  // bf16 row dot for the LM head (the embedding is bf16 in every format).
+  __device__ __forceinline__ void lm_dot(const unsigned char* row, float (&acc)[NB]) {
+    const int H = p.H;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) acc[b] = 0.f;
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+      const int k = lane * 8 + it * 256;
+      const uint4 u = *reinterpret_cast<const uint4*>(row + 2 * k);
+      const float w[8] = {lo16(u.x), hi16(u.x), lo16(u.y), hi16(u.y),
+                          lo16(u.z), hi16(u.z), lo16(u.w), hi16(u.w)};
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        if (b < p.B) {
+          const float4 z0 = *reinterpret_cast<const float4*>(zs + b * H + k);
+          const float4 z1 = *reinterpret_cast<const float4*>(zs + b * H + k + 4);
+          float t = acc[b];
+          t = fmaf(w[0], z0.x, t); t = fmaf(w[1], z0.y, t); t = fmaf(w[2], z0.z, t);
+          t = fmaf(w[3], z0.w, t); t = fmaf(w[4], z1.x, t); t = fmaf(w[5], z1.y, t);
+          t = fmaf(w[6], z1.z, t); t = fmaf(w[7], z1.w, t);
+          acc[b] = t;
+        }
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < NB; ++b) acc[b] = warp_sum(acc[b]);
+  }
+
+  // Fold this CTA's greedy keys; the last CTA to finish writes the ids.
+  __device__ void finish_head() {
+    if (tid < kMaxB) best[tid] = 0ull;
+    consumer_sync();
+#pragma unroll
+    for (int bb = 0; bb < kMaxB; ++bb) {
+      unsigned long long k = wbest[bb];
+      for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long other = __shfl_xor_sync(0xffffffffu, k, o);
+        k = other > k ? other : k;
+      }
+      if (lane == 0 && bb < p.B && k) atomicMax(best + bb, k);
+    }
+    consumer_sync();
+    if (tid < p.B && !quit && best[tid]) atomicMax(p.am_key + tid, best[tid]);
+    __threadfence();
+    consumer_sync();
+    if (tid == 0) {
+      const unsigned int old = atomicAdd(p.am_cnt, 1u);
+      *flag = (old == (unsigned int)G - 1);
+    }
+    consumer_sync();
+    if (*flag) {
+      __threadfence();
+      if (tid < p.B) {
+        const unsigned long long key = atomicExch(p.am_key + tid, 0ull);
+        int id = 0;
+        if (key == 0ull) {
+          if (!quit) atomicCAS(p.err, 0, kErrBounds);
+        } else {
+          id = (int)(0xffffffffu - (uint32_t)(key & 0xffffffffu));
+        }
+        if (p.argmax) p.argmax[tid] = id;
+      }
+      if (tid == 0) atomicExch(p.am_cnt, 0u);
+    }
+    tr(p.L, 4);
+  }
+};
+
+template <int NB, bool Q8W, int IT>
+__global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_constant__ Params p) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  Ring ring;
+  ring.stages = smem;
+  ring.n = p.n_stages;
+  ring.full = reinterpret_cast<uint64_t*>(smem + p.off_bar);
+  ring.empty = ring.full + kMaxStages;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.n_stages; ++s) {
+      mbar_init(&ring.full[s], 1);
+      mbar_init(&ring.empty[s], kConsumerWarps);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  {
+    const unsigned* src = reinterpret_cast<const unsigned*>(p.layers);
+    unsigned* dst = reinterpret_cast<unsigned*>(smem + p.off_tab);
+    const int words = p.L * (int)sizeof(LayerDev) / 4;
+    for (int k = threadIdx.x; k < words; k += blockDim.x) dst[k] = src[k];
+    const unsigned* tsrc = reinterpret_cast<const unsigned*>(p.tl);
+    unsigned* tdst = dst + words;
+    const int twords = p.L * (int)sizeof(TLayer) / 4;
+    for (int k = threadIdx.x; k < twords; k += blockDim.x) tdst[k] = tsrc[k];
+    if (p.bt_in_smem) {
+      int32_t* bt = reinterpret_cast<int32_t*>(smem + p.off_tab +
+                                               (size_t)p.L * (sizeof(LayerDev) + sizeof(TLayer)));
+      const int pps = p.kv.pages_per_seq;
+      for (int k = threadIdx.x; k < p.B * pps; k += blockDim.x)
+        bt[k] = p.kv.block_table[(size_t)p.seq[k / pps] * pps + k % pps];
+    }
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = gridDim.x, c = blockIdx.x;
+  const int qkvd = (p.nq + 2 * p.nkv) * p.d;
+  volatile unsigned int* counts =
+      reinterpret_cast<volatile unsigned int*>(smem + p.off_misc + 4096 + 8 * kMaxB + 8);
+  if (warp == kConsumerWarps) {
+    if (lane == 0) {
+      Producer pr(p, ring);
+      for (int l = p.l0; l < p.l1 && !pr.quit; ++l) {
+        int a, b;
+        slice(qkvd, G, c, a, b);
+        pr.phase_a(l, a, b);
+        pr.phase_b(l, c, G);
+        slice(p.I, G, c, a, b);
+        pr.phase_c(l, a, b);
+      }
+      int a, b;
+      slice(p.V, G, c, a, b);
+      if (!pr.quit) pr.tail(a, b);
+      if (p.trace) p.trace[((size_t)c * (p.L + 1) + p.L) * kTraceSlots + 3] = now_ns();
+      counts[0] = pr.i;
+    } else {
+      // the idle lanes clear this CTA's share of the other accumulator set
+      long long a0 = p.clear_words * c / G, a1 = p.clear_words * (c + 1) / G;
+      for (long long k = a0 + lane - 1; k < a1; k += 31) p.clear[k] = 0ull;
+    }
+  } else {
+    Consumer<NB, Q8W, IT> cs(p, ring, smem);
+    for (int l = p.l0; l < p.l1 && !cs.quit; ++l) {
+      int a, b;
+      slice(qkvd, G, c, a, b);
+      cs.phase_a(l, a, b);
+      cs.phase_b(l);
+      slice(p.I, G, c, a, b);
+      cs.phase_c(l, a, b);
+    }
+    int a, b;
+    slice(p.V, G, c, a, b);
+    cs.tail(a, b);
+    if (threadIdx.x == 0) counts[1] = cs.i;
+  }
+  __syncthreads();
+  // Drain: copies issued but never consumed (after an abort) must land before
+  // the CTA's shared memory is released.
+  if (threadIdx.x == 0) {
+    const unsigned int issued = counts[0], used = counts[1];
+    const unsigned int n = (unsigned int)ring.n;
+    const unsigned int first = issued > n ? issued - n : 0u;  // the newest copy of each stage
+    (void)used;
+    for (unsigned int k = first; k < issued; ++k) {
+      const unsigned long long t0 = now_ns();
+      while (!mbar_test(&ring.full[k % n], (k / n) & 1))
+        if (now_ns() - t0 > 10000000ull) break;  // 10 ms
+    }
+  }
+}
+
+// Transposes of Wo and Wd for the fused O and down shares.
+template <typename T>
+__global__ void transpose_kernel(const T* __restrict__ in, int rows, int cols, T* __restrict__ out) {
+  __shared__ T tile[32][33];
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int y = threadIdx.y; y < 32; y += 8) {
+    const int r = r0 + y, c = c0 + threadIdx.x;
+    if (r < rows && c < cols) tile[y][threadIdx.x] = in[(size_t)r * cols + c];
+  }
+  __syncthreads();
+  for (int y = threadIdx.y; y < 32; y += 8) {
+    const int c = c0 + y, r = r0 + threadIdx.x;
+    if (r < rows && c < cols) out[(size_t)c * rows + r] = tile[threadIdx.x][y];
+  }
+}
+
+}  // namespace fused
+
+// ---------------------------------------------------------------------------
+// Host side
+
+namespace {
+
+struct FusedState {
+  unsigned long long* xq = nullptr;
+  unsigned long long* acc = nullptr;  // [2 sets][set words]
+  long long set_words = 0;
+  long long dirty[2] = {0, 0};        // words of each set written since its last clear
+  unsigned long long* am_key = nullptr;
+  unsigned int* am_cnt = nullptr;
+  int* abort_flag = nullptr;
+  LayerDev* layers = nullptr;
+  fused::TLayer* tl = nullptr;
+  void* wo_t[64] = {};
+  void* wd_t[64] = {};
+  void* so_t[64] = {};
+  void* sd_t[64] = {};
+  uint32_t next_tag = 1;
+  unsigned long long step = 0;
+  int sms = 0;
+  bool eligible = false;
+  unsigned long long wait_ns = 1000000000ull;
+  int withhold = -1;
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool shape_ok(const fs_model* m) {
+  const Shape& s = m->s;
+  const int rep = s.nq / s.nkv;
+  if (rep < 1 || rep > fused::kMaxRep || (s.d != 64 && s.d != 128)) return false;
+  if (s.H != 256 && s.H != 1024) return false;
+  if (s.V >= 0x7fffffff || s.L > 64) return false;
+  if (s.I % 32 || s.q_dim() % 32) return false;
+  if (s.I < m->num_sms) return false;  // every CTA owns intermediate columns
+  if (s.I / m->num_sms + 2 > 128) return false;  // act_s holds 128 columns per row
+  if (fused::rows_cap(s.H, m->q8) < 1 || fused::pairs_cap(s.H, m->q8) < 1) return false;
+  return true;
+}
+
+void state_free(FusedState* st) {
+  void* bufs[] = {st->xq, st->acc, st->am_key, st->am_cnt, st->abort_flag, st->layers, st->tl};
+  for (void* b : bufs)
+    if (b) cudaFree(b);
+  for (int l = 0; l < 64; ++l) {
+    if (st->wo_t[l]) cudaFree(st->wo_t[l]);
+    if (st->wd_t[l]) cudaFree(st->wd_t[l]);
+    if (st->so_t[l]) cudaFree(st->so_t[l]);
+    if (st->sd_t[l]) cudaFree(st->sd_t[l]);
+  }
+}
+
+template <typename T>
+void launch_transpose(const void* in, int rows, int cols, void* out) {
+  dim3 grid((cols + 31) / 32, (rows + 31) / 32), block(32, 8);
+  count_launches();
+  fused::transpose_kernel<T><<<grid, block>>>(static_cast<const T*>(in), rows, cols,
+                                              static_cast<T*>(out));
+}
+
+}  // namespace
+
+bool fused_eligible(const fs_model* m) {
+  const FusedState* st = static_cast<const FusedState*>(m->extras);
+  return st && st->eligible;
+}
+
+fs_status fused_init(fs_model* m) {
+  FusedState* st = new FusedState();
+  m->extras = st;
+  st->sms = m->num_sms;
+  st->eligible = shape_ok(m);
+  if (!st->eligible) return FS_OK;
+  const Shape& s = m->s;
+  auto alloc = [&](void** p, size_t bytes) {
+    if (cudaMalloc(p, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      *p = nullptr;
+      return false;
+    }
+    cudaMemset(*p, 0, bytes);
+    return true;
+  };
+  const size_t w = sizeof(unsigned long long);
+  // per set: arrival counters [2L][kMaxCopies], then the accumulator words
+  st->set_words = (long long)2 * s.L * fused::kMaxCopies * (1 + fused::kMaxB * s.H);
+  bool ok = alloc((void**)&st->xq, (size_t)fused::kMaxB * s.qkv_dim() * w) &&
+            alloc((void**)&st->acc, (size_t)2 * st->set_words * w) &&
+            alloc((void**)&st->am_key, (size_t)fused::kMaxB * w) &&
+            alloc((void**)&st->am_cnt, 64) && alloc((void**)&st->abort_flag, 64) &&
+            alloc((void**)&st->layers, (size_t)s.L * sizeof(LayerDev)) &&
+            alloc((void**)&st->tl, (size_t)s.L * sizeof(fused::TLayer));
+  // Transposed Wo [H][nq d] -> [nq d][H] and Wd [H][I] -> [I][H] (codes and
+  // scales for Q8_0), library-owned.
+  std::vector<fused::TLayer> tl(s.L);
+  for (int l = 0; ok && l < s.L; ++l) {
+    const LayerDev& Lw = m->layers[l];
+    const size_t eb = m->q8 ? 1 : 2;
+    ok = alloc(&st->wo_t[l], (size_t)s.q_dim() * s.H * eb) &&
+         alloc(&st->wd_t[l], (size_t)s.I * s.H * eb);
+    if (ok && m->q8)
+      ok = alloc(&st->so_t[l], (size_t)(s.q_dim() / 32) * s.H * 2) &&
+           alloc(&st->sd_t[l], (size_t)(s.I / 32) * s.H * 2);
+    if (!ok) break;
+    if (m->q8) {
+      launch_transpose<int8_t>(Lw.w[kWo], s.H, s.q_dim(), st->wo_t[l]);
+      launch_transpose<int8_t>(Lw.w[kWd], s.H, s.I, st->wd_t[l]);
+      launch_transpose<unsigned short>(Lw.s[kWo], s.H, s.q_dim() / 32, st->so_t[l]);
+      launch_transpose<unsigned short>(Lw.s[kWd], s.H, s.I / 32, st->sd_t[l]);
+    } else {
+      launch_transpose<unsigned short>(Lw.w[kWo], s.H, s.q_dim(), st->wo_t[l]);
+      launch_transpose<unsigned short>(Lw.w[kWd], s.H, s.I, st->wd_t[l]);
+    }
+    tl[l] = fused::TLayer{st->wo_t[l], static_cast<const __half*>(st->so_t[l]), st->wd_t[l],
+                          static_cast<const __half*>(st->sd_t[l])};
+  }
+  if (!ok || cudaGetLastError() != cudaSuccess) {
+    state_free(st);
+    delete st;
+    m->extras = nullptr;
+    set_error("out of device memory for the decode kernel's buffers");
+    return FS_ERR_OOM;
+  }
+  cudaMemcpy(st->layers, m->layers.data(), (size_t)s.L * sizeof(LayerDev), cudaMemcpyHostToDevice);
+  cudaMemcpy(st->tl, tl.data(), (size_t)s.L * sizeof(fused::TLayer), cudaMemcpyHostToDevice);
+  const void* kernels[] = {
+      (const void*)fused::decode_fused_kernel<1, false, 4>, (const void*)fused::decode_fused_kernel<1, true, 4>,
+      (const void*)fused::decode_fused_kernel<4, false, 4>, (const void*)fused::decode_fused_kernel<4, true, 4>,
+      (const void*)fused::decode_fused_kernel<1, false, 1>, (const void*)fused::decode_fused_kernel<1, true, 1>,
+      (const void*)fused::decode_fused_kernel<4, false, 1>, (const void*)fused::decode_fused_kernel<4, true, 1>};
+  for (const void* k : kernels)
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+  return FS_OK;
+}
+
+void fused_release(fs_model* m) {
+  FusedState* st = static_cast<FusedState*>(m->extras);
+  if (!st) return;
+  state_free(st);
+  delete st;
+  m->extras = nullptr;
+}
+
+// Clears the exchange state after a step was aborted (device error seen).
+void fused_reset(fs_model* m) {
+  FusedState* st = static_cast<FusedState*>(m->extras);
+  if (!st || !st->eligible) return;
+  cudaDeviceSynchronize();
+  cudaMemset(st->acc, 0, (size_t)2 * st->set_words * sizeof(unsigned long long));
+  st->dirty[0] = st->dirty[1] = 0;
+  cudaMemset(st->am_key, 0, (size_t)fused::kMaxB * sizeof(unsigned long long));
+  cudaMemset(st->am_cnt, 0, 64);
+  cudaMemset(st->abort_flag, 0, 64);
+  st->next_tag += 1u << 20;  // every tag in flight is now stale
+}
+
+void fused_debug_wait(fs_model* m, unsigned long long wait_ns, int withhold_layer) {
+  FusedState* st = static_cast<FusedState*>(m->extras);
+  if (!st) return;
+  st->wait_ns = wait_ns;
+  st->withhold = withhold_layer;
+}
+
+fs_status decode_fused(fs_model* m, const fs_kv* kv, const RowMap& map, int B, const int32_t* tok,
+                       const float* h_in, float* h_out, int l0, int l1, bool run_head,
+                       float* logits, int32_t* argmax, cudaStream_t stream) {
+  FusedState* st = static_cast<FusedState*>(m->extras);
+  if (!st || !st->eligible || B > fused::kMaxB || B < 1) return FS_ERR_UNSUPPORTED;
+  const Shape& s = m->s;
+  fused::Params p{};
+  p.L = s.L; p.H = s.H; p.nq = s.nq; p.nkv = s.nkv; p.d = s.d; p.I = s.I; p.V = s.V;
+  p.eps = s.eps;
+  p.q8 = m->q8 ? 1 : 0;
+  p.layers = st->layers;
+  p.tl = st->tl;
+  p.embed = m->embed;
+  p.final_norm = m->final_norm;
+  p.rope = m->rope;
+  p.kv = kv_view(kv);
+  p.B = B;
+  for (int b = 0; b < B; ++b) {
+    const RowInfo ri = map.get(b);
+    p.seq[b] = ri.seq;
+    p.pos[b] = ri.pos;
+  }
+  p.tokens = tok;
+  p.xq = st->xq;
+  const int set = (int)(st->step & 1);
+  p.cnt = st->acc + (size_t)set * st->set_words;
+  p.acc = p.cnt + (size_t)2 * s.L * fused::kMaxCopies;
+  p.P = std::max(1, std::min(fused::kMaxCopies, fused::kMaxCopies / B));
+  // the other set: clear the rows its last user wrote
+  p.clear = st->acc + (size_t)(1 - set) * st->set_words;
+  p.clear_words = st->dirty[1 - set];
+  st->dirty[1 - set] = 0;
+  st->dirty[set] = std::max(st->dirty[set], (long long)2 * s.L * (fused::kMaxCopies + p.P * B * s.H));
+  p.n_units = s.nkv * (s.d / fused::kSlice);
+  p.c_ctas = std::min(s.I, st->sms);
+  p.l0 = l0;
+  p.l1 = l1;
+  p.h_in = h_in;
+  p.h_out = h_out;
+  p.run_head = run_head ? 1 : 0;
+  p.logits = logits;
+  p.argmax = argmax;
+  p.am_key = st->am_key;
+  p.am_cnt = st->am_cnt;
+  p.capture = m->capture;
+  p.capture_stride = m->capture_max_rows;
+  p.err = m->err;
+  p.abort_flag = st->abort_flag;
+  p.wait_ns = st->wait_ns;
+  p.withhold_layer = st->withhold;
+  st->withhold = -1;  // one-shot
+  p.trace = m->trace;
+  m->trace = nullptr;  // one-shot
+  if (st->next_tag > 0xF0000000u) {
+    // wrap: clear the tags so the numbering can restart
+    cudaStreamSynchronize(stream);
+    cudaMemsetAsync(st->xq, 0, (size_t)fused::kMaxB * s.qkv_dim() * sizeof(unsigned long long),
+                    stream);
+    st->next_tag = 1;
+  }
+  p.tag0 = st->next_tag;
+  st->next_tag += (uint32_t)(l1 - l0) + 1u;
+  // shared memory carve-up
+  const size_t rows_bytes = align_up((size_t)B * s.H * 4, 128);
+  const size_t misc = 4096 + 256;
+  const size_t attn = align_up((size_t)(fused::kMaxRep * 128 + 256 +
+                                        fused::kConsumerWarps * fused::kMaxRep * 10) * 4, 128);
+  const size_t tab_ptrs = (size_t)s.L * (sizeof(LayerDev) + sizeof(fused::TLayer));
+  const size_t bt_bytes = (size_t)B * kv->pages_per_seq * sizeof(int32_t);
+  const bool bt_smem = bt_bytes <= 8192;
+  const size_t tab = align_up(tab_ptrs + (bt_smem ? bt_bytes : 0), 128);
+  const size_t bars = 2 * fused::kMaxStages * 8;
+  const size_t fixed = 3 * rows_bytes + misc + attn + tab + bars;
+  const size_t budget = 232448;
+  int n_stages = (int)((budget - fixed) / fused::kStageBytes);
+  n_stages = std::min(n_stages, fused::kMaxStages);
+  if (n_stages < 4) return FS_ERR_UNSUPPORTED;
+  size_t off = (size_t)n_stages * fused::kStageBytes;
+  p.off_r = (int)off; off += rows_bytes;
+  p.off_z = (int)off; off += 2 * rows_bytes;
+  p.off_misc = (int)off; off += misc;
+  p.off_attn = (int)off; off += attn;
+  p.off_bar = (int)off; off += bars;
+  p.off_tab = (int)off; off += tab;
+  p.bt_in_smem = bt_smem ? 1 : 0;
+  p.n_stages = n_stages;
+  p.lm_owner = n_stages >= fused::kConsumerWarps ? 1 : 0;
+  p.lm_rows = std::min(8, fused::rows_cap(s.H, false));
+  void* args[] = {&p};
+  const bool h1k = s.H == 1024;
+  const void* fn;
+  if (B == 1)
+    fn = m->q8 ? (h1k ? (const void*)fused::decode_fused_kernel<1, true, 4>
+                      : (const void*)fused::decode_fused_kernel<1, true, 1>)
+               : (h1k ? (const void*)fused::decode_fused_kernel<1, false, 4>
+                      : (const void*)fused::decode_fused_kernel<1, false, 1>);
+  else
+    fn = m->q8 ? (h1k ? (const void*)fused::decode_fused_kernel<4, true, 4>
+                      : (const void*)fused::decode_fused_kernel<4, true, 1>)
+               : (h1k ? (const void*)fused::decode_fused_kernel<4, false, 4>
+                      : (const void*)fused::decode_fused_kernel<4, false, 1>);
+  count_launches();
+  cudaError_t e = cudaLaunchCooperativeKernel(fn, dim3(st->sms), dim3(fused::kThreads), args, off,
+                                              stream);
+  if (e != cudaSuccess) {
+    set_error(std::string("decode kernel launch failed: ") + cudaGetErrorString(e));
+    return FS_ERR_CUDA;
+  }
+  ++st->step;
+  return FS_OK;
+}
+
+}  // namespace fs

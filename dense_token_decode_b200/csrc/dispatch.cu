@@ -5,10 +5,10 @@
 
 namespace fs {
 
-fs_status init_extras(fs_model* m) { return mega_init(m); }
+fs_status init_extras(fs_model* m) { return fused_init(m); }
 
 void release_extras(fs_model* m) {
-  mega_release(m);
+  fused_release(m);
   tc_release(m);
 }
 
@@ -44,8 +44,8 @@ fs_status block_prefill_or_general(fs_model* m, const fs_kv* kv, const RowMap& m
 fs_status decode_rows(fs_model* m, const fs_kv* kv, const RowMap& map, int rows,
                       const int32_t* tok, float* logits, int32_t* argmax, cudaStream_t st) {
   // Distinct sequences (checked by the caller), at most 4: the persistent kernel.
-  fs_status s = decode_mega(m, kv, map, rows, tok, nullptr, nullptr, 0, m->s.L, true, logits,
-                            argmax, st);
+  fs_status s = decode_fused(m, kv, map, rows, tok, nullptr, nullptr, 0, m->s.L, true, logits,
+                             argmax, st);
   if (s != FS_ERR_UNSUPPORTED) return s;
   return forward_general(m, kv, map, rows, tok, 0, logits, argmax, 0, rows, st);
 }

@@ -131,6 +131,12 @@ cudaError_t launch_attention_decode(const float* q, int rows, const RowMap& map,
 cudaError_t launch_lm_head(const float* xf, int rows, const Shape& s, const __nv_bfloat16* E,
                            float* logits, int32_t* argmax, float2* partial, int n_part, int* err,
                            cudaStream_t st);
+// Seeded sampling of one id per row (sample.cu): temperature > 0, top_k (0 =
+// off), top_p in (0, 1]; the draw of row r uses Philox4x32-10 at counter
+// (step, r).
+cudaError_t launch_sample(const float* logits, int rows, int V, float temperature, int top_k,
+                          float top_p, unsigned long long seed, unsigned long long step,
+                          int32_t* out, cudaStream_t st);
 cudaError_t launch_dequant_q8_0(const int8_t* codes, const __half* scales, int n, int k,
                                 float* out, cudaStream_t st);
 cudaError_t launch_kv_copy(KVView kv, int seq, int layer, int pos0, int n, __nv_bfloat16* k,

@@ -224,7 +224,7 @@ extern "C" fs_status fs_device_error(fs_model* m, int32_t* code) {
   int v = 0;
   FS_CUDA(cudaMemcpy(&v, m->err, sizeof(int), cudaMemcpyDeviceToHost));
   FS_CUDA(cudaMemset(m->err, 0, sizeof(int)));
-  if (v) fs::mega_reset(m);
+  if (v) fs::fused_reset(m);
   *code = v;
   return FS_OK;
 }
@@ -564,12 +564,41 @@ extern "C" fs_status fs_decode_step(fs_model* m, fs_kv* kv, const int32_t* seqs,
 }
 
 // ---------------------------------------------------------------------------
-// Greedy generation
+// Generation: greedy (fs_greedy) and seeded sampling (fs_generate)
 
-extern "C" fs_status fs_greedy(fs_model* m, fs_kv* kv, int32_t seq, const int32_t* prompt,
-                               int32_t n_prompt, int32_t max_new, const int32_t* eos,
-                               int32_t n_eos, int32_t* out_tokens, int32_t* n_out,
-                               int32_t* stop_reason, void* stream) {
+namespace {
+
+struct Sampler {
+  float temperature;  // > 0 (greedy generation passes no sampler)
+  int32_t top_k;
+  float top_p;
+  uint64_t seed;
+};
+
+fs_status check_sampler(float temperature, int32_t top_k, float top_p) {
+  if (!(temperature >= 0.f) || !std::isfinite(temperature))
+    return fail(FS_ERR_INVALID, "temperature must be finite and >= 0");
+  if (top_k < 0) return fail(FS_ERR_INVALID, "top_k must be >= 0");
+  if (!(top_p > 0.f && top_p <= 1.f)) return fail(FS_ERR_INVALID, "top_p must be in (0, 1]");
+  return FS_OK;
+}
+
+// The next id from the last row's logits (lg, device fp32 [V]) into *dst:
+// the sampler's draw for generated-token index `step`.
+fs_status sample_into(fs_model* m, const Sampler& sp, const float* lg, uint64_t step, int32_t* dst,
+                      cudaStream_t st) {
+  FS_CUDA(fs::launch_sample(lg, 1, m->s.V, sp.temperature, sp.top_k, sp.top_p, sp.seed, step, dst,
+                            st));
+  return FS_OK;
+}
+
+// Prompt -> ids under the stop contract of "Coming back to Failed Star", "Next:
+// one complete deterministic generation arc". Each forward's last-row logits
+// give the next id: the greedy argmax (sp == nullptr) or the sampler's draw.
+fs_status generate_impl(fs_model* m, fs_kv* kv, int32_t seq, const int32_t* prompt,
+                        int32_t n_prompt, int32_t max_new, const int32_t* eos, int32_t n_eos,
+                        const Sampler* sp, int32_t* out_tokens, int32_t* n_out,
+                        int32_t* stop_reason, cudaStream_t st) {
   if (!m || !kv || !n_out || !stop_reason) return fail(FS_ERR_NULL, "NULL argument");
   if (kv->model != m) return fail(FS_ERR_INVALID, "kv belongs to another model");
   if (n_prompt <= 0) return fail(FS_ERR_EMPTY, "empty prompt");
@@ -577,7 +606,6 @@ extern "C" fs_status fs_greedy(fs_model* m, fs_kv* kv, int32_t seq, const int32_
   if (max_new < 0) return fail(FS_ERR_INVALID, "max_new < 0");
   if (n_eos < 0 || (n_eos > 0 && !eos)) return fail(FS_ERR_INVALID, "bad EOS list");
   if (seq < 0 || seq >= kv->max_seqs) return fail(FS_ERR_SEQ, "sequence out of range");
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int limit = fs::kv_capacity(kv);
   const int n = kv->len[seq] + n_prompt;
   if (n > limit) return fail(FS_ERR_CONTEXT, "prompt exceeds max_pos or the KV capacity");
@@ -594,7 +622,10 @@ extern "C" fs_status fs_greedy(fs_model* m, fs_kv* kv, int32_t seq, const int32_
   fs_status s = fs::ensure_gen_buffer(m, steps);
   if (s != FS_OK) return s;
   int32_t* gen = m->gen_tok;
-  if ((s = fs::prefill_impl(m, kv, seq, prompt, n_prompt, nullptr, gen, st)) != FS_OK) return s;
+  float* lg = sp ? m->lm_scratch : nullptr;
+  if ((s = fs::prefill_impl(m, kv, seq, prompt, n_prompt, lg, sp ? nullptr : gen, st)) != FS_OK)
+    return s;
+  if (sp && (s = sample_into(m, *sp, lg, 0, gen, st)) != FS_OK) return s;
   const int base_len = kv->len[seq];  // == n
   std::vector<int32_t> host(steps);
   int produced = steps;
@@ -605,8 +636,10 @@ extern "C" fs_status fs_greedy(fs_model* m, fs_kv* kv, int32_t seq, const int32_
   while (!stopped) {
     const int upto = std::min(steps, std::max(done, 1) + (done == 1 ? chunk - 1 : chunk));
     for (int i = done; i < upto; ++i) {
-      if ((s = fs::decode_impl(m, kv, &seq, gen + i - 1, 1, nullptr, gen + i, st)) != FS_OK)
+      if ((s = fs::decode_impl(m, kv, &seq, gen + i - 1, 1, lg, sp ? nullptr : gen + i, st)) !=
+          FS_OK)
         return s;
+      if (sp && (s = sample_into(m, *sp, lg, (uint64_t)i, gen + i, st)) != FS_OK) return s;
     }
     done = upto;
     if (n_eos > 0) {
@@ -640,11 +673,54 @@ extern "C" fs_status fs_greedy(fs_model* m, fs_kv* kv, int32_t seq, const int32_
   FS_CUDA(cudaMemcpy(&derr, m->err, sizeof(int), cudaMemcpyDeviceToHost));
   if (derr) {
     cudaMemset(m->err, 0, sizeof(int));
-    fs::mega_reset(m);
+    fs::fused_reset(m);
     return fail(FS_ERR_DEVICE, "a kernel reported device error " + std::to_string(derr));
   }
   *n_out = produced;
   *stop_reason = reason;
+  return FS_OK;
+}
+
+}  // namespace
+
+extern "C" fs_status fs_greedy(fs_model* m, fs_kv* kv, int32_t seq, const int32_t* prompt,
+                               int32_t n_prompt, int32_t max_new, const int32_t* eos,
+                               int32_t n_eos, int32_t* out_tokens, int32_t* n_out,
+                               int32_t* stop_reason, void* stream) {
+  return generate_impl(m, kv, seq, prompt, n_prompt, max_new, eos, n_eos, nullptr, out_tokens,
+                       n_out, stop_reason, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" fs_status fs_generate(fs_model* m, fs_kv* kv, int32_t seq, const int32_t* prompt,
+                                 int32_t n_prompt, int32_t max_new, const int32_t* eos,
+                                 int32_t n_eos, float temperature, int32_t top_k, float top_p,
+                                 uint64_t seed, int32_t* out_tokens, int32_t* n_out,
+                                 int32_t* stop_reason, void* stream) {
+  fs_status s = check_sampler(temperature, top_k, top_p);
+  if (s != FS_OK) return s;
+  Sampler sp{temperature, top_k, top_p, seed};
+  return generate_impl(m, kv, seq, prompt, n_prompt, max_new, eos, n_eos,
+                       temperature > 0.f ? &sp : nullptr, out_tokens, n_out, stop_reason,
+                       static_cast<cudaStream_t>(stream));
+}
+
+extern "C" fs_status fs_sample(fs_model* m, const float* logits, int32_t rows, float temperature,
+                               int32_t top_k, float top_p, uint64_t seed, uint64_t step,
+                               int32_t* out_ids, void* stream) {
+  if (!m) return fail(FS_ERR_NULL, "model is NULL");
+  if (rows <= 0 || rows > fs::kMaxBatch) return fail(FS_ERR_INVALID, "rows must be in [1, 64]");
+  fs_status s = check_sampler(temperature, top_k, top_p);
+  if (s != FS_OK) return s;
+  if ((s = check_device_ptr(logits, "logits")) != FS_OK) return s;
+  if (!out_ids) return fail(FS_ERR_NULL, "out_ids is NULL");
+  if ((s = check_i32_out(out_ids, "out_ids")) != FS_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (temperature == 0.f) {
+    FS_CUDA(fs::launch_argmax_rows(logits, rows, m->s.V, out_ids, st));
+  } else {
+    FS_CUDA(fs::launch_sample(logits, rows, m->s.V, temperature, top_k, top_p, seed, step, out_ids,
+                              st));
+  }
   return FS_OK;
 }
 
@@ -687,8 +763,8 @@ extern "C" fs_status fs_debug_block(fs_model* m, fs_kv* kv, int32_t seq, int32_t
     map.n_list = 1;
     map.seq[0] = seq;
     map.pos[0] = pos0;
-    s = fs::decode_mega(m, kv, map, 1, nullptr, h_in, h_out, layer, layer + 1, false, nullptr,
-                        nullptr, st);
+    s = fs::decode_fused(m, kv, map, 1, nullptr, h_in, h_out, layer, layer + 1, false, nullptr,
+                         nullptr, st);
     if (s != FS_ERR_UNSUPPORTED) return s;
   }
   FS_CUDA(cudaMemcpyAsync(m->h, h_in, (size_t)rows * m->s.H * sizeof(float),
@@ -725,6 +801,16 @@ extern "C" fs_status fs_debug_lm_head(fs_model* m, const float* x, int32_t rows,
   FS_CUDA(fs::launch_rmsnorm(x, rows, m->s.H, m->final_norm, m->s.eps, m->xf, st));
   FS_CUDA(fs::launch_lm_head(m->xf, rows, m->s, m->embed, logits, argmax, m->partial, m->n_part,
                              m->err, st));
+  return FS_OK;
+}
+
+extern "C" fs_status fs_debug_wait_limit(fs_model* m, uint64_t wait_ns, int32_t withhold_layer) {
+  if (!m) return fail(FS_ERR_NULL, "model is NULL");
+  if (wait_ns < 1000 || wait_ns > 60000000000ull)
+    return fail(FS_ERR_INVALID, "wait limit must be in [1 us, 60 s]");
+  if (withhold_layer < -1 || withhold_layer >= m->s.L)
+    return fail(FS_ERR_INVALID, "withhold_layer must be -1 or a layer index");
+  fs::fused_debug_wait(m, wait_ns, withhold_layer);
   return FS_OK;
 }
 

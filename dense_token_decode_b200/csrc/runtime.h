@@ -82,13 +82,16 @@ fs_status prefill_chunk(fs_model* m, const fs_kv* kv, const RowMap& map, int row
 fs_status decode_rows(fs_model* m, const fs_kv* kv, const RowMap& map, int rows,
                       const int32_t* tok, float* logits, int32_t* argmax, cudaStream_t st);
 
-// Persistent decode kernel (decode_mega.cu).
-fs_status mega_init(fs_model* m);
-void mega_release(fs_model* m);
-void mega_reset(fs_model* m);
-fs_status decode_mega(fs_model* m, const fs_kv* kv, const RowMap& map, int B, const int32_t* tok,
-                      const float* h_in, float* h_out, int l0, int l1, bool run_head,
-                      float* logits, int32_t* argmax, cudaStream_t stream);
+// Persistent decode kernel (decode_fused.cu): set-up (transposed Wo / Wd,
+// exchange buffers), release, reset after a device error, the debug wait
+// limit, and one step of blocks [l0, l1) (+ the LM head) for 1..4 rows.
+fs_status fused_init(fs_model* m);
+void fused_release(fs_model* m);
+void fused_reset(fs_model* m);
+void fused_debug_wait(fs_model* m, unsigned long long wait_ns, int withhold_layer);
+fs_status decode_fused(fs_model* m, const fs_kv* kv, const RowMap& map, int B, const int32_t* tok,
+                       const float* h_in, float* h_out, int l0, int l1, bool run_head,
+                       float* logits, int32_t* argmax, cudaStream_t stream);
 
 // Tensor-core prefill (prefill_tc.cu): available for this model (prepares
 // the fp16 weights on first use), one block on m->h, release.

@@ -108,6 +108,32 @@ class Model:
                                 _stream(stream)), "fs_greedy")
         return out[: n_out.value].tolist(), why.value
 
+    def generate(self, kv: "KV", seq: int, prompt, max_new: int, temperature: float,
+                 top_k: int = 0, top_p: float = 1.0, seed: int = 0, eos=(), out=None,
+                 stream=None):
+        """fs_generate: like greedy() with seeded sampling. Returns (ids, reason)."""
+        if not isinstance(prompt, torch.Tensor):
+            prompt = torch.tensor(list(prompt), dtype=torch.int32)
+        if out is None:
+            out = torch.empty(max(max_new, 1), dtype=torch.int32)
+        eos_arr = (C.c_int32 * max(len(eos), 1))(*eos)
+        n_out, why = C.c_int32(0), C.c_int32(0)
+        abi.check(abi.fs_generate(self.handle, kv.handle, seq, _ptr(prompt), prompt.numel(),
+                                  max_new, eos_arr, len(eos), temperature, top_k, top_p, seed,
+                                  _ptr(out), C.byref(n_out), C.byref(why), _stream(stream)),
+                  "fs_generate")
+        return out[: n_out.value].tolist(), why.value
+
+    def sample(self, logits: torch.Tensor, temperature: float, top_k: int = 0,
+               top_p: float = 1.0, seed: int = 0, step: int = 0, out=None, stream=None):
+        """fs_sample on device logits [rows, V]; returns the int32 ids tensor."""
+        rows = 1 if logits.dim() == 1 else logits.shape[0]
+        if out is None:
+            out = torch.empty(rows, dtype=torch.int32, device=logits.device)
+        abi.check(abi.fs_sample(self.handle, logits.data_ptr(), rows, temperature, top_k, top_p,
+                                seed, step, out.data_ptr(), _stream(stream)), "fs_sample")
+        return out
+
     def capture(self, hidden: torch.Tensor | None, max_rows: int = 0):
         abi.check(abi.fs_debug_capture(self.handle, _ptr(hidden), max_rows), "fs_debug_capture")
 
@@ -127,6 +153,10 @@ class Model:
         code = C.c_int32(0)
         abi.check(abi.fs_device_error(self.handle, C.byref(code)), "fs_device_error")
         return code.value
+
+    def wait_limit(self, wait_ns: int, withhold_layer: int = -1):
+        abi.check(abi.fs_debug_wait_limit(self.handle, wait_ns, withhold_layer),
+                  "fs_debug_wait_limit")
 
     def set_prefill_split(self, split: int):
         abi.check(abi.fs_set_prefill_split(self.handle, split), "fs_set_prefill_split")

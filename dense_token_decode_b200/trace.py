@@ -19,10 +19,10 @@ import torch
 from . import abi, synth
 from .engine import Model
 
-SLOTS = [(0, "QKV phase begins"), (1, "QKV input ready"), (12, "QKV done / attention begins"),
-         (2, "attention input ready"), (9, "attention done"), (3, "O phase begins"),
-         (4, "O input ready"), (10, "O done"), (5, "gate/up input ready"), (11, "gate/up done"),
-         (6, "down input ready"), (7, "layer done")]
+SLOTS = [(0, "QKV phase begins"), (1, "QKV input complete"), (2, "QKV rows done"),
+         (3, "attention phase begins"), (4, "q/k/v ready"), (5, "attention done"),
+         (6, "O share added"), (7, "MLP phase begins"), (8, "MLP input complete"),
+         (9, "gate/up done"), (10, "down share added")]
 
 
 def main():
@@ -43,7 +43,7 @@ def main():
     torch.cuda.synchronize()
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     L = shape.n_layers
-    buf = torch.zeros((sms * (L + 1) + L + 2, 16), dtype=torch.int64, device=dev)
+    buf = torch.zeros((sms * (L + 1), 16), dtype=torch.int64, device=dev)
     abi.check(abi.fs_debug_trace(m.handle, buf.data_ptr()), "fs_debug_trace")
     m.decode_step(kv, [0], gen[n:n + 1], None, gen[n + 1:n + 2])
     torch.cuda.synchronize()
@@ -63,9 +63,11 @@ def main():
         if rows:
             a = np.median(np.array(rows), axis=0)
             print(f"{name:34s} {a[0]:7.2f} {a[1]:7.2f} {a[2]:7.2f}")
-    ends = np.nanmedian(t[:, :L, 7], axis=0)
-    print(f"layer time (median) {np.median(np.diff(ends)):.2f} us; LM head "
-          f"{np.nanmedian(t[:, L, 7]) - ends[-1]:.2f} us")
+    ends = np.nanmax(t[:, :L, 10], axis=0)
+    total = np.nanmax(t[:, L, 4]) - np.nanmin(t[:, 0, 0])
+    print(f"layer time (median) {np.median(np.diff(ends)):.2f} us; tail (final norm, LM head, "
+          f"greedy) {np.nanmax(t[:, L, 4]) - ends[-1]:.2f} us; whole step in the kernel "
+          f"{total:.1f} us")
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()

@@ -207,6 +207,38 @@ fs_status fs_greedy(fs_model* model, fs_kv* kv, int32_t seq, const int32_t* prom
                     int32_t n_prompt, int32_t max_new, const int32_t* eos_ids, int32_t n_eos,
                     int32_t* out_tokens, int32_t* n_out, int32_t* stop_reason, void* stream);
 
+/* Seeded sampling of one id per row ("Coming back to Failed Star", "Next:
+ * one complete deterministic generation arc": after greedy, temperature, then
+ * top-k, then top-p, as explicit filters; "Failed Star / fs — Milestones",
+ * M3). For each of `rows` rows of `logits` (device fp32 [rows, vocab]):
+ * divide by `temperature`; rank ids by logit descending, ties to the lowest
+ * id; keep the first `top_k` (0 or >= the finite count keeps all); over those,
+ * keep the shortest prefix of the ranking whose softmax mass reaches `top_p`
+ * (1 keeps all); renormalise; draw u in [0, 1) and return the first kept id
+ * in ascending id order whose cumulative probability exceeds u. u is the top
+ * 24 bits of the first word of Philox4x32-10 (Salmon et al., SC'11) with key
+ * = `seed` (low word first) and counter = (step low word, row, step high
+ * word, 0), times 2^-24. Non-finite logits are never drawn; a row with none
+ * finite gives id 0. `temperature` == 0 is greedy selection (argmax, lowest
+ * id on ties; top_k / top_p ignored). Probabilities are summed as exact
+ * fixed-point integers (units of 2^-32 of the largest), so the result does
+ * not depend on the order of summation. out_ids: device int32 [rows].
+ * Requirements: 1 <= rows <= 64, temperature finite and >= 0, top_k >= 0,
+ * 0 < top_p <= 1. Errors: FS_ERR_NULL, FS_ERR_INVALID, FS_ERR_ALIGN,
+ * FS_ERR_CUDA. */
+fs_status fs_sample(fs_model* model, const float* logits, int32_t rows, float temperature,
+                    int32_t top_k, float top_p, uint64_t seed, uint64_t step, int32_t* out_ids,
+                    void* stream);
+
+/* fs_greedy with the next id drawn by fs_sample from each forward's last-row
+ * logits instead of the argmax: generated id i (0-based) uses counter step i,
+ * row 0. `temperature` == 0 is exactly fs_greedy. Same stop rules, outputs
+ * and errors as fs_greedy, plus the argument checks of fs_sample. */
+fs_status fs_generate(fs_model* model, fs_kv* kv, int32_t seq, const int32_t* prompt,
+                      int32_t n_prompt, int32_t max_new, const int32_t* eos_ids, int32_t n_eos,
+                      float temperature, int32_t top_k, float top_p, uint64_t seed,
+                      int32_t* out_tokens, int32_t* n_out, int32_t* stop_reason, void* stream);
+
 /* Debug: the next fs_prefill or fs_decode_step also writes the residual
  * stream before block 0 and after every block into `hidden` (device fp32
  * [(L+1), max_rows, H]): slot l, row r holds row r of the call (token r of a
@@ -227,15 +259,27 @@ fs_status fs_debug_block(fs_model* model, fs_kv* kv, int32_t seq, int32_t layer,
 
 /* Debug: the next decode step that runs on the persistent decode kernel
  * records %globaltimer stamps (ns) into `buf` (device uint64
- * [SMs][n_layers+1][16]): per CTA and layer, slot 0 phase start, 1 block
- * input ready, 2 attention input ready, 3 O start, 4 O input ready, 5 MLP
- * input ready, 6 down input ready, 7 layer done, 8 warp 0's QKV rows done, 9
- * attention item done, 10 O rows done by every warp, 11 gate/up rows done by
- * every warp, 12 attention item start; row n_layers holds the LM head (0
- * start, 1 input ready, 2 and 3 first and last weight copy issued, 13 warp
- * 0's rows done, 7 done). Slots a CTA never reaches are
- * left as they were. One-shot; NULL disarms. Timing only: no work changes. */
+ * [SMs][n_layers+1][16]): per CTA and block, slot 0 start of the QKV phase,
+ * 1 its input (the residual) complete, 2 QKV rows done, 3 start of the
+ * attention phase, 4 q/k/v of the first batch row ready, 5 attention done,
+ * 6 O-projection share added, 7 start of the MLP phase, 8 its input
+ * complete, 9 gate/up rows done, 10 down share added; row n_layers holds the
+ * tail (0 start, 1 input complete, 2 LM-head rows done, 3 the producer's last
+ * copy issued, 4 greedy ids folded). Slots a CTA never reaches are left as
+ * they were. One-shot; NULL disarms. Timing only: no work changes. */
 fs_status fs_debug_trace(fs_model* model, uint64_t* buf);
+
+/* Debug: the time limit of every wait inside the persistent decode kernel
+ * (a CTA waiting for another CTA's output or for a weight copy), `wait_ns`
+ * in [1 us, 60 s], default 1 s, for all later steps. When a wait runs out
+ * the kernel stops waiting everywhere, returns, and sets the device error
+ * word to 3 (fs_device_error, which also clears the kernel's exchange state;
+ * fs_greedy reports FS_ERR_DEVICE). `withhold_layer` >= 0 makes the next
+ * step on that kernel never publish block `withhold_layer`'s Q/K/V
+ * projections, so the waits for them run out (a test of that path; the step's
+ * outputs are then undefined); -1 withholds nothing.
+ * Errors: FS_ERR_NULL, FS_ERR_INVALID. */
+fs_status fs_debug_wait_limit(fs_model* model, uint64_t wait_ns, int32_t withhold_layer);
 
 /* Debug: dequantise Q8_0 blocks to fp32, out[n*k] = codes[n*k] * scales[n*(k/32)]
  * (all device, row-major). Bit-exact by construction. k % 32 == 0. */

@@ -233,23 +233,29 @@ class Qwen3Oracle:
 
     ``kv_bf16=False`` keeps K/V unrounded (only for comparing with an fp64
     library implementation that has no bf16 cache).
+
+    ``dtype=np.float32`` evaluates the same steps in fp32 arithmetic (weights
+    widened exactly, K/V still rounded to bf16): an emulation of an ideal
+    fp32 implementation, used only to measure how much of a GPU's deviation
+    any fp32 forward would show. The oracle proper is fp64.
     """
 
-    def __init__(self, cfg, weights: dict, kv_bf16: bool = True):
+    def __init__(self, cfg, weights: dict, kv_bf16: bool = True, dtype=np.float64):
         self.cfg = cfg
         self.kv_bf16 = kv_bf16
+        self.dtype = np.dtype(dtype)
         shapes = expected_shapes(cfg)
-        self.embed = bf16_bits_to_f64(weights["embed"])
+        self.embed = bf16_bits_to_f64(weights["embed"]).astype(self.dtype)
         if self.embed.shape != shapes["embed"]:
             raise ValueError(f"embed shape {self.embed.shape} != {shapes['embed']}")
-        self.final_norm = bf16_bits_to_f64(weights["final_norm"])
+        self.final_norm = bf16_bits_to_f64(weights["final_norm"]).astype(self.dtype)
         self.layers = []
         for lw in weights["layers"]:
             layer = {}
             for name in _LINEARS:
-                layer[name] = _widen_linear(lw[name])
+                layer[name] = _widen_linear(lw[name]).astype(self.dtype)
             for name in _NORMS:
-                layer[name] = bf16_bits_to_f64(lw[name])
+                layer[name] = bf16_bits_to_f64(lw[name]).astype(self.dtype)
             for name, s in shapes["layer"].items():
                 if layer[name].shape != s:
                     raise ValueError(f"{name} shape {layer[name].shape} != {s}")
@@ -259,7 +265,7 @@ class Qwen3Oracle:
 
     def new_cache(self) -> KVCache:
         c = self.cfg
-        z = np.zeros((0, c.n_kv_heads, c.head_dim))
+        z = np.zeros((0, c.n_kv_heads, c.head_dim), dtype=self.dtype)
         return KVCache(k=[z.copy() for _ in range(c.n_layers)],
                        v=[z.copy() for _ in range(c.n_layers)])
 
@@ -281,33 +287,42 @@ class Qwen3Oracle:
         S, p0 = tokens.size, cache.length
         if p0 + S > c.max_pos:
             raise ValueError("context exhausted")
-        d, nq, nkv = c.head_dim, c.n_q_heads, c.n_kv_heads
         pos = np.arange(p0, p0 + S)
-        cos, sin = rope_cos_sin(pos, d, c.rope_theta)
-
         x = self.embed[tokens]
         hidden = [x.copy()]
-        for l, W in enumerate(self.layers):
-            xn = rms_norm(x, W["attn_norm"], c.rms_eps)
-            q = (xn @ W["wq"].T).reshape(S, nq, d)
-            k = (xn @ W["wk"].T).reshape(S, nkv, d)
-            v = (xn @ W["wv"].T).reshape(S, nkv, d)
-            q = apply_rope(rms_norm(q, W["q_norm"], c.rms_eps), cos, sin)
-            k = apply_rope(rms_norm(k, W["k_norm"], c.rms_eps), cos, sin)
-            if self.kv_bf16:
-                k, v = round_to_bf16(k), round_to_bf16(v)
-            cache.k[l] = np.concatenate([cache.k[l], k], axis=0)
-            cache.v[l] = np.concatenate([cache.v[l], v], axis=0)
-            o = causal_gqa_attention(q, cache.k[l], cache.v[l], pos,
-                                     np.arange(p0 + S))
-            x = x + o.reshape(S, nq * d) @ W["wo"].T
-            xn = rms_norm(x, W["ffn_norm"], c.rms_eps)
-            a = silu(xn @ W["wg"].T) * (xn @ W["wu"].T)
-            x = x + a @ W["wd"].T
+        for l in range(len(self.layers)):
+            x = self.block(l, x, pos, cache)
             hidden.append(x.copy())
         rows = x if all_logits else x[-1:]
         logits = rms_norm(rows, self.final_norm, c.rms_eps) @ self.embed.T
         return (logits if all_logits else logits[0]), np.stack(hidden), cache
+
+    def block(self, l: int, x: np.ndarray, pos: np.ndarray, cache: KVCache) -> np.ndarray:
+        """Block ``l`` on rows ``x`` [S, H] at positions ``pos`` (consecutive,
+        starting at cache.length): appends the rows' K/V to layer l of the
+        cache and returns the block output. "Coming back to Failed Star",
+        "Second sitting": RMSNorm in both residual halves; "Milestones", M2."""
+        c, W, dt = self.cfg, self.layers[l], self.dtype
+        S = x.shape[0]
+        d, nq, nkv = c.head_dim, c.n_q_heads, c.n_kv_heads
+        cos, sin = rope_cos_sin(pos, d, c.rope_theta)
+        cos, sin = cos.astype(dt), sin.astype(dt)
+        xn = rms_norm(x, W["attn_norm"], c.rms_eps)
+        q = (xn @ W["wq"].T).reshape(S, nq, d)
+        k = (xn @ W["wk"].T).reshape(S, nkv, d)
+        v = (xn @ W["wv"].T).reshape(S, nkv, d)
+        q = apply_rope(rms_norm(q, W["q_norm"], c.rms_eps), cos, sin)
+        k = apply_rope(rms_norm(k, W["k_norm"], c.rms_eps), cos, sin)
+        if self.kv_bf16:
+            k, v = round_to_bf16(k).astype(dt), round_to_bf16(v).astype(dt)
+        cache.k[l] = np.concatenate([cache.k[l], k], axis=0)
+        cache.v[l] = np.concatenate([cache.v[l], v], axis=0)
+        o = causal_gqa_attention(q, cache.k[l], cache.v[l], pos,
+                                 np.arange(cache.k[l].shape[0])).astype(dt)
+        x = x + o.reshape(S, nq * d) @ W["wo"].T
+        xn = rms_norm(x, W["ffn_norm"], c.rms_eps)
+        a = silu(xn @ W["wg"].T) * (xn @ W["wu"].T)
+        return x + a @ W["wd"].T
 
     def logits_uncached(self, tokens) -> np.ndarray:
         """Last-row logits recomputed from scratch over the whole prefix."""

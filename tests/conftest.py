@@ -17,6 +17,19 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
 
 
+def pytest_terminal_summary(terminalreporter):
+    """The measured errors of the parity checks that ran, against their bounds."""
+    try:
+        from parity_util import REPORT
+    except ImportError:
+        return
+    if not REPORT:
+        return
+    terminalreporter.write_line("parity measurements (value / bound):")
+    for what, val, tol in REPORT:
+        terminalreporter.write_line(f"  {what}: {val:.3e} / {tol:g}")
+
+
 def bf16_to_bits(t: torch.Tensor) -> np.ndarray:
     """bf16 tensor -> uint16 bit patterns (no arithmetic)."""
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)

@@ -20,6 +20,11 @@ GREEDY_STEPS = 32     # greedy ids must agree for this many steps, end to end
 E2E_BLOCK_REL_L2 = 3e-3
 
 
+# (label, measured value, bound) of every per-block and logit check of the
+# session, printed in the terminal summary (tests/conftest.py).
+REPORT = []
+
+
 def rel_l2(a, b) -> float:
     a = np.asarray(a, dtype=np.float64)
     b = np.asarray(b, dtype=np.float64)
@@ -30,12 +35,15 @@ def assert_blocks_close(gpu_hidden, ref_hidden, tol=BLOCK_REL_L2, what=""):
     """gpu_hidden, ref_hidden: [L+1, rows, H]. Returns the per-block errors."""
     errs = [rel_l2(gpu_hidden[l], ref_hidden[l]) for l in range(ref_hidden.shape[0])]
     worst = max(errs)
+    REPORT.append((f"{what} per-block rel-L2", worst, tol))
     assert worst <= tol, f"{what} per-block rel-L2 {worst:.3e} > {tol} (all: {errs})"
     return errs
 
 
 def assert_logits_close(gpu_logits, ref_logits, tol=LOGIT_ABS, what=""):
     d = float(np.max(np.abs(np.asarray(gpu_logits, np.float64) - ref_logits)))
+    if what:
+        REPORT.append((f"{what} max |dlogit|", d, tol))
     assert d <= tol, f"{what} max |dlogit| {d:.3e} > {tol}"
     return d
 
