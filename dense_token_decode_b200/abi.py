@@ -77,6 +77,7 @@ SIGNATURES = {
     "fs_kv_set_length": (_I, [_P, _I, _I]),
     "fs_prefill": (_I, [_P, _P, _I, _P, _I, _P, _P, _P]),
     "fs_decode_step": (_I, [_P, _P, _P, _P, _I, _P, _P, _P]),
+    "fs_forward_batch": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P]),
     "fs_greedy": (_I, [_P, _P, _I, _P, _I, _I, _P, _I, _P, _PI, _PI, _P]),
     "fs_sample": (_I, [_P, _P, _I, C.c_float, _I, C.c_float, C.c_uint64, C.c_uint64, _P, _P]),
     "fs_generate": (_I, [_P, _P, _I, _P, _I, _I, _P, _I, C.c_float, _I, C.c_float, C.c_uint64,
@@ -86,6 +87,8 @@ SIGNATURES = {
     "fs_debug_dequant_q8_0": (_I, [_P, _P, _I, _I, _P, _P]),
     "fs_debug_trace": (_I, [_P, _P]),
     "fs_debug_wait_limit": (_I, [_P, C.c_uint64, _I]),
+    "fs_debug_decode_path": (_I, [_P, _I]),
+    "fs_debug_decode_kernel": (_I, [_P, _I, _PI]),
     "fs_debug_lm_head": (_I, [_P, _P, _I, _P, _P, _P]),
     "fs_device_error": (_I, [_P, _PI]),
     "fs_set_prefill_split": (_I, [_P, _I]),
@@ -152,6 +155,7 @@ fs_kv_export = _wrap("fs_kv_export")
 fs_kv_set_length = _wrap("fs_kv_set_length")
 fs_prefill = _wrap("fs_prefill")
 fs_decode_step = _wrap("fs_decode_step")
+fs_forward_batch = _wrap("fs_forward_batch")
 fs_greedy = _wrap("fs_greedy")
 fs_sample = _wrap("fs_sample")
 fs_generate = _wrap("fs_generate")
@@ -160,6 +164,8 @@ fs_debug_block = _wrap("fs_debug_block")
 fs_debug_dequant_q8_0 = _wrap("fs_debug_dequant_q8_0")
 fs_debug_trace = _wrap("fs_debug_trace")
 fs_debug_wait_limit = _wrap("fs_debug_wait_limit")
+fs_debug_decode_path = _wrap("fs_debug_decode_path")
+fs_debug_decode_kernel = _wrap("fs_debug_decode_kernel")
 fs_debug_lm_head = _wrap("fs_debug_lm_head")
 fs_device_error = _wrap("fs_device_error")
 fs_set_prefill_split = _wrap("fs_set_prefill_split")

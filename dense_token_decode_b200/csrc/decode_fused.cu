@@ -17,20 +17,16 @@
 //      owns columns [a_c, b_c) of Wg, Wu and the matching rows of Wd^T, so its
 //      SwiGLU outputs feed its own share of the down projection, added to the
 //      residual.
-// Three hand-offs per block: A -> B (tagged words), B -> C and C -> next A
-// (the residual sums).
-//
-// Residual sums. Every contribution is added with one 64-bit integer atomic
-// per element, the value in fixed point (2^-32 units), so the sum does not
-// depend on the order of arrival (the step is bit-for-bit reproducible).
-// Contributions are spread over P copies of each accumulator (contributor k
-// adds into copy k % P) to spread the atomics over more L2 lines; readers
-// add the copies. After its atomics a contributing CTA passes a barrier and
-// one thread publishes them with a release fence and an increment of the
-// copy's arrival counter; a reader's first thread acquires the counters, the
-// CTA passes a barrier, and every thread then loads its words once.
-// Accumulators of a step live in one of two sets; each step clears the other
-// set for the step after it.
+// Hand-offs between CTAs are 64-bit words (fp32 value | 32-bit tag) written
+// with plain stores; a reader polls the words it needs until their tag is the
+// current one (tags grow across steps, so nothing is ever cleared and no flag
+// or fence is needed). A -> B passes the Q/K/V rows. The residual sums after
+// B and after C are reduced without atomics: every contributor (attention
+// unit, or CTA of the MLP phase) stores its partial vector in a slot of its
+// own; every CTA then sums a slice of about H / G elements over all slots in
+// a fixed order (adding the residual the block started the half from) and
+// publishes it; every CTA polls the published vector. The sums are therefore
+// reproducible bit for bit.
 //
 // Weight stream. A producer warp (one lane) copies the CTA's weights, the
 // group's K/V pages and, for the LM head, its rows of the embedding into a
@@ -55,14 +51,12 @@ constexpr int kConsumerWarps = 11;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;  // + producer warp
 constexpr int kMaxB = 4;
-constexpr int kData = 16384;   // main area of a stage
+constexpr int kData = 16384;   // main area of a Q8_0 stage
 constexpr int kExtra = 2048;   // Q8_0 scale area after it
-constexpr int kStageBytes = kData + kExtra;
+constexpr int kStageQ8 = kData + kExtra;
+constexpr int kStageBf16 = 8 * (2 * 1024 + 16);  // eight padded bf16 rows of K = 1024
 constexpr int kMaxStages = 16;
 constexpr int kSlice = 8;      // head-dimension slice of one attention unit
-constexpr int kMaxCopies = 4;  // copies of each residual accumulator
-constexpr float kFix = 4294967296.0f;       // 2^32
-constexpr float kUnfix = 2.3283064365386963e-10f;  // 2^-32
 constexpr int kMaxRep = 2;     // query heads per kv head
 constexpr int kTraceSlots = 16;
 
@@ -90,12 +84,10 @@ struct Params {
   int pos[kMaxB];
   const int32_t* tokens;
   unsigned long long* xq;    // [B][(nq+2nkv)d] tagged words
-  unsigned long long* acc;   // this step's accumulators [2L][P][B][H]
-  unsigned long long* cnt;   // their arrival counters [2L][kMaxCopies]
-  unsigned long long* clear; // the other set, cleared by this step
-  long long clear_words;     // words of the other set to clear
-  int P;                     // copies per accumulator
-  int n_units;               // attention units nkv * d/8
+  unsigned long long* part_b;  // [n_units][B][H] partial O projections (tagged)
+  unsigned long long* part_c;  // [G][B][H] partial down projections (tagged)
+  unsigned long long* rsum;    // [2][B][H] reduced residual after attention / after the block
+  int n_units;                 // attention units nkv * d/8
   int c_ctas;                // CTAs with intermediate columns
   uint32_t tag0;
   int l0, l1;
@@ -114,10 +106,12 @@ struct Params {
   int withhold_layer;  // debug: phase-A outputs of this layer are never published
   unsigned long long* trace;
   int n_stages;
-  int off_r, off_z, off_misc, off_attn, off_tab, off_bar;
+  int off_r, off_z, off_misc, off_attn, off_tab, off_bar, off_red;
   int bt_in_smem;
-  int lm_owner;  // LM-head chunks each consumed by one warp (ring of >= 11 stages)
-  int lm_rows;   // rows per LM-head chunk
+  int stage_bytes;
+  int off_zt;     // [2 slots][2B rows: hi, lo of each batch row][H + 8] bf16 GEMV operands
+  int lm_owners;  // warps that consume LM-head chunks (chunk i: warp i % lm_owners)
+  int lm_rows;    // rows per LM-head chunk
 };
 
 // ---------------------------------------------------------------------------
@@ -169,20 +163,6 @@ __device__ __forceinline__ void st_tag(unsigned long long* p, float v, uint32_t 
   const unsigned long long w = ((unsigned long long)tag << 32) | __float_as_uint(v);
   asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
 }
-__device__ __forceinline__ void red_add(unsigned long long* p, unsigned long long v) {
-  asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-// Publishes the CTA's earlier atomics (ordered before this thread by a CTA
-// barrier) and counts one arrival.
-__device__ __forceinline__ void release_count(unsigned long long* c) {
-  asm volatile("fence.acq_rel.gpu;" ::: "memory");
-  asm volatile("red.relaxed.gpu.global.add.u64 [%0], 1;" ::"l"(c) : "memory");
-}
-__device__ __forceinline__ unsigned long long ld_acquire(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
 __device__ __forceinline__ void mbar_arrive_n(uint64_t* bar, uint32_t n) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(su32(bar)), "r"(n) : "memory");
 }
@@ -216,24 +196,54 @@ __device__ __forceinline__ float warp_sum(float v) {
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
-// One contribution to an accumulator word: the value in fixed point.
-__device__ __forceinline__ unsigned long long fix_word(float x) {
-  return (unsigned long long)__float2ll_rn(x * kFix);
+// Warp-level tensor-core operations for the skinny products of decode: A
+// (16 x 16 bf16, rows of weights or their transpose) from shared memory by
+// ldmatrix, B (16 x 8 bf16) the activation as two bf16 terms per batch row,
+// fp32 accumulation.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
 }
-__device__ __forceinline__ long long word_value(unsigned long long w) { return (long long)w; }
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t (&r)[2]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4],
+                                         const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+__device__ __forceinline__ uint32_t word_tag(unsigned long long w) { return (uint32_t)(w >> 32); }
+__device__ __forceinline__ float word_value(unsigned long long w) {
+  return __uint_as_float((uint32_t)w);
+}
 
 __host__ __device__ inline void slice(int N, int G, int c, int& a, int& b) {
   a = (int)((long long)N * c / G);
   b = (int)((long long)N * (c + 1) / G);
 }
 
-// Rows per chunk of each kind (the consumers and the producer agree on them).
-__host__ __device__ inline int rows_cap(int H, bool q8) {  // rows of K = H
-  const int r = q8 ? kData / H : kData / (2 * H);
+// Layout of weight rows in a stage (the consumers and the producer agree on
+// it). bf16 rows (K = H) sit 2H + 16 bytes apart, so the rows an ldmatrix
+// reads together fall in different shared-memory banks; Q8_0 code rows are
+// packed (H bytes apart) with their scales at kData.
+__host__ __device__ inline int row_stride(int H, bool q8) { return q8 ? H : 2 * H + 16; }
+__host__ __device__ inline int rows_cap(int H, bool q8) {  // rows of K = H per chunk
+  const int r = q8 ? kData / H : kStageBf16 / (2 * H + 16);
   return r < 16 ? r : 16;
 }
 __host__ __device__ inline int pairs_cap(int H, bool q8) {
-  const int r = q8 ? kData / (2 * H) : kData / (4 * H);
+  const int r = q8 ? kData / (2 * H) : rows_cap(H, false) / 2;
   return r < 8 ? r : 8;
 }
 // End of the QKV chunk from row n (never across the wq|wk|wv boundaries).
@@ -284,11 +294,10 @@ __device__ __forceinline__ size_t kv_off(const Params& p, int layer, int b, int 
          (((size_t)page * p.kv.n_kv_heads + g) * kPage + (pos % kPage)) * p.kv.head_dim;
 }
 
-// Accumulator words of version v (2l: after the attention half of block l,
-// 2l+1: after block l), copy q, row b. A launch uses the first 2L*P*B*H words
-// of its set.
-__device__ __forceinline__ unsigned long long* acc_row(const Params& p, int v, int q, int b) {
-  return p.acc + (((size_t)v * p.P + q) * p.B + b) * p.H;
+// Tag of hand-off k of block l: 0 Q/K/V rows, 1 O-projection partials, 2 the
+// residual after attention, 3 down-projection partials, 4 the block output.
+__host__ __device__ __forceinline__ uint32_t tag_of(uint32_t tag0, int l, int l0, int k) {
+  return tag0 + 5u * (uint32_t)(l - l0) + (uint32_t)k;
 }
 
 // ---------------------------------------------------------------------------
@@ -324,7 +333,7 @@ struct Producer {
       }
     }
     mbar_expect_tx(&r.full[s], bytes);
-    return r.stages + (size_t)s * kStageBytes;
+    return r.stages + (size_t)s * p.stage_bytes;
   }
   __device__ __forceinline__ uint64_t* bar() { return &r.full[stage]; }
   __device__ __forceinline__ void advance() {
@@ -335,6 +344,20 @@ struct Producer {
     }
   }
 
+  // Rows [n, e) of a [N][K = H] matrix into `st` from row slot `slot` on:
+  // bf16 rows one copy each at the padded stride, Q8_0 codes packed.
+  __device__ void copy_rows(unsigned char* st, int slot, const void* w, int n, int nr, bool q8) {
+    const int H = p.H;
+    const uint32_t rb = q8 ? H : 2 * H;
+    const unsigned char* src = static_cast<const unsigned char*>(w) + (size_t)n * rb;
+    if (q8) {
+      bulk_load(st + slot * rb, src, nr * rb, bar(), policy);
+    } else {
+      const int rs = row_stride(H, false);
+      for (int i = 0; i < nr; ++i)
+        bulk_load(st + (slot + i) * rs, src + (size_t)i * rb, rb, bar(), policy);
+    }
+  }
   // Rows [n, e) of a [N][K = H] matrix (bf16, or Q8_0 codes + scales).
   __device__ void rows(const void* w, const __half* s, int n, int e, bool q8) {
     const int H = p.H, nr = e - n;
@@ -342,7 +365,7 @@ struct Producer {
     const uint32_t sb = q8 ? H / 16 : 0;
     unsigned char* st = acquire(nr * (rb + sb));
     if (!st) return;
-    bulk_load(st, static_cast<const unsigned char*>(w) + (size_t)n * rb, nr * rb, bar(), policy);
+    copy_rows(st, 0, w, n, nr, q8);
     if (q8)
       bulk_load(st + kData, reinterpret_cast<const unsigned char*>(s) + (size_t)n * sb, nr * sb,
                 bar(), policy);
@@ -393,8 +416,7 @@ struct Producer {
         } else {
           unsigned char* st = acquire(kSlice * 2 * H);
           if (!st) return;
-          bulk_load(st, static_cast<const __nv_bfloat16*>(T.wo_t) + (size_t)c0 * H,
-                    kSlice * 2 * H, bar(), policy);
+          copy_rows(st, 0, T.wo_t, c0, kSlice, false);
         }
         advance();
       }
@@ -412,10 +434,8 @@ struct Producer {
       const int e = min(b, n + pc), nr = e - n;
       unsigned char* st = acquire(2 * nr * (rb + sb));
       if (!st) return;
-      bulk_load(st, static_cast<const unsigned char*>(Lw.w[kWg]) + (size_t)n * rb, nr * rb, bar(),
-                policy);
-      bulk_load(st + pc * rb, static_cast<const unsigned char*>(Lw.w[kWu]) + (size_t)n * rb,
-                nr * rb, bar(), policy);
+      copy_rows(st, 0, Lw.w[kWg], n, nr, q8);
+      copy_rows(st, pc, Lw.w[kWu], n, nr, q8);
       if (q8) {
         bulk_load(st + kData, reinterpret_cast<const unsigned char*>(Lw.s[kWg]) + (size_t)n * sb,
                   nr * sb, bar(), policy);
@@ -431,8 +451,7 @@ struct Producer {
       const int e = down_chunk_end(n, b, rc, q8), nr = e - n;
       unsigned char* st = acquire(nr * rb + (q8 ? 2 * H : 0));
       if (!st) return;
-      bulk_load(st, static_cast<const unsigned char*>(T.wd_t) + (size_t)n * rb, nr * rb, bar(),
-                policy);
+      copy_rows(st, 0, T.wd_t, n, nr, q8);
       if (q8) bulk_load(st + kData, T.sd_t + (size_t)(n / 32) * H, 2 * H, bar(), policy);
       advance();
       n = e;
@@ -453,7 +472,7 @@ struct Producer {
 // ---------------------------------------------------------------------------
 // Consumers
 
-template <int NB, bool Q8W, int IT>
+template <int NB, bool Q8W, int IT, int DQ>
 struct Consumer {
   const Params& p;
   Ring r;
@@ -488,11 +507,34 @@ struct Consumer {
   float* ss_s = nullptr;                                 // [11][kMaxB] of the current slot
   __device__ float* act_s() { return misc + 128; }       // [kMaxB][128]
   __device__ float* o_s() { return misc + 128 + 512; }   // [kMaxB][kMaxRep][kSlice]
-
-  __device__ void tr(int layer, int k) {
-    if (p.trace && tid == 0) p.trace[((size_t)cta * (p.L + 1) + layer) * kTraceSlots + k] = now_ns();
+  // Shared-memory layout of the rest of `misc` (bytes): ys [48][4] fp32 at
+  // 2816, the greedy keys / flag / counts at 4096, 64 zero bytes at 4160, the
+  // tensor-core coefficient rows [8][40] bf16 at 4224, the row table [48] at 4864.
+  __device__ float* ys() { return misc + 704; }
+  __device__ uint32_t zero_addr() const { return su32(reinterpret_cast<const unsigned char*>(misc) + 4160); }
+  __device__ __nv_bfloat16* coef() {
+    return reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<unsigned char*>(misc) + 4224);
   }
-  __device__ void give_up() {
+  __device__ uint32_t* rowaddr() {
+    return reinterpret_cast<uint32_t*>(reinterpret_cast<unsigned char*>(misc) + 4864);
+  }
+  __nv_bfloat16* zt = nullptr;  // the current slot of the tensor-core operand rows
+  static constexpr int kCoefStride = 40;  // bf16 per coefficient row (80 bytes)
+  __device__ int zt_stride() const { return p.H + 8; }  // bf16 per operand row
+  // Shared address of the chunk `ahead` places after the oldest unreleased one.
+  __device__ uint32_t stage_addr(int ahead) const {
+    int s = stage + ahead;
+    if (s >= r.n) s -= r.n;
+    return su32(r.stages + (size_t)s * p.stage_bytes);
+  }
+
+  // Trace stamp k of (this CTA, layer): the SM's cycle counter (converted on
+  // the host with the CTA's own globaltimer / clock pairs at start and end).
+  __device__ __noinline__ void tr(int layer, int k) {
+    if (p.trace && tid == 0)
+      p.trace[((size_t)cta * (p.L + 1) + layer) * kTraceSlots + k] = clock64();
+  }
+  __device__ __noinline__ void give_up() {
     if (!aborted(p.abort_flag)) {
       atomicExch(p.abort_flag, 1);
       atomicCAS(p.err, 0, kErrTimeout);
@@ -504,13 +546,17 @@ struct Consumer {
   // warp has not released; returns its stage. Every chunk before it has been
   // waited for by this warp, so the stage's full barrier is in this chunk's
   // phase or the one before it.
-  __device__ const unsigned char* chunk_wait(int ahead = 0) {
+  __device__ __forceinline__ const unsigned char* chunk_wait(int ahead = 0) {
     int s = stage + ahead;
     uint32_t par = parity;
     if (s >= r.n) {
       s -= r.n;
       par ^= 1u;
     }
+    if (__all_sync(0xffffffffu, mbar_test(&r.full[s], par))) return r.stages + (size_t)s * p.stage_bytes;
+    return chunk_wait_slow(s, par);
+  }
+  __device__ __noinline__ const unsigned char* chunk_wait_slow(int s, uint32_t par) {
     unsigned long long t0 = 0;
     int spins = 0;
     while (true) {
@@ -525,7 +571,7 @@ struct Consumer {
         if (__shfl_sync(0xffffffffu, bad, 0)) give_up();
       }
     }
-    return r.stages + (size_t)s * kStageBytes;
+    return r.stages + (size_t)s * p.stage_bytes;
   }
   __device__ void cursor_advance() {
     ++i;
@@ -536,16 +582,18 @@ struct Consumer {
   }
   __device__ void chunk_release() {
     __syncwarp();
-    if (lane == 0) mbar_arrive(&r.empty[stage]);
+    // A thread that gave up has skipped its waits: it must not release a
+    // chunk it never saw (an arrival beyond a phase's count is undefined).
+    if (lane == 0 && !quit) mbar_arrive(&r.empty[stage]);
     cursor_advance();
   }
   // Wait (whole warp) for the next chunk when this warp alone consumes it and
-  // skips the chunks of other warps (ring of at least kConsumerWarps stages):
+  // skips the chunks of other warps (W owner warps, ring of n >= W stages):
   // first the release of the chunk n places earlier in the same stage, then
-  // the chunk itself. With n >= kConsumerWarps the release test cannot see an
-  // older phase: this warp waited on a chunk at most kConsumerWarps places
-  // back, so every chunk 2n places back has been released.
-  __device__ const unsigned char* chunk_wait_owned() {
+  // the chunk itself. With n >= W the release test cannot see an older phase:
+  // this warp waited on a chunk W places back, so every chunk 2n places back
+  // has been released.
+  __device__ __noinline__ const unsigned char* chunk_wait_owned() {
     const int s = stage;
     unsigned long long t0 = 0;
     int spins = 0;
@@ -562,13 +610,20 @@ struct Consumer {
         if (__shfl_sync(0xffffffffu, bad, 0)) give_up();
       }
     }
-    return r.stages + (size_t)s * kStageBytes;
+    return r.stages + (size_t)s * p.stage_bytes;
   }
 
   // ---- residual input of a phase -----------------------------------------
 
   static constexpr int kEPT = (NB * IT * 256 + kConsumers - 1) / kConsumers;  // elements / thread
   float inv[NB];
+  __device__ __forceinline__ float inv_of(int b) const {
+    float v = inv[0];
+#pragma unroll
+    for (int bb = 1; bb < NB; ++bb)
+      if (bb == b) v = inv[bb];
+    return v;
+  }
 
   // Gains of this thread's elements (k = tid + 352 e of the [B][H] rows),
   // fetched before the wait for the residual so their latency overlaps it.
@@ -580,59 +635,111 @@ struct Consumer {
     }
   }
 
-  // Thread 0 waits until every copy of accumulator version v has all of its
-  // `contrib` contributors (contributor c counts in copy c % P); the caller's
-  // barrier then orders every thread's loads after it.
-  __device__ void wait_counts(int v, int contrib) {
-    if (tid != 0 || quit) return;
-    const int P = p.P;
+  // Polls one tagged word until its tag is `want` (bounded wait); x is the
+  // value already loaded.
+  __device__ __forceinline__ unsigned long long poll_word(const unsigned long long* w,
+                                                          unsigned long long x, uint32_t want) {
+    if (word_tag(x) == want || quit) return x;
+    return poll_word_slow(w, want);
+  }
+  __device__ __noinline__ unsigned long long poll_word_slow(const unsigned long long* w,
+                                                            uint32_t want) {
+    unsigned long long x = 0;
     unsigned long long t0 = 0;
     int spins = 0;
-    for (int q = 0; q < P; ++q) {
-      const unsigned long long want = (unsigned long long)((contrib - q + P - 1) / P);
-      const unsigned long long* c = p.cnt + (size_t)v * kMaxCopies + q;
-      while (ld_acquire(c) < want) {
-        __nanosleep(32);
-        if ((++spins & 63) == 0) {
+    do {
+      __nanosleep(20);
+      x = ld_word(w);
+      if ((++spins & 7) == 0) {
+        // another CTA's abort ends the wait within a few polls; the time
+        // limit is read less often
+        bool stop = aborted(p.abort_flag);
+        if (!stop && (spins & 63) == 0) {
           if (t0 == 0) t0 = now_ns();
-          if (aborted(p.abort_flag) || now_ns() - t0 > p.wait_ns) {
-            give_up();
-            return;
-          }
+          stop = now_ns() - t0 > p.wait_ns;
+        }
+        if (stop) {
+          give_up();
+          break;
         }
       }
-    }
+    } while (word_tag(x) != want);
+    return x;
   }
 
-  // The phase input rows into rs (source: v >= 0 an accumulator version, -1
-  // the embedding rows of the tokens or h_in), zs = gain * rs, and 1/rms of
-  // each row into inv. Ends on a barrier.
+  // This CTA's slice of a residual sum: elements [e0, e1) of the flattened
+  // [B][H] rows, each = base[e] (rs: the residual the half started from) plus
+  // the partials of contributors 0..n_contrib-1 (slot c at src + c*B*H,
+  // tagged tag_in), summed in a fixed order; published to dst with tag_out.
+  // Ends on a barrier.
+  __device__ __noinline__ void reduce_slice(const unsigned long long* src, int n_contrib, uint32_t tag_in,
+                               unsigned long long* dst, uint32_t tag_out) {
+    const int n = p.B * p.H;
+    int e0, e1;
+    slice(n, G, cta, e0, e1);
+    const int E = e1 - e0, total = n_contrib * E;
+    float* buf = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(rs) - p.off_r + p.off_red);
+    for (int f0 = tid; f0 < total; f0 += 4 * kConsumers) {
+      unsigned long long w[4];
+      const unsigned long long* ptr[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int f = f0 + u * kConsumers;
+        ptr[u] = f < total ? src + (size_t)(f / E) * n + e0 + f % E : src;
+        w[u] = f < total ? ld_word(ptr[u]) : 0ull;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int f = f0 + u * kConsumers;
+        if (f < total) buf[f] = word_value(poll_word(ptr[u], w[u], tag_in));
+      }
+    }
+    consumer_sync();
+    // four threads per element: contributors c = q, q+4, ... in order, then
+    // the base value and the four partial sums in a fixed order
+    float* part4 = buf + (size_t)n_contrib * E;
+    if (tid < 4 * E) {
+      const int e = tid >> 2, q = tid & 3;
+      float sacc = 0.f;
+      for (int c = q; c < n_contrib; c += 4) sacc += buf[c * E + e];
+      part4[tid] = sacc;
+    }
+    consumer_sync();
+    if (tid < E && !quit) {
+      const float* q4 = part4 + 4 * tid;
+      st_tag(dst + e0 + tid, rs[e0 + tid] + ((q4[0] + q4[1]) + (q4[2] + q4[3])), tag_out);
+    }
+    consumer_sync();  // rs is read above before any thread overwrites it
+  }
+
+  // The phase input rows into rs (source: kind >= 0 the published residual
+  // rsum[kind] with tag `tag`; -1 the embedding rows of the tokens or h_in),
+  // zs = gain * rs, and 1/rms of each row into inv. Ends on a barrier.
   // `slot` (0: phase A and the LM head, 1: phase C) picks the buffers of zs and
   // of the partial sums, so a warp that runs ahead into the next phase never
   // writes what a slower warp still reads.
-  __device__ void gather_norm(int v, int contrib, const float (&gr)[kEPT], int slot) {
+  __device__ __noinline__ void gather_norm(int kind, uint32_t tag, const float (&gr)[kEPT], int slot) {
     const int H = p.H, n = p.B * H;
-    zs = zs_base + (size_t)slot * p.B * H;
+    zs = zs_base + (size_t)slot * n;
+    zt = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<unsigned char*>(misc) - p.off_misc +
+                                          p.off_zt) +
+         (size_t)slot * 2 * p.B * zt_stride();
     ss_s = misc + slot * 64;
     float ss[NB];
 #pragma unroll
     for (int b = 0; b < NB; ++b) ss[b] = 0.f;
-    long long sum[kEPT];
-    if (v >= 0) {
-      wait_counts(v, contrib);
-      if (__syncthreads_or_consumers(quit)) quit = true;
-      // every word of every copy of this thread's elements, loads issued together
+    unsigned long long w[kEPT];
+    const unsigned long long* src = kind >= 0 ? p.rsum + (size_t)kind * n : nullptr;
+    if (kind >= 0) {
 #pragma unroll
-      for (int e = 0; e < kEPT; ++e) sum[e] = 0;
-      for (int q = 0; q < p.P; ++q) {
-        unsigned long long w[kEPT];
+      for (int e = 0; e < kEPT; ++e) {
+        const int k = tid + e * kConsumers;
+        w[e] = k < n ? ld_word(src + k) : 0ull;
+      }
 #pragma unroll
-        for (int e = 0; e < kEPT; ++e) {
-          const int k = tid + e * kConsumers;
-          w[e] = k < n ? ld_word(acc_row(p, v, q, k / H) + k % H) : 0ull;
-        }
-#pragma unroll
-        for (int e = 0; e < kEPT; ++e) sum[e] += word_value(w[e]);
+      for (int e = 0; e < kEPT; ++e) {
+        const int k = tid + e * kConsumers;
+        if (k < n) w[e] = poll_word(src + k, w[e], tag);
       }
     }
 #pragma unroll
@@ -641,8 +748,8 @@ struct Consumer {
       if (k >= n) break;
       const int b = k / H;
       float x;
-      if (v >= 0) {
-        x = __ll2float_rn(sum[e]) * kUnfix;
+      if (kind >= 0) {
+        x = word_value(w[e]);
       } else if (p.h_in) {
         x = p.h_in[k];
       } else {
@@ -654,7 +761,13 @@ struct Consumer {
         x = __bfloat162float(p.embed[(size_t)t * H + k % H]);
       }
       rs[k] = x;
-      zs[k] = x * gr[e];
+      const float z = x * gr[e];
+      if (Q8W) zs[k] = z;
+      // the tensor-core operand: z as hi + lo bf16 terms (rows 2b, 2b + 1)
+      const __nv_bfloat16 hi = __float2bfloat16_rn(z);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(z - __bfloat162float(hi));
+      zt[(size_t)(2 * b) * zt_stride() + k % H] = hi;
+      zt[(size_t)(2 * b + 1) * zt_stride() + k % H] = lo;
 #pragma unroll
       for (int bb = 0; bb < NB; ++bb)
         if (bb == b) ss[bb] += x * x;
@@ -669,7 +782,7 @@ struct Consumer {
     for (int b = 0; b < NB; ++b) {
       float t = 0.f;
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) t += ss_s[w * kMaxB + b];
+      for (int w2 = 0; w2 < kConsumerWarps; ++w2) t += ss_s[w2 * kMaxB + b];
       inv[b] = rsqrtf(t / (float)H + p.eps);
     }
   }
@@ -715,9 +828,132 @@ struct Consumer {
     for (int b = 0; b < NB; ++b) acc[b] = warp_sum(acc[b]);
   }
 
+  // ---- tensor-core products ----------------------------------------------
+
+  // ys[r * 4 + b] = sum_k W[r][k] z_b[k] for the R rows whose bf16 data start
+  // at the shared addresses rowaddr()[0..R) (K = H): A = the rows (16-row
+  // tiles), B = the 2B operand rows of zt (hi and lo term of each batch row),
+  // so column 2b + t of the product is term t of batch row b. Work items are
+  // (row tile, block of 8 k-steps), warp w taking items w, w + 11, ...; the
+  // items' partial sums meet in shared memory and are added in a fixed order.
+  // Ends on a barrier.
+  __device__ __noinline__ void mma_rows(int R) {
+    const uint32_t* ra = rowaddr();
+    float* part = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(rs) - p.off_r + p.off_red);
+    const int nkb = p.H / 128, mt = (R + 15) / 16, items = mt * nkb, twoB = 2 * p.B;
+    const uint32_t z0 = su32(zt), zrow = (uint32_t)zt_stride() * 2, zero = zero_addr();
+    for (int it = warp; it < items; it += kConsumerWarps) {
+      const int m = it / nkb, kb0 = (it % nkb) * 8;
+      const int row = m * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+      const bool arow = row < R;
+      uint32_t aaddr = arow ? ra[row] + ((lane >> 4) << 4) + kb0 * 32 : zero;
+      const int n = lane & 7;
+      const bool brow = n < twoB;
+      uint32_t baddr = brow ? z0 + n * zrow + (((lane >> 3) & 1) << 4) + kb0 * 32 : zero;
+      const uint32_t astep = arow ? 32u : 0u, bstep = brow ? 32u : 0u;
+      float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < 8; ks += 2) {
+        uint32_t a[4], b[2], a2[4], b2[2];
+        ldsm_x4(aaddr, a);
+        ldsm_x2(baddr, b);
+        ldsm_x4(aaddr + astep, a2);
+        ldsm_x2(baddr + bstep, b2);
+        mma16816(d0, a, b);
+        mma16816(d1, a2, b2);
+        aaddr += 2 * astep;
+        baddr += 2 * bstep;
+      }
+      const int g = lane >> 2, q = lane & 3;
+      part[(it * 16 + g) * 4 + q] = (d0[0] + d1[0]) + (d0[1] + d1[1]);
+      part[(it * 16 + g + 8) * 4 + q] = (d0[2] + d1[2]) + (d0[3] + d1[3]);
+    }
+    consumer_sync();
+    float* y = ys();
+    for (int t = tid; t < R * 4; t += kConsumers) {
+      const int rr = (t >> 2) & 15, q = t & 3, m = t >> 6;
+      float sum = 0.f;
+      for (int kb = 0; kb < nkb; ++kb) sum += part[((m * nkb + kb) * 16 + rr) * 4 + q];
+      y[t] = sum;
+    }
+    consumer_sync();
+  }
+
+  // The coefficient rows of mma_cols from fp32 values v(b, r), r < KR (zero
+  // from KR to 32): row 2b holds the bf16 hi term, row 2b + 1 the lo term.
+  template <class V>
+  __device__ __forceinline__ void fill_coef(int KR, V&& v) {
+    __nv_bfloat16* c = coef();
+    for (int t = tid; t < 8 * 32; t += kConsumers) {
+      const int row = t >> 5, r = t & 31, b = row >> 1;
+      float x = 0.f;
+      if (b < p.B && r < KR) x = v(b, r);
+      const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+      c[row * kCoefStride + r] = (row & 1) ? __float2bfloat16_rn(x - __bfloat162float(hi)) : hi;
+    }
+  }
+
+  // For every column c < H of a transposed matrix held as KR rows (row r's
+  // bf16 data at rowaddr()[r], KR <= 32) and the coefficients of coef():
+  // out(c, b) = sum_r W[r][c] coef_b[r], on the tensor cores with A = W^T
+  // (ldmatrix .trans), one 16-column tile per item, warp w taking tiles
+  // w, w + 11, ...; emit(c, b, value) for each column and batch row.
+  template <class F>
+  __device__ __forceinline__ void mma_cols(int KR, F&& emit) {
+    const uint32_t* ra = rowaddr();
+    const int ksn = (KR + 15) / 16, tiles = p.H / 16, twoB = 2 * p.B;
+    const uint32_t c0 = su32(coef()), zero = zero_addr();
+    const int g = lane >> 2, q = lane & 3, n = lane & 7;
+    for (int t = warp; t < tiles; t += kConsumerWarps) {
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int ks = 0; ks < ksn; ++ks) {
+        const int r = ks * 16 + (lane & 7) + (lane >> 4) * 8;
+        const int col = t * 16 + ((lane >> 3) & 1) * 8;
+        const uint32_t aaddr = r < KR ? ra[r] + col * 2 : zero;
+        const uint32_t baddr =
+            n < twoB ? c0 + n * (kCoefStride * 2) + ks * 32 + (((lane >> 3) & 1) << 4) : zero;
+        uint32_t a[4], b[2];
+        ldsm_x4_t(aaddr, a);
+        ldsm_x2(baddr, b);
+        mma16816(d, a, b);
+      }
+      if (q < p.B) {
+        emit(t * 16 + g, q, d[0] + d[1]);
+        emit(t * 16 + g + 8, q, d[2] + d[3]);
+      }
+    }
+  }
+
+  // One LM-head chunk (nr <= 8 rows of the embedding at the padded stride) on
+  // this warp: logits of every batch row, folded into the greedy keys.
+  __device__ __noinline__ void lm_rows_mma(const unsigned char* st, int n0, int nr) {
+    const uint32_t rs2 = (uint32_t)row_stride(p.H, false), zero = zero_addr();
+    const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
+    const bool arow = row < nr;
+    uint32_t aaddr = arow ? su32(st) + row * rs2 + ((lane >> 4) << 4) : zero;
+    const int n = lane & 7;
+    const bool brow = n < 2 * p.B;
+    uint32_t baddr = brow ? su32(zt) + n * zt_stride() * 2 + (((lane >> 3) & 1) << 4) : zero;
+    const uint32_t astep = arow ? 32u : 0u, bstep = brow ? 32u : 0u;
+    float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int ks = 0; ks < p.H / 16; ks += 2) {
+      uint32_t a[4], b[2], a2[4], b2[2];
+      ldsm_x4(aaddr, a);
+      ldsm_x2(baddr, b);
+      ldsm_x4(aaddr + astep, a2);
+      ldsm_x2(baddr + bstep, b2);
+      mma16816(d0, a, b);
+      mma16816(d1, a2, b2);
+      aaddr += 2 * astep;
+      baddr += 2 * bstep;
+    }
+    const int g = lane >> 2, q = lane & 3;
+    if (g < nr && q < p.B) fold_logit(q, n0 + g, ((d0[0] + d1[0]) + (d0[1] + d1[1])) * inv_of(q));
+  }
+
   // ---- phase A: RMSNorm + QKV rows --------------------------------------
 
-  __device__ void capture_rows(int slot) {
+  __device__ __noinline__ void capture_rows(int slot) {
     if (!p.capture || cta != 0) return;
     for (int k = tid; k < p.B * p.H; k += kConsumers) {
       const int b = k / p.H, e = k % p.H;
@@ -725,18 +961,50 @@ struct Consumer {
     }
   }
 
-  __device__ void phase_a(int l, int a, int b) {
+  __device__ __noinline__ void phase_a(int l, int a, int b) {
     tr(l, 0);
     const LayerDev& Lw = layer_s(p, l);
     float gr[kEPT];
     load_gains(Lw.attn_norm, gr);
-    gather_norm(l == p.l0 ? -1 : 2 * (l - 1) + 1, p.c_ctas, gr, 0);
+    if (l == p.l0) {
+      gather_norm(-1, 0u, gr, 0);
+    } else {
+      reduce_slice(p.part_c, p.c_ctas, tag_of(p.tag0, l - 1, p.l0, 3), p.rsum + (size_t)p.B * p.H,
+                   tag_of(p.tag0, l - 1, p.l0, 4));
+      tr(l, 11);
+      gather_norm(1, tag_of(p.tag0, l - 1, p.l0, 4), gr, 0);
+    }
     tr(l, 1);
     capture_rows(l);
     const int qkvd = (p.nq + 2 * p.nkv) * p.d;
     const int qd = p.nq * p.d, kvd = p.nkv * p.d, cap = rows_cap(p.H, Q8W);
-    const uint32_t tag = p.tag0 + (uint32_t)(l - p.l0);
+    const uint32_t tag = tag_of(p.tag0, l, p.l0, 0);
     const bool publish = l != p.withhold_layer;
+    if constexpr (!Q8W) {
+      // every chunk of the phase resident at once, then the tensor cores
+      int nch = 0;
+      for (int n = a; n < b; n = qkv_chunk_end(n, b, cap, qd, kvd)) ++nch;
+      for (int c = 0; c < nch; ++c) chunk_wait(c);
+      if (warp == 0) {
+        const int rs2 = row_stride(p.H, false);
+        int c = 0;
+        for (int n = a; n < b; ++c) {
+          const int e = qkv_chunk_end(n, b, cap, qd, kvd);
+          for (int i = lane; i < e - n; i += 32) rowaddr()[n - a + i] = stage_addr(c) + i * rs2;
+          n = e;
+        }
+      }
+      consumer_sync();
+      mma_rows(b - a);
+      for (int t = tid; t < (b - a) * p.B; t += kConsumers) {
+        const int rr = t / p.B, bb = t % p.B;
+        if (publish && !quit)
+          st_tag(p.xq + (size_t)bb * qkvd + a + rr, ys()[rr * 4 + bb] * inv_of(bb), tag);
+      }
+      for (int c = 0; c < nch; ++c) chunk_release();
+      tr(l, 2);
+      return;
+    }
     const int rb = Q8W ? p.H : 2 * p.H;
     for (int n = a; n < b;) {
       const int e = qkv_chunk_end(n, b, cap, qd, kvd), nr = e - n;
@@ -798,24 +1066,8 @@ struct Consumer {
       const int i = lane * E + e;
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
-        const unsigned long long* w = src + i + part * half;
-        unsigned long long x = xs[e][part];
-        if ((uint32_t)(x >> 32) != want && !quit) {
-          unsigned long long t0 = 0;
-          int spins = 0;
-          do {
-            __nanosleep(20);
-            x = ld_word(w);
-            if ((++spins & 63) == 0) {
-              if (t0 == 0) t0 = now_ns();
-              if (aborted(p.abort_flag) || now_ns() - t0 > p.wait_ns) {
-                give_up();
-                break;
-              }
-            }
-          } while ((uint32_t)(x >> 32) != want);
-        }
-        (part ? hi[e] : lo[e]) = __uint_as_float((uint32_t)x);
+        const unsigned long long x = poll_word(src + i + part * half, xs[e][part], want);
+        (part ? hi[e] : lo[e]) = word_value(x);
       }
     }
   }
@@ -847,12 +1099,12 @@ struct Consumer {
 
   // q heads, k and v of (row b, group g) into shared memory; the j = 0 unit
   // also appends k and v (bf16) to the cache. Ends on a barrier.
-  __device__ void attn_prep(int l, int b, int g, int j) {
+  __device__ __noinline__ void attn_prep(int l, int b, int g, int j) {
     const int d = p.d, rep = p.nq / p.nkv, qd = p.nq * d, kvd = p.nkv * d;
     const int qkvd = qd + 2 * kvd, pos = p.pos[b];
     const LayerDev& Lw = layer_s(p, l);
     const unsigned long long* row = p.xq + (size_t)b * qkvd;
-    const uint32_t want = p.tag0 + (uint32_t)(l - p.l0);
+    const uint32_t want = tag_of(p.tag0, l, p.l0, 0);
     if (warp < rep) {
       HeadConst hc;
       head_const(Lw.q_norm, pos, hc);
@@ -905,7 +1157,6 @@ struct Consumer {
   // q holds the lane's quarter of each head in rotated 8-element blocks:
   // block c of the registers is block (c + kk) % (DQ/8) of the quarter, so
   // the 8 key lanes of one quarter read different bank groups of their keys.
-  template <int DQ>
   __device__ __forceinline__ void attend8(const float (&q)[kMaxRep][DQ], const __nv_bfloat16* Kp,
                                           const __nv_bfloat16* Vp, int nk, int vcol, int rep,
                                           AttnState& S) {
@@ -957,8 +1208,7 @@ struct Consumer {
     }
   }
 
-  template <int DQ>
-  __device__ void attn_keys(int l, int b, int g, int j, AttnState& S) {
+  __device__ __noinline__ void attn_keys(int l, int b, int g, int j, AttnState& S) {
     const int rep = p.nq / p.nkv, old = p.pos[b];
     float q[kMaxRep][DQ];
     const int qq = lane & 3;
@@ -989,7 +1239,7 @@ struct Consumer {
         int gi = g0 + ((warp - g0) % kConsumerWarps + kConsumerWarps) % kConsumerWarps;
         for (; gi < g1; gi += kConsumerWarps) {
           const int kbase = gi * 8 - j0;
-          attend8<DQ>(q, Kp + (size_t)kbase * 4 * DQ, Vp + (size_t)kbase * 4 * DQ,
+          attend8(q, Kp + (size_t)kbase * 4 * DQ, Vp + (size_t)kbase * 4 * DQ,
                       min(8, nk - kbase), vcol, rep, S);
         }
       }
@@ -1002,8 +1252,7 @@ struct Consumer {
 
   // The new key (position pos, from k_sm / v_sm) on warp 0, then the merge of
   // the warps' states into o_s[b][h][t]. Ends on a barrier.
-  template <int DQ>
-  __device__ void attn_finish(int b, int j, AttnState& S) {
+  __device__ __noinline__ void attn_finish(int b, int j, AttnState& S) {
     const int rep = p.nq / p.nkv, d = 4 * DQ, qq = lane & 3, kk = lane >> 2;
     if (warp == 0 && !quit) {
       float s[kMaxRep];
@@ -1071,20 +1320,16 @@ struct Consumer {
     consumer_sync();
   }
 
-  // Adds one contribution (per batch row: 4 consecutive elements from n4*4)
-  // to copy `copy` of accumulator version v; `with_input` adds the rows of rs.
-  __device__ __forceinline__ void contribute(int v, int copy, int n4, const float (&a)[NB][4],
-                                             bool with_input) {
+  // Stores one contributor's partial (per batch row: 4 consecutive elements
+  // from n4*4) into its slot `slot` ([B][H] words) with tag `tag`.
+  __device__ __forceinline__ void contribute(unsigned long long* slot, int n4,
+                                             const float (&a)[NB][4], uint32_t tag) {
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
       if (b >= p.B) break;
-      unsigned long long* dst = acc_row(p, v, copy, b) + 4 * n4;
+      unsigned long long* dst = slot + (size_t)b * p.H + 4 * n4;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float x = a[b][e];
-        if (with_input) x += rs[b * p.H + 4 * n4 + e];
-        red_add(dst + e, fix_word(x));
-      }
+      for (int e = 0; e < 4; ++e) st_tag(dst + e, a[b][e], tag);
     }
   }
 
@@ -1114,7 +1359,7 @@ struct Consumer {
       for (int e = 0; e < 4; ++e) acc4[b][e] = fmaf(s[b], w[e], acc4[b][e]);
   }
 
-  __device__ void phase_b(int l) {
+  __device__ __noinline__ void phase_b(int l) {
     tr(l, 3);
     const int d = p.d, ds = d / kSlice, rep = p.nq / p.nkv, H = p.H;
     for (int u = cta; u < p.n_units; u += G) {
@@ -1123,15 +1368,30 @@ struct Consumer {
         attn_prep(l, b, g, j);
         if (b == 0) tr(l, 4);
         AttnState S;
-        if (d == 128) {
-          attn_keys<32>(l, b, g, j, S);
-          attn_finish<32>(b, j, S);
-        } else {
-          attn_keys<16>(l, b, g, j, S);
-          attn_finish<16>(b, j, S);
-        }
+        attn_keys(l, b, g, j, S);
+        if (b == 0) tr(l, 13);
+        attn_finish(b, j, S);
       }
       tr(l, 5);
+      if constexpr (!Q8W) {
+        // O projection share on the tensor cores: the unit's 8 rows of Wo^T
+        // per query head (one chunk each) times its o values
+        for (int h = 0; h < rep; ++h) chunk_wait(h);
+        const int rs2 = row_stride(H, false);
+        if (warp == 0 && lane < rep * kSlice)
+          rowaddr()[lane] = stage_addr(lane / kSlice) + (lane % kSlice) * rs2;
+        fill_coef(rep * kSlice, [&](int bb, int r) {
+          return o_s()[(bb * kMaxRep + r / kSlice) * kSlice + r % kSlice];
+        });
+        consumer_sync();
+        unsigned long long* slot = p.part_b + (size_t)u * p.B * H;
+        const uint32_t t1 = tag_of(p.tag0, l, p.l0, 1);
+        mma_cols(rep * kSlice, [&](int c, int bb, float v) {
+          if (!quit) st_tag(slot + (size_t)bb * H + c, v, t1);
+        });
+        for (int h = 0; h < rep; ++h) chunk_release();
+        continue;
+      }
       // O projection share: Wo^T rows (g*rep + h)*d + 8j + t
       const int n4 = tid;
       float acc4[NB][4];
@@ -1154,23 +1414,62 @@ struct Consumer {
         }
         chunk_release();
       }
-      if (!quit && n4 < H / 4) contribute(2 * l, u % p.P, n4, acc4, u == 0);
-      consumer_sync();
-      if (tid == 0) release_count(p.cnt + (size_t)(2 * l) * kMaxCopies + u % p.P);
+      if (!quit && n4 < H / 4)
+        contribute(p.part_b + (size_t)u * p.B * H, n4, acc4, tag_of(p.tag0, l, p.l0, 1));
     }
     tr(l, 6);
   }
 
   // ---- phase C: RMSNorm + gate/up + SwiGLU + down share ------------------
 
-  __device__ void phase_c(int l, int a, int b) {
+  __device__ __noinline__ void phase_c(int l, int a, int b) {
     tr(l, 7);
     const LayerDev& Lw = layer_s(p, l);
     float gr[kEPT];
     load_gains(Lw.ffn_norm, gr);
-    gather_norm(2 * l, p.n_units, gr, 1);
+    reduce_slice(p.part_b, p.n_units, tag_of(p.tag0, l, p.l0, 1), p.rsum,
+                 tag_of(p.tag0, l, p.l0, 2));
+    tr(l, 12);
+    gather_norm(0, tag_of(p.tag0, l, p.l0, 2), gr, 1);
     tr(l, 8);
     const int H = p.H, pc = pairs_cap(H, Q8W), rb = Q8W ? H : 2 * H, sb = Q8W ? H / 32 : 0;
+    if constexpr (!Q8W) {
+      // gate/up rows: all chunks resident, one tensor-core pass over 2P rows
+      const int P = b - a, rs2 = row_stride(H, false);
+      const int ngu = (P + pc - 1) / pc;
+      for (int c = 0; c < ngu; ++c) chunk_wait(c);
+      if (warp == 0)
+        for (int q2 = lane; q2 < P; q2 += 32) {
+          const uint32_t st2 = stage_addr(q2 / pc);
+          rowaddr()[q2] = st2 + (q2 % pc) * rs2;
+          rowaddr()[P + q2] = st2 + (pc + q2 % pc) * rs2;
+        }
+      consumer_sync();
+      mma_rows(2 * P);
+      for (int t = tid; t < P * p.B; t += kConsumers) {
+        const int q2 = t / p.B, bb = t % p.B;
+        const float y = ys()[q2 * 4 + bb] * inv_of(bb), z = ys()[(P + q2) * 4 + bb] * inv_of(bb);
+        act_s()[bb * 128 + q2] = y / (1.f + expf(-y)) * z;
+      }
+      for (int c = 0; c < ngu; ++c) chunk_release();
+      tr(l, 9);
+      // down share: the CTA's P rows of Wd^T times its SwiGLU outputs
+      const int rc = rows_cap(H, false), nd = (P + rc - 1) / rc;
+      for (int c = 0; c < nd; ++c) chunk_wait(c);
+      consumer_sync();  // act_s complete; rowaddr free again
+      if (warp == 0)
+        for (int j = lane; j < P; j += 32) rowaddr()[j] = stage_addr(j / rc) + (j % rc) * rs2;
+      fill_coef(P, [&](int bb, int r) { return act_s()[bb * 128 + r]; });
+      consumer_sync();
+      unsigned long long* slot = p.part_c + (size_t)cta * p.B * H;
+      const uint32_t t3 = tag_of(p.tag0, l, p.l0, 3);
+      mma_cols(P, [&](int c, int bb, float v) {
+        if (!quit) st_tag(slot + (size_t)bb * H + c, v, t3);
+      });
+      for (int c = 0; c < nd; ++c) chunk_release();
+      tr(l, 10);
+      return;
+    }
     for (int n = a; n < b;) {
       const int e = min(b, n + pc), nr = e - n;
       const unsigned char* st = chunk_wait();
@@ -1219,94 +1518,52 @@ struct Consumer {
       chunk_release();
       n = e;
     }
-    if (!quit && a < b && n4 < H / 4) contribute(2 * l + 1, cta % p.P, n4, acc4, cta == 0);
-    consumer_sync();
-    if (tid == 0 && a < b) release_count(p.cnt + (size_t)(2 * l + 1) * kMaxCopies + cta % p.P);
+    if (!quit && n4 < H / 4)
+      contribute(p.part_c + (size_t)cta * p.B * H, n4, acc4, tag_of(p.tag0, l, p.l0, 3));
     tr(l, 10);
   }
 
   // ---- tail: final norm + LM head + greedy, or the block output -----------
 
-  __device__ void tail(int a, int b) {
+  __device__ __noinline__ void tail(int a, int b) {
     const int L = p.L;
     tr(L, 0);
     float gr[kEPT];
     load_gains(p.final_norm, gr);
+    const uint32_t t_out = tag_of(p.tag0, p.l1 - 1, p.l0, 4);
+    reduce_slice(p.part_c, p.c_ctas, tag_of(p.tag0, p.l1 - 1, p.l0, 3),
+                 p.rsum + (size_t)p.B * p.H, t_out);
+    tr(L, 11);
     if (!p.run_head) {
-      // the block output: only CTA 0 waits for it (gather_norm's barrier is
-      // CTA-local)
+      // the block output: every CTA reduced its slice; CTA 0 collects it
       if (cta == 0) {
-        gather_norm(2 * (p.l1 - 1) + 1, p.c_ctas, gr, 0);
+        gather_norm(1, t_out, gr, 0);
         capture_rows(p.l1);
         if (p.h_out)
           for (int k = tid; k < p.B * p.H; k += kConsumers) p.h_out[k] = rs[k];
       }
       return;
     }
-    gather_norm(2 * (p.l1 - 1) + 1, p.c_ctas, gr, 0);
+    gather_norm(1, t_out, gr, 0);
     tr(L, 1);
     consumer_sync();  // rs complete before CTA 0 copies it out
     capture_rows(p.l1);
     if (cta == 0 && p.h_out)
       for (int k = tid; k < p.B * p.H; k += kConsumers) p.h_out[k] = rs[k];
-    const int cap = p.lm_rows, rb = 2 * p.H;
-    for (int n = a; n < b && p.lm_owner;) {
+    const int cap = p.lm_rows;
+    for (int n = a; n < b;) {
       const int e = min(b, n + cap), nr = e - n;
-      if ((int)(i % kConsumerWarps) == warp) {
+      if ((int)(i % p.lm_owners) == warp) {
         const unsigned char* st = chunk_wait_owned();
-        if (!quit) lm_rows_owned(st, n, nr);
+        if (!quit) lm_rows_mma(st, n, nr);
         __syncwarp();
-        if (lane == 0) mbar_arrive_n(&r.empty[stage], kConsumerWarps);
+        if (lane == 0 && !quit) mbar_arrive_n(&r.empty[stage], kConsumerWarps);
       }
       cursor_advance();
       n = e;
     }
-    for (int n = a; n < b && !p.lm_owner;) {
-      const int e = min(b, n + cap), nr = e - n;
-      const unsigned char* st = chunk_wait();
-      int r0 = (warp - (n - a)) % kConsumerWarps;
-      if (r0 < 0) r0 += kConsumerWarps;
-      if (!quit) {
-        for (int rr = r0; rr < nr; rr += kConsumerWarps) {
-          float acc[NB];
-          lm_dot(st + rr * rb, acc);
-          if (lane == 0) {
-#pragma unroll
-            for (int bb = 0; bb < NB; ++bb) {
-              if (bb >= p.B) break;
-              fold_logit(bb, n + rr, acc[bb] * inv[bb]);
-            }
-          }
-        }
-      }
-      chunk_release();
-      n = e;
-    }
     tr(L, 2);
     finish_head();
-  }
-
-  // Sum of 8 per-lane values over the warp in 9 shuffles: each step halves
-  // the values a lane keeps. Lane l ends with the total of value
-  // 4*bit4(l) + 2*bit3(l) + bit2(l).
-  __device__ __forceinline__ float reduce8(const float (&v)[8]) {
-    const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4;
-    float a4[4], c2[2];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const float keep = h16 ? v[r + 4] : v[r], send = h16 ? v[r] : v[r + 4];
-      a4[r] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-    }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const float keep = h8 ? a4[r + 2] : a4[r], send = h8 ? a4[r] : a4[r + 2];
-      c2[r] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-    }
-    const float keep = h4 ? c2[1] : c2[0], send = h4 ? c2[0] : c2[1];
-    float t = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-    t += __shfl_xor_sync(0xffffffffu, t, 2);
-    t += __shfl_xor_sync(0xffffffffu, t, 1);
-    return t;
   }
 
   // Greedy key of logit y at vocabulary id `id`: order-preserving in y (+0 and
@@ -1323,85 +1580,8 @@ struct Consumer {
     }
   }
 
-  // All rows (up to 8) of an LM-head chunk on this warp: the lane's 8-element
-  // blocks of every row with shared activation loads, one transposing
-  // reduction per batch row.
-  __device__ __forceinline__ void lm_rows_owned(const unsigned char* st, int n0, int nr) {
-    const int H = p.H;
-    float acc[8][NB];
-#pragma unroll
-    for (int r = 0; r < 8; ++r)
-#pragma unroll
-      for (int b = 0; b < NB; ++b) acc[r][b] = 0.f;
-#pragma unroll
-    for (int it = 0; it < IT; ++it) {
-      const int k = lane * 8 + it * 256;
-      float z[NB][8];
-#pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        if (b < p.B) {
-          const float4 z0 = *reinterpret_cast<const float4*>(zs + b * H + k);
-          const float4 z1 = *reinterpret_cast<const float4*>(zs + b * H + k + 4);
-          z[b][0] = z0.x; z[b][1] = z0.y; z[b][2] = z0.z; z[b][3] = z0.w;
-          z[b][4] = z1.x; z[b][5] = z1.y; z[b][6] = z1.z; z[b][7] = z1.w;
-        } else {
-#pragma unroll
-          for (int q = 0; q < 8; ++q) z[b][q] = 0.f;
-        }
-      }
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        if (r >= nr) break;
-        const uint4 u = *reinterpret_cast<const uint4*>(st + r * 2 * H + 2 * k);
-        const float w[8] = {lo16(u.x), hi16(u.x), lo16(u.y), hi16(u.y),
-                            lo16(u.z), hi16(u.z), lo16(u.w), hi16(u.w)};
-#pragma unroll
-        for (int b = 0; b < NB; ++b)
-#pragma unroll
-          for (int q = 0; q < 8; ++q) acc[r][b] = fmaf(w[q], z[b][q], acc[r][b]);
-      }
-    }
-    const int my_r = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      float col[8];
-#pragma unroll
-      for (int r = 0; r < 8; ++r) col[r] = acc[r][b];
-      const float tot = reduce8(col);
-      if (b < p.B && (lane & 3) == 0 && my_r < nr) fold_logit(b, n0 + my_r, tot * inv[b]);
-    }
-  }
-
-  // bf16 row dot for the LM head (the embedding is bf16 in every format).
-  __device__ __forceinline__ void lm_dot(const unsigned char* row, float (&acc)[NB]) {
-    const int H = p.H;
-#pragma unroll
-    for (int b = 0; b < NB; ++b) acc[b] = 0.f;
-#pragma unroll
-    for (int it = 0; it < IT; ++it) {
-      const int k = lane * 8 + it * 256;
-      const uint4 u = *reinterpret_cast<const uint4*>(row + 2 * k);
-      const float w[8] = {lo16(u.x), hi16(u.x), lo16(u.y), hi16(u.y),
-                          lo16(u.z), hi16(u.z), lo16(u.w), hi16(u.w)};
-#pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        if (b < p.B) {
-          const float4 z0 = *reinterpret_cast<const float4*>(zs + b * H + k);
-          const float4 z1 = *reinterpret_cast<const float4*>(zs + b * H + k + 4);
-          float t = acc[b];
-          t = fmaf(w[0], z0.x, t); t = fmaf(w[1], z0.y, t); t = fmaf(w[2], z0.z, t);
-          t = fmaf(w[3], z0.w, t); t = fmaf(w[4], z1.x, t); t = fmaf(w[5], z1.y, t);
-          t = fmaf(w[6], z1.z, t); t = fmaf(w[7], z1.w, t);
-          acc[b] = t;
-        }
-      }
-    }
-#pragma unroll
-    for (int b = 0; b < NB; ++b) acc[b] = warp_sum(acc[b]);
-  }
-
   // Fold this CTA's greedy keys; the last CTA to finish writes the ids.
-  __device__ void finish_head() {
+  __device__ __noinline__ void finish_head() {
     if (tid < kMaxB) best[tid] = 0ull;
     consumer_sync();
 #pragma unroll
@@ -1440,7 +1620,7 @@ struct Consumer {
   }
 };
 
-template <int NB, bool Q8W, int IT>
+template <int NB, bool Q8W, int IT, int DQ>
 __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) unsigned char smem[];
   Ring ring;
@@ -1472,10 +1652,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
         bt[k] = p.kv.block_table[(size_t)p.seq[k / pps] * pps + k % pps];
     }
   }
+  if (threadIdx.x < 16)  // the 64 zero bytes the tensor-core loads use for padding rows
+    reinterpret_cast<uint32_t*>(smem + p.off_misc + 4160)[threadIdx.x] = 0u;
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x, c = blockIdx.x;
   const int qkvd = (p.nq + 2 * p.nkv) * p.d;
+  unsigned long long* trow =
+      p.trace ? p.trace + ((size_t)c * (p.L + 1) + p.L) * kTraceSlots : nullptr;
+  if (trow && threadIdx.x == 0) {
+    trow[12] = now_ns();
+    trow[13] = clock64();
+  }
   volatile unsigned int* counts =
       reinterpret_cast<volatile unsigned int*>(smem + p.off_misc + 4096 + 8 * kMaxB + 8);
   if (warp == kConsumerWarps) {
@@ -1492,16 +1680,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
       int a, b;
       slice(p.V, G, c, a, b);
       if (!pr.quit) pr.tail(a, b);
-      if (p.trace) p.trace[((size_t)c * (p.L + 1) + p.L) * kTraceSlots + 3] = now_ns();
+      if (trow) trow[3] = clock64();
       counts[0] = pr.i;
-    } else {
-      // the idle lanes clear this CTA's share of the other accumulator set
-      long long a0 = p.clear_words * c / G, a1 = p.clear_words * (c + 1) / G;
-      for (long long k = a0 + lane - 1; k < a1; k += 31) p.clear[k] = 0ull;
     }
   } else {
-    Consumer<NB, Q8W, IT> cs(p, ring, smem);
-    for (int l = p.l0; l < p.l1 && !cs.quit; ++l) {
+    Consumer<NB, Q8W, IT, DQ> cs(p, ring, smem);
+    // `quit` is per thread (a wait that gave up), so it must not steer any
+    // path that holds a consumer barrier: after an abort every thread still
+    // walks all phases, with each wait returning at once and no stores.
+    for (int l = p.l0; l < p.l1; ++l) {
       int a, b;
       slice(qkvd, G, c, a, b);
       cs.phase_a(l, a, b);
@@ -1515,6 +1702,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     if (threadIdx.x == 0) counts[1] = cs.i;
   }
   __syncthreads();
+  if (trow && threadIdx.x == 0) {
+    trow[14] = now_ns();
+    trow[15] = clock64();
+  }
   // Drain: copies issued but never consumed (after an abort) must land before
   // the CTA's shared memory is released.
   if (threadIdx.x == 0) {
@@ -1554,10 +1745,10 @@ __global__ void transpose_kernel(const T* __restrict__ in, int rows, int cols, T
 namespace {
 
 struct FusedState {
-  unsigned long long* xq = nullptr;
-  unsigned long long* acc = nullptr;  // [2 sets][set words]
-  long long set_words = 0;
-  long long dirty[2] = {0, 0};        // words of each set written since its last clear
+  unsigned long long* xq = nullptr;      // [kMaxB][qkv dim]
+  unsigned long long* part_b = nullptr;  // [attention units][kMaxB][H]
+  unsigned long long* part_c = nullptr;  // [SMs][kMaxB][H]
+  unsigned long long* rsum = nullptr;    // [2][kMaxB][H]
   unsigned long long* am_key = nullptr;
   unsigned int* am_cnt = nullptr;
   int* abort_flag = nullptr;
@@ -1570,6 +1761,7 @@ struct FusedState {
   uint32_t next_tag = 1;
   unsigned long long step = 0;
   int sms = 0;
+  int need_stages = 1;
   bool eligible = false;
   unsigned long long wait_ns = 1000000000ull;
   int withhold = -1;
@@ -1580,18 +1772,44 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 bool shape_ok(const fs_model* m) {
   const Shape& s = m->s;
   const int rep = s.nq / s.nkv;
-  if (rep < 1 || rep > fused::kMaxRep || (s.d != 64 && s.d != 128)) return false;
-  if (s.H != 256 && s.H != 1024) return false;
+  if (rep < 1 || rep > fused::kMaxRep) return false;
+  // compiled pairs: hidden 1024 with head_dim 128, hidden 256 with head_dim 64
+  if (!((s.H == 1024 && s.d == 128) || (s.H == 256 && s.d == 64))) return false;
   if (s.V >= 0x7fffffff || s.L > 64) return false;
   if (s.I % 32 || s.q_dim() % 32) return false;
   if (s.I < m->num_sms) return false;  // every CTA owns intermediate columns
   if (s.I / m->num_sms + 2 > 128) return false;  // act_s holds 128 columns per row
   if (fused::rows_cap(s.H, m->q8) < 1 || fused::pairs_cap(s.H, m->q8) < 1) return false;
+  // tensor-core GEMVs: at most 48 rows per pass (QKV rows of a CTA, 2x its
+  // gate/up pairs) and 32 coefficient rows (down share, O share)
+  const int per = (s.I + m->num_sms - 1) / m->num_sms;
+  const int qkv_per = (s.qkv_dim() + m->num_sms - 1) / m->num_sms;
+  if (2 * per > 48 || qkv_per > 48 || per > 32 || rep * fused::kSlice > 32) return false;
   return true;
 }
 
+// The most chunks one phase holds at once in the ring (the bf16 phases wait
+// for all their chunks before the tensor-core pass).
+int chunks_needed(const Shape& s, int sms, bool q8) {
+  if (q8) return 1;
+  const int qd = s.nq * s.d, kvd = s.nkv * s.d, qkvd = s.qkv_dim();
+  const int cap = fused::rows_cap(s.H, false), pc = fused::pairs_cap(s.H, false);
+  int most = s.nq / s.nkv;
+  for (int c = 0; c < sms; ++c) {
+    int a, b, n = 0;
+    fused::slice(qkvd, sms, c, a, b);
+    for (int k = a; k < b; k = fused::qkv_chunk_end(k, b, cap, qd, kvd)) ++n;
+    most = std::max(most, n);
+    fused::slice(s.I, sms, c, a, b);
+    most = std::max(most, (b - a + pc - 1) / pc);
+    most = std::max(most, (b - a + cap - 1) / cap);
+  }
+  return most;
+}
+
 void state_free(FusedState* st) {
-  void* bufs[] = {st->xq, st->acc, st->am_key, st->am_cnt, st->abort_flag, st->layers, st->tl};
+  void* bufs[] = {st->xq,     st->part_b,     st->part_c, st->rsum,  st->am_key,
+                  st->am_cnt, st->abort_flag, st->layers, st->tl};
   for (void* b : bufs)
     if (b) cudaFree(b);
   for (int l = 0; l < 64; ++l) {
@@ -1624,6 +1842,7 @@ fs_status fused_init(fs_model* m) {
   st->eligible = shape_ok(m);
   if (!st->eligible) return FS_OK;
   const Shape& s = m->s;
+  st->need_stages = chunks_needed(s, m->num_sms, m->q8);
   auto alloc = [&](void** p, size_t bytes) {
     if (cudaMalloc(p, bytes) != cudaSuccess) {
       cudaGetLastError();
@@ -1635,9 +1854,12 @@ fs_status fused_init(fs_model* m) {
   };
   const size_t w = sizeof(unsigned long long);
   // per set: arrival counters [2L][kMaxCopies], then the accumulator words
-  st->set_words = (long long)2 * s.L * fused::kMaxCopies * (1 + fused::kMaxB * s.H);
+  const size_t units = (size_t)s.nkv * (s.d / fused::kSlice);
+  const size_t rows = (size_t)fused::kMaxB * s.H;
   bool ok = alloc((void**)&st->xq, (size_t)fused::kMaxB * s.qkv_dim() * w) &&
-            alloc((void**)&st->acc, (size_t)2 * st->set_words * w) &&
+            alloc((void**)&st->part_b, units * rows * w) &&
+            alloc((void**)&st->part_c, (size_t)st->sms * rows * w) &&
+            alloc((void**)&st->rsum, 2 * rows * w) &&
             alloc((void**)&st->am_key, (size_t)fused::kMaxB * w) &&
             alloc((void**)&st->am_cnt, 64) && alloc((void**)&st->abort_flag, 64) &&
             alloc((void**)&st->layers, (size_t)s.L * sizeof(LayerDev)) &&
@@ -1676,10 +1898,10 @@ fs_status fused_init(fs_model* m) {
   cudaMemcpy(st->layers, m->layers.data(), (size_t)s.L * sizeof(LayerDev), cudaMemcpyHostToDevice);
   cudaMemcpy(st->tl, tl.data(), (size_t)s.L * sizeof(fused::TLayer), cudaMemcpyHostToDevice);
   const void* kernels[] = {
-      (const void*)fused::decode_fused_kernel<1, false, 4>, (const void*)fused::decode_fused_kernel<1, true, 4>,
-      (const void*)fused::decode_fused_kernel<4, false, 4>, (const void*)fused::decode_fused_kernel<4, true, 4>,
-      (const void*)fused::decode_fused_kernel<1, false, 1>, (const void*)fused::decode_fused_kernel<1, true, 1>,
-      (const void*)fused::decode_fused_kernel<4, false, 1>, (const void*)fused::decode_fused_kernel<4, true, 1>};
+      (const void*)fused::decode_fused_kernel<1, false, 4, 32>, (const void*)fused::decode_fused_kernel<1, true, 4, 32>,
+      (const void*)fused::decode_fused_kernel<4, false, 4, 32>, (const void*)fused::decode_fused_kernel<4, true, 4, 32>,
+      (const void*)fused::decode_fused_kernel<1, false, 1, 16>, (const void*)fused::decode_fused_kernel<1, true, 1, 16>,
+      (const void*)fused::decode_fused_kernel<4, false, 1, 16>, (const void*)fused::decode_fused_kernel<4, true, 1, 16>};
   for (const void* k : kernels)
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
   return FS_OK;
@@ -1698,8 +1920,6 @@ void fused_reset(fs_model* m) {
   FusedState* st = static_cast<FusedState*>(m->extras);
   if (!st || !st->eligible) return;
   cudaDeviceSynchronize();
-  cudaMemset(st->acc, 0, (size_t)2 * st->set_words * sizeof(unsigned long long));
-  st->dirty[0] = st->dirty[1] = 0;
   cudaMemset(st->am_key, 0, (size_t)fused::kMaxB * sizeof(unsigned long long));
   cudaMemset(st->am_cnt, 0, 64);
   cudaMemset(st->abort_flag, 0, 64);
@@ -1737,15 +1957,9 @@ fs_status decode_fused(fs_model* m, const fs_kv* kv, const RowMap& map, int B, c
   }
   p.tokens = tok;
   p.xq = st->xq;
-  const int set = (int)(st->step & 1);
-  p.cnt = st->acc + (size_t)set * st->set_words;
-  p.acc = p.cnt + (size_t)2 * s.L * fused::kMaxCopies;
-  p.P = std::max(1, std::min(fused::kMaxCopies, fused::kMaxCopies / B));
-  // the other set: clear the rows its last user wrote
-  p.clear = st->acc + (size_t)(1 - set) * st->set_words;
-  p.clear_words = st->dirty[1 - set];
-  st->dirty[1 - set] = 0;
-  st->dirty[set] = std::max(st->dirty[set], (long long)2 * s.L * (fused::kMaxCopies + p.P * B * s.H));
+  p.part_b = st->part_b;
+  p.part_c = st->part_c;
+  p.rsum = st->rsum;
   p.n_units = s.nkv * (s.d / fused::kSlice);
   p.c_ctas = std::min(s.I, st->sms);
   p.l0 = l0;
@@ -1769,15 +1983,20 @@ fs_status decode_fused(fs_model* m, const fs_kv* kv, const RowMap& map, int B, c
   if (st->next_tag > 0xF0000000u) {
     // wrap: clear the tags so the numbering can restart
     cudaStreamSynchronize(stream);
-    cudaMemsetAsync(st->xq, 0, (size_t)fused::kMaxB * s.qkv_dim() * sizeof(unsigned long long),
-                    stream);
+    const size_t w = sizeof(unsigned long long), rows = (size_t)fused::kMaxB * s.H;
+    cudaMemsetAsync(st->xq, 0, (size_t)fused::kMaxB * s.qkv_dim() * w, stream);
+    cudaMemsetAsync(st->part_b, 0, (size_t)p.n_units * rows * w, stream);
+    cudaMemsetAsync(st->part_c, 0, (size_t)st->sms * rows * w, stream);
+    cudaMemsetAsync(st->rsum, 0, 2 * rows * w, stream);
     st->next_tag = 1;
   }
   p.tag0 = st->next_tag;
-  st->next_tag += (uint32_t)(l1 - l0) + 1u;
+  st->next_tag += 5u * (uint32_t)(l1 - l0) + 1u;
   // shared memory carve-up
   const size_t rows_bytes = align_up((size_t)B * s.H * 4, 128);
-  const size_t misc = 4096 + 256;
+  const size_t zs_bytes = m->q8 ? 2 * rows_bytes : 0;
+  const size_t zt_bytes = align_up((size_t)2 * 2 * B * (s.H + 8) * 2, 128);
+  const size_t misc = 5120;
   const size_t attn = align_up((size_t)(fused::kMaxRep * 128 + 256 +
                                         fused::kConsumerWarps * fused::kMaxRep * 10) * 4, 128);
   const size_t tab_ptrs = (size_t)s.L * (sizeof(LayerDev) + sizeof(fused::TLayer));
@@ -1785,35 +2004,47 @@ fs_status decode_fused(fs_model* m, const fs_kv* kv, const RowMap& map, int B, c
   const bool bt_smem = bt_bytes <= 8192;
   const size_t tab = align_up(tab_ptrs + (bt_smem ? bt_bytes : 0), 128);
   const size_t bars = 2 * fused::kMaxStages * 8;
-  const size_t fixed = 3 * rows_bytes + misc + attn + tab + bars;
+  // the slice reducer: [contributors][slice] values + 4 partial sums per element
+  const int emax = (B * s.H + st->sms - 1) / st->sms;
+  // ... and the tensor-core partial sums: 3 row tiles x H/128 k-blocks x 64
+  const size_t red = align_up(std::max((size_t)(std::max(p.n_units, st->sms) + 4) * emax * 4,
+                                       (size_t)3 * (s.H / 128) * 64 * 4),
+                              128);
+  const size_t fixed = rows_bytes + zs_bytes + zt_bytes + misc + attn + tab + bars + red;
   const size_t budget = 232448;
-  int n_stages = (int)((budget - fixed) / fused::kStageBytes);
+  p.stage_bytes = m->q8 ? fused::kStageQ8 : fused::kStageBf16;
+  int n_stages = (int)((budget - fixed) / (size_t)p.stage_bytes);
   n_stages = std::min(n_stages, fused::kMaxStages);
-  if (n_stages < 4) return FS_ERR_UNSUPPORTED;
-  size_t off = (size_t)n_stages * fused::kStageBytes;
+  if (n_stages < 4 || n_stages < st->need_stages) return FS_ERR_UNSUPPORTED;
+  size_t off = (size_t)n_stages * p.stage_bytes;
   p.off_r = (int)off; off += rows_bytes;
-  p.off_z = (int)off; off += 2 * rows_bytes;
+  p.off_z = (int)off; off += zs_bytes;
+  p.off_zt = (int)off; off += zt_bytes;
   p.off_misc = (int)off; off += misc;
   p.off_attn = (int)off; off += attn;
   p.off_bar = (int)off; off += bars;
   p.off_tab = (int)off; off += tab;
+  p.off_red = (int)off; off += red;
   p.bt_in_smem = bt_smem ? 1 : 0;
   p.n_stages = n_stages;
-  p.lm_owner = n_stages >= fused::kConsumerWarps ? 1 : 0;
+  // A warp that consumes only every lm_owners-th chunk tests the release of
+  // the chunk a ring earlier before the chunk itself; that test is
+  // unambiguous when the ring holds at least lm_owners stages.
+  p.lm_owners = std::min(fused::kConsumerWarps, n_stages);
   p.lm_rows = std::min(8, fused::rows_cap(s.H, false));
   void* args[] = {&p};
   const bool h1k = s.H == 1024;
   const void* fn;
   if (B == 1)
-    fn = m->q8 ? (h1k ? (const void*)fused::decode_fused_kernel<1, true, 4>
-                      : (const void*)fused::decode_fused_kernel<1, true, 1>)
-               : (h1k ? (const void*)fused::decode_fused_kernel<1, false, 4>
-                      : (const void*)fused::decode_fused_kernel<1, false, 1>);
+    fn = m->q8 ? (h1k ? (const void*)fused::decode_fused_kernel<1, true, 4, 32>
+                      : (const void*)fused::decode_fused_kernel<1, true, 1, 16>)
+               : (h1k ? (const void*)fused::decode_fused_kernel<1, false, 4, 32>
+                      : (const void*)fused::decode_fused_kernel<1, false, 1, 16>);
   else
-    fn = m->q8 ? (h1k ? (const void*)fused::decode_fused_kernel<4, true, 4>
-                      : (const void*)fused::decode_fused_kernel<4, true, 1>)
-               : (h1k ? (const void*)fused::decode_fused_kernel<4, false, 4>
-                      : (const void*)fused::decode_fused_kernel<4, false, 1>);
+    fn = m->q8 ? (h1k ? (const void*)fused::decode_fused_kernel<4, true, 4, 32>
+                      : (const void*)fused::decode_fused_kernel<4, true, 1, 16>)
+               : (h1k ? (const void*)fused::decode_fused_kernel<4, false, 4, 32>
+                      : (const void*)fused::decode_fused_kernel<4, false, 1, 16>);
   count_launches();
   cudaError_t e = cudaLaunchCooperativeKernel(fn, dim3(st->sms), dim3(fused::kThreads), args, off,
                                               stream);

@@ -5,11 +5,28 @@
 
 namespace fs {
 
-fs_status init_extras(fs_model* m) { return fused_init(m); }
+fs_status init_extras(fs_model* m) {
+  fs_status s = fused_init(m);
+  if (s != FS_OK) return s;
+  return cluster_init(m);
+}
 
 void release_extras(fs_model* m) {
+  cluster_release(m);
   fused_release(m);
   tc_release(m);
+}
+
+fs_status decode_persistent(fs_model* m, const fs_kv* kv, const RowMap& map, int B,
+                            const int32_t* tok, const float* h_in, float* h_out, int l0, int l1,
+                            bool run_head, float* logits, int32_t* argmax, cudaStream_t stream) {
+  if (m->decode_path == 2) return FS_ERR_UNSUPPORTED;
+  if (m->decode_path == 0) {
+    fs_status s = decode_cluster(m, kv, map, B, tok, h_in, h_out, l0, l1, run_head, logits,
+                                 argmax, stream);
+    if (s != FS_ERR_UNSUPPORTED) return s;
+  }
+  return decode_fused(m, kv, map, B, tok, h_in, h_out, l0, l1, run_head, logits, argmax, stream);
 }
 
 fs_status ensure_gen_buffer(fs_model* m, int n) {
@@ -44,8 +61,8 @@ fs_status block_prefill_or_general(fs_model* m, const fs_kv* kv, const RowMap& m
 fs_status decode_rows(fs_model* m, const fs_kv* kv, const RowMap& map, int rows,
                       const int32_t* tok, float* logits, int32_t* argmax, cudaStream_t st) {
   // Distinct sequences (checked by the caller), at most 4: the persistent kernel.
-  fs_status s = decode_fused(m, kv, map, rows, tok, nullptr, nullptr, 0, m->s.L, true, logits,
-                             argmax, st);
+  fs_status s = decode_persistent(m, kv, map, rows, tok, nullptr, nullptr, 0, m->s.L, true,
+                                  logits, argmax, st);
   if (s != FS_ERR_UNSUPPORTED) return s;
   return forward_general(m, kv, map, rows, tok, 0, logits, argmax, 0, rows, st);
 }

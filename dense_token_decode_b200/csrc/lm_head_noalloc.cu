@@ -86,8 +86,17 @@ extern "C" fs_status fs_lm_head_argmax_noalloc(const void* embed, const void* fi
   }
   void* base = nullptr;
   {
-    // Set-up, once per device, on the first call made with that device current.
+    // The array's device address: looked up again on every call made outside
+    // a stream capture (so a context torn down by cudaDeviceReset and made
+    // anew never leaves a stale address behind), and taken from the last
+    // lookup inside a capture, where the lookup is not allowed.
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(static_cast<cudaStream_t>(stream), &cap) != cudaSuccess) {
+      cudaGetLastError();
+      cap = cudaStreamCaptureStatusNone;
+    }
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (cap == cudaStreamCaptureStatusNone) g_noalloc_addr[dev] = nullptr;
     if (!g_noalloc_addr[dev]) {
       cudaError_t e = cudaGetSymbolAddress(&g_noalloc_addr[dev], g_noalloc_scratch);
       if (e != cudaSuccess) {

@@ -224,7 +224,10 @@ extern "C" fs_status fs_device_error(fs_model* m, int32_t* code) {
   int v = 0;
   FS_CUDA(cudaMemcpy(&v, m->err, sizeof(int), cudaMemcpyDeviceToHost));
   FS_CUDA(cudaMemset(m->err, 0, sizeof(int)));
-  if (v) fs::fused_reset(m);
+  if (v) {
+    fs::fused_reset(m);
+    fs::cluster_reset(m);
+  }
   *code = v;
   return FS_OK;
 }
@@ -548,12 +551,87 @@ fs_status decode_impl(fs_model* m, fs_kv* kv, const int32_t* seqs, const int32_t
   return FS_OK;
 }
 
+// A mixed batch: segment i appends n_tokens[i] ids of sequence seqs[i]. The
+// rows go through one general forward, ordered so that every segment's last
+// row comes at the end (in segment order): the LM head then runs on exactly
+// those rows. Every row's K/V is appended before any row attends, so the
+// order does not change what a row sees.
+fs_status batch_impl(fs_model* m, fs_kv* kv, const int32_t* seqs, const int32_t* n_tokens,
+                     int32_t n_seqs, const int32_t* tokens, float* logits, int32_t* argmax,
+                     cudaStream_t st) {
+  if (!m || !kv) return fail(FS_ERR_NULL, "model or kv is NULL");
+  if (kv->model != m) return fail(FS_ERR_INVALID, "kv belongs to another model");
+  if (!seqs || !n_tokens || !tokens) return fail(FS_ERR_NULL, "seqs, n_tokens or tokens is NULL");
+  if (n_seqs <= 0) return fail(FS_ERR_EMPTY, "a batch needs at least one segment");
+  fs_status s;
+  if ((s = check_out_ptr(logits, "logits_out")) != FS_OK) return s;
+  if ((s = check_i32_out(argmax, "argmax_out")) != FS_OK) return s;
+  long long total = 0;
+  const int cap = kv_capacity(kv);
+  for (int i = 0; i < n_seqs; ++i) {
+    const int q = seqs[i];
+    if (q < 0 || q >= kv->max_seqs) return fail(FS_ERR_SEQ, "sequence out of range");
+    for (int j = 0; j < i; ++j)
+      if (seqs[j] == q) return fail(FS_ERR_SEQ, "a sequence appears twice in one batch");
+    if (n_tokens[i] <= 0) return fail(FS_ERR_EMPTY, "every segment needs at least one token");
+    if ((long long)kv->len[q] + n_tokens[i] > cap)
+      return fail(FS_ERR_CONTEXT, "a segment would exceed max_pos or the KV capacity");
+    total += n_tokens[i];
+  }
+  if (total > kMaxBatch) return fail(FS_ERR_INVALID, "a batch holds at most 64 rows in all");
+  const int rows = (int)total;
+  std::vector<int32_t> in(rows);
+  if (pointer_kind(tokens) == 1) {
+    FS_CUDA(cudaMemcpyAsync(in.data(), tokens, (size_t)rows * sizeof(int32_t),
+                            cudaMemcpyDeviceToHost, st));
+    FS_CUDA(cudaStreamSynchronize(st));
+  } else {
+    std::copy(tokens, tokens + rows, in.begin());
+  }
+  RowMap map{};
+  map.n_list = rows;
+  std::vector<int32_t> ordered(rows);
+  int r = 0, c0 = 0;
+  for (int i = 0; i < n_seqs; ++i) {  // all but the last row of every segment
+    for (int t = 0; t + 1 < n_tokens[i]; ++t, ++r) {
+      map.seq[r] = seqs[i];
+      map.pos[r] = kv->len[seqs[i]] + t;
+      ordered[r] = in[c0 + t];
+    }
+    c0 += n_tokens[i];
+  }
+  c0 = 0;
+  for (int i = 0; i < n_seqs; ++i, ++r) {  // the last rows
+    const int t = n_tokens[i] - 1;
+    map.seq[r] = seqs[i];
+    map.pos[r] = kv->len[seqs[i]] + t;
+    ordered[r] = in[c0 + t];
+    c0 += n_tokens[i];
+  }
+  const int32_t* dev_tok = nullptr;
+  if ((s = stage_tokens(m, ordered.data(), rows, m->tok, &dev_tok, st)) != FS_OK) return s;
+  if ((s = forward_general(m, kv, map, rows, dev_tok, rows - n_seqs, logits, argmax, 0, rows,
+                           st)) != FS_OK)
+    return s;
+  for (int i = 0; i < n_seqs; ++i) kv->len[seqs[i]] += n_tokens[i];
+  if (m->capture) m->capture = nullptr;
+  return FS_OK;
+}
+
 }  // namespace fs
 
 extern "C" fs_status fs_prefill(fs_model* m, fs_kv* kv, int32_t seq, const int32_t* tokens,
                                 int32_t n, float* logits, int32_t* argmax, void* stream) {
   return fs::prefill_impl(m, kv, seq, tokens, n, logits, argmax,
                           static_cast<cudaStream_t>(stream));
+}
+
+extern "C" fs_status fs_forward_batch(fs_model* m, fs_kv* kv, const int32_t* seqs,
+                                      const int32_t* n_tokens, int32_t n_seqs,
+                                      const int32_t* tokens, float* logits, int32_t* argmax,
+                                      void* stream) {
+  return fs::batch_impl(m, kv, seqs, n_tokens, n_seqs, tokens, logits, argmax,
+                        static_cast<cudaStream_t>(stream));
 }
 
 extern "C" fs_status fs_decode_step(fs_model* m, fs_kv* kv, const int32_t* seqs,
@@ -674,6 +752,7 @@ fs_status generate_impl(fs_model* m, fs_kv* kv, int32_t seq, const int32_t* prom
   if (derr) {
     cudaMemset(m->err, 0, sizeof(int));
     fs::fused_reset(m);
+    fs::cluster_reset(m);
     return fail(FS_ERR_DEVICE, "a kernel reported device error " + std::to_string(derr));
   }
   *n_out = produced;
@@ -763,7 +842,7 @@ extern "C" fs_status fs_debug_block(fs_model* m, fs_kv* kv, int32_t seq, int32_t
     map.n_list = 1;
     map.seq[0] = seq;
     map.pos[0] = pos0;
-    s = fs::decode_fused(m, kv, map, 1, nullptr, h_in, h_out, layer, layer + 1, false, nullptr,
+    s = fs::decode_persistent(m, kv, map, 1, nullptr, h_in, h_out, layer, layer + 1, false, nullptr,
                          nullptr, st);
     if (s != FS_ERR_UNSUPPORTED) return s;
   }
@@ -811,6 +890,23 @@ extern "C" fs_status fs_debug_wait_limit(fs_model* m, uint64_t wait_ns, int32_t 
   if (withhold_layer < -1 || withhold_layer >= m->s.L)
     return fail(FS_ERR_INVALID, "withhold_layer must be -1 or a layer index");
   fs::fused_debug_wait(m, wait_ns, withhold_layer);
+  fs::cluster_debug_wait(m, wait_ns, withhold_layer);
+  return FS_OK;
+}
+
+extern "C" fs_status fs_debug_decode_path(fs_model* m, int32_t path) {
+  if (!m) return fail(FS_ERR_NULL, "model is NULL");
+  if (path < 0 || path > 2) return fail(FS_ERR_INVALID, "path must be 0, 1 or 2");
+  m->decode_path = path;
+  return FS_OK;
+}
+
+extern "C" fs_status fs_debug_decode_kernel(const fs_model* m, int32_t batch, int32_t* kind) {
+  if (!m || !kind) return fail(FS_ERR_NULL, "model or kind is NULL");
+  if (batch < 1 || batch > fs::kMaxBatch) return fail(FS_ERR_INVALID, "batch out of range");
+  *kind = 0;
+  if (batch <= 4 && m->decode_path != 2)
+    *kind = (m->decode_path == 0 && fs::cluster_eligible(m)) ? 2 : 1;
   return FS_OK;
 }
 

@@ -41,6 +41,8 @@ struct fs_model {
   int prefill_split = 1;
   unsigned long long* trace = nullptr;  // armed fs_debug_trace buffer
   void* extras = nullptr;     // persistent decode kernel state
+  void* cl_extras = nullptr;  // cluster decode kernel state
+  int decode_path = 0;        // fs_debug_decode_path: 0 auto, 1 cooperative kernel, 2 general
   void* tc_extras = nullptr;  // tensor-core prefill state
 };
 
@@ -92,6 +94,22 @@ void fused_debug_wait(fs_model* m, unsigned long long wait_ns, int withhold_laye
 fs_status decode_fused(fs_model* m, const fs_kv* kv, const RowMap& map, int B, const int32_t* tok,
                        const float* h_in, float* h_out, int l0, int l1, bool run_head,
                        float* logits, int32_t* argmax, cudaStream_t stream);
+
+// Cluster decode kernel (decode_cluster.cu): the same calls for the kernel
+// that runs one 16-CTA cluster per kv head (bf16 weights, 1..4 rows).
+fs_status cluster_init(fs_model* m);
+void cluster_release(fs_model* m);
+void cluster_reset(fs_model* m);
+void cluster_debug_wait(fs_model* m, unsigned long long wait_ns, int withhold_layer);
+bool cluster_eligible(const fs_model* m);
+fs_status decode_cluster(fs_model* m, const fs_kv* kv, const RowMap& map, int B,
+                         const int32_t* tok, const float* h_in, float* h_out, int l0, int l1,
+                         bool run_head, float* logits, int32_t* argmax, cudaStream_t stream);
+// The persistent kernel that fs_debug_decode_path selects: the cluster kernel,
+// else the cooperative one; FS_ERR_UNSUPPORTED when neither covers the call.
+fs_status decode_persistent(fs_model* m, const fs_kv* kv, const RowMap& map, int B,
+                            const int32_t* tok, const float* h_in, float* h_out, int l0, int l1,
+                            bool run_head, float* logits, int32_t* argmax, cudaStream_t stream);
 
 // Tensor-core prefill (prefill_tc.cu): available for this model (prepares
 // the fp16 weights on first use), one block on m->h, release.

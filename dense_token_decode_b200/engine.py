@@ -95,6 +95,16 @@ class Model:
                                      _ptr(logits), _ptr(argmax), _stream(stream)),
                   "fs_decode_step")
 
+    def forward_batch(self, kv: "KV", segments, logits=None, argmax=None, stream=None):
+        """fs_forward_batch: ``segments`` is a list of (seq, token list)."""
+        seqs = (C.c_int32 * len(segments))(*[q for q, _ in segments])
+        lens = (C.c_int32 * len(segments))(*[len(t) for _, t in segments])
+        flat = [t for _, ts in segments for t in ts]
+        toks = (C.c_int32 * len(flat))(*flat)
+        abi.check(abi.fs_forward_batch(self.handle, kv.handle, seqs, lens, len(segments),
+                                       C.cast(toks, C.c_void_p), _ptr(logits), _ptr(argmax),
+                                       _stream(stream)), "fs_forward_batch")
+
     def greedy(self, kv: "KV", seq: int, prompt, max_new: int, eos=(), out=None, stream=None):
         """Returns (ids list, stop reason). ``prompt``/``out`` may be host or device."""
         if not isinstance(prompt, torch.Tensor):
@@ -157,6 +167,17 @@ class Model:
     def wait_limit(self, wait_ns: int, withhold_layer: int = -1):
         abi.check(abi.fs_debug_wait_limit(self.handle, wait_ns, withhold_layer),
                   "fs_debug_wait_limit")
+
+    def decode_path(self, path: int):
+        """0 auto (cluster kernel first), 1 cooperative kernel, 2 general sequence."""
+        abi.check(abi.fs_debug_decode_path(self.handle, path), "fs_debug_decode_path")
+
+    def decode_kernel(self, batch: int = 1) -> int:
+        """2 cluster kernel, 1 cooperative kernel, 0 general sequence."""
+        kind = C.c_int32(0)
+        abi.check(abi.fs_debug_decode_kernel(self.handle, batch, C.byref(kind)),
+                  "fs_debug_decode_kernel")
+        return kind.value
 
     def set_prefill_split(self, split: int):
         abi.check(abi.fs_set_prefill_split(self.handle, split), "fs_set_prefill_split")

@@ -19,20 +19,57 @@ import torch
 from . import abi, synth
 from .engine import Model
 
-SLOTS = [(0, "QKV phase begins"), (1, "QKV input complete"), (2, "QKV rows done"),
-         (3, "attention phase begins"), (4, "q/k/v ready"), (5, "attention done"),
-         (6, "O share added"), (7, "MLP phase begins"), (8, "MLP input complete"),
-         (9, "gate/up done"), (10, "down share added")]
+SLOTS = {  # cooperative kernel
+    1: [(0, "QKV phase begins"), (11, "QKV input slice reduced"), (1, "QKV input loaded"),
+        (2, "QKV rows done"), (3, "attention phase begins"), (4, "q/k/v ready"),
+        (13, "attention keys done"), (5, "attention merged"), (6, "O share added"),
+        (7, "MLP phase begins"), (12, "MLP input slice reduced"), (8, "MLP input loaded"),
+        (9, "gate/up done"), (10, "down share added")],
+    # cluster kernel
+    2: [(0, "block begins"), (1, "block input exchanged"), (2, "QKV rows done"),
+        (3, "q/k/v exchanged, normed, rotated"), (4, "keys done, states sent"),
+        (5, "attention merged and exchanged"), (6, "O shares published"),
+        (7, "MLP input exchanged"), (8, "gate/up + SwiGLU done"),
+        (9, "activations exchanged"), (10, "down shares published")],
+}
+HOPS = {
+    1: [("QKV rows -> q/k/v ready", 2, 4, 0), ("O shares -> MLP slice reduced", 6, 12, 0),
+        ("down shares -> next QKV slice reduced", 10, 11, 1)],
+    2: [("O shares -> MLP input exchanged", 6, 7, 0),
+        ("down shares -> next block input exchanged", 10, 1, 1)],
+}
+
+
+def to_us(raw, sms, L):
+    """Per-CTA cycle stamps -> us on a common time base: each CTA's stamps are
+    placed with its own (globaltimer, clock) pairs taken at start and end."""
+    t = raw[: sms * (L + 1)].reshape(sms, L + 1, 16).astype(np.float64)
+    g0, c0, g1, c1 = (t[:, L, i] for i in (12, 13, 14, 15))
+    ghz = (c1 - c0) / np.maximum(g1 - g0, 1.0)  # cycles per ns
+    out = np.full_like(t, np.nan)
+    ok = t > 0
+    for c in range(sms):
+        if ghz[c] <= 0:
+            continue
+        out[c] = (g0[c] + (t[c] - c0[c]) / ghz[c]) / 1000.0
+    out[~ok] = np.nan
+    out[:, L, 12:] = np.nan
+    return out, float(np.median(ghz[ghz > 0]))
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--fmt", default="bf16", choices=["bf16", "q8_0"])
     ap.add_argument("--context", type=int, default=100)
+    ap.add_argument("--path", type=int, default=0, choices=[0, 1],
+                    help="0 the default decode kernel, 1 the cooperative kernel")
     args = ap.parse_args()
     dev = "cuda:0"
     shape = synth.QWEN3_0P6B
     m = Model(shape, synth.model_weights(shape, 1, args.fmt), dev, max_pos=4096)
+    m.decode_path(args.path)
+    kind = m.decode_kernel(1)
+    print("kernel:", {2: "cluster", 1: "cooperative", 0: "general"}[kind])
     n = args.context
     kv = m.kv(1, n + 128)
     prompt = synth.token_ids(8, shape.vocab, seed=1).to(dev)
@@ -47,12 +84,13 @@ def main():
     abi.check(abi.fs_debug_trace(m.handle, buf.data_ptr()), "fs_debug_trace")
     m.decode_step(kv, [0], gen[n:n + 1], None, gen[n + 1:n + 2])
     torch.cuda.synchronize()
-    raw = buf.cpu().numpy().astype(np.float64)
-    t = raw[: sms * (L + 1)].reshape(sms, L + 1, 16)
-    t = np.where(t > 0, t / 1000.0, np.nan)  # us
-    print(f"context {n + 8}; us from the first QKV start of the layer, median of layers 3..{L - 3}")
+    raw = buf.cpu().numpy()
+    t, ghz = to_us(raw, sms, L)
+    print(f"context {n + 8}; SM clock {ghz:.3f} GHz; us from the first QKV start of the layer, "
+          f"median of layers 3..{L - 3}")
     print(f"{'slot':34s} {'first':>7s} {'median':>7s} {'last':>7s}")
-    for k, name in SLOTS:
+    # the tail row's slots 12..15 hold the start / end pairs, not phases
+    for k, name in SLOTS.get(kind, []):
         rows = []
         for l in range(3, L - 2):
             col = t[:, l, k]
@@ -63,6 +101,10 @@ def main():
         if rows:
             a = np.median(np.array(rows), axis=0)
             print(f"{name:34s} {a[0]:7.2f} {a[1]:7.2f} {a[2]:7.2f}")
+    # hand-offs: the last producer of a phase's input to the median consumer
+    for name, k_from, k_to, dl in HOPS.get(kind, []):
+        v = [np.nanmedian(t[:, l + dl, k_to]) - np.nanmax(t[:, l, k_from]) for l in range(3, L - 2)]
+        print(f"hand-off {name:40s} {np.median(v):6.2f} us")
     ends = np.nanmax(t[:, :L, 10], axis=0)
     total = np.nanmax(t[:, L, 4]) - np.nanmin(t[:, 0, 0])
     print(f"layer time (median) {np.median(np.diff(ends)):.2f} us; tail (final norm, LM head, "

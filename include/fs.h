@@ -125,13 +125,20 @@ typedef struct fs_kv fs_kv;
 /* Create a model on the current CUDA device from a config and caller-owned
  * device weights. Validates the config, every pointer (non-NULL, 16-byte
  * aligned device memory) and builds the RoPE cos/sin table on the host in fp64
- * (rounded to fp32). Allocates the library-owned workspace.
+ * (rounded to fp32). Allocates the library-owned workspace. When the
+ * persistent decode kernel covers the shape, it also makes library-owned
+ * transposed copies of every block's wo and wd ([in, out]; Q8_0: codes and
+ * scales), read by the decode kernel in place of the caller's: the weights
+ * must not change after this call.
  * Errors: FS_ERR_NULL, FS_ERR_INVALID, FS_ERR_ALIGN, FS_ERR_UNSUPPORTED,
  * FS_ERR_OOM, FS_ERR_CUDA. On error *out is set to NULL. */
 fs_status fs_model_create(const fs_config* cfg, const fs_weights* weights, fs_model** out);
 
 /* Free library-owned memory of a model (weights are the caller's). NULL is a no-op.
- * The caller must make sure no work using the model is still running. */
+ * The caller must make sure no work using the model is still running.
+ * No page defines teardown; this is the release half of the device buffers
+ * the engine brings up ("Failed Star / fs — Milestones", M5: device, queue,
+ * buffers and pipelines owned by the engine). */
 void fs_model_destroy(fs_model* model);
 
 /* Allocate a paged bf16 KV cache for up to `max_seqs` sequences of up to
@@ -146,17 +153,24 @@ void fs_model_destroy(fs_model* model);
 fs_status fs_kv_alloc(const fs_model* model, int32_t max_seqs, int32_t max_tokens_per_seq,
                       fs_kv** out);
 
-/* Free a KV cache. NULL is a no-op. No work using it may still be running. */
+/* Free a KV cache. NULL is a no-op. No work using it may still be running.
+ * ("Failed Star / fs — Milestones", M4: the cache is memory-only, so it lives
+ * exactly as long as this object; nothing is persisted.) */
 void fs_kv_free(fs_kv* kv);
 
-/* Mark sequence `seq` empty (length 0). Waits for the device to go idle. */
+/* Mark sequence `seq` empty (length 0). Waits for the device to go idle.
+ * ("Failed Star / fs — Milestones", M4: a new generation on the sequence
+ * starts from an empty cache; the pages are reused, not freed.) */
 fs_status fs_kv_reset(fs_kv* kv, int32_t seq);
 
 /* Current length (positions stored) of sequence `seq`, into *len (host). */
 fs_status fs_kv_length(const fs_kv* kv, int32_t seq, int32_t* len);
 
 /* Copy caller K/V into sequence `seq`, layer `layer`, positions
- * [pos0, pos0+n). `k` and `v` are device bf16 arrays in logical layout
+ * [pos0, pos0+n) ("Failed Star / fs — Milestones", M4: cached and uncached
+ * outputs must agree, so a cache state has to be loadable and readable from
+ * outside the forward; import also sets up a long pre-filled context without
+ * running its prefill). `k` and `v` are device bf16 arrays in logical layout
  * [n, n_kv_heads, head_dim] holding stored values (already normalised and
  * rotated). The sequence length becomes max(length, pos0+n) once every layer
  * is imported — the caller states it with fs_kv_set_length.
@@ -164,7 +178,9 @@ fs_status fs_kv_length(const fs_kv* kv, int32_t seq, int32_t* len);
 fs_status fs_kv_import(fs_kv* kv, int32_t seq, int32_t layer, int32_t pos0, int32_t n,
                        const void* k, const void* v, void* stream);
 
-/* The reverse of fs_kv_import: device bf16 [n, n_kv_heads, head_dim] out. */
+/* The reverse of fs_kv_import: device bf16 [n, n_kv_heads, head_dim] out
+ * (the same M4 passage: the stored K/V are compared with an uncached
+ * recompute). Errors: as fs_kv_import. */
 fs_status fs_kv_export(const fs_kv* kv, int32_t seq, int32_t layer, int32_t pos0, int32_t n,
                        void* k, void* v, void* stream);
 
@@ -181,7 +197,10 @@ fs_status fs_kv_set_length(fs_kv* kv, int32_t seq, int32_t len);
 fs_status fs_prefill(fs_model* model, fs_kv* kv, int32_t seq, const int32_t* tokens,
                      int32_t n_tokens, float* logits_out, int32_t* argmax_out, void* stream);
 
-/* Decode one token for each of `batch` distinct sequences: sequence seqs[b]
+/* Decode one token for each of `batch` distinct sequences (ferrite, status
+ * section: forward() run at consecutive positions on the same cache, each
+ * output depending on the context stored so far; "Failed Star / fs —
+ * Milestones", M4: decode does one token of work): sequence seqs[b]
  * (HOST array) takes token tokens[b] at its current length, appends its K/V
  * and gets logits fp32 [batch, V] (device, row b for seqs[b]; may be NULL) and
  * its greedy choice argmax_out[b] (device int32 [batch]; may be NULL).
@@ -191,6 +210,26 @@ fs_status fs_prefill(fs_model* model, fs_kv* kv, int32_t seq, const int32_t* tok
  * FS_ERR_CUDA. */
 fs_status fs_decode_step(fs_model* model, fs_kv* kv, const int32_t* seqs, const int32_t* tokens,
                          int32_t batch, float* logits_out, int32_t* argmax_out, void* stream);
+
+/* One forward over a mixed batch of prefill chunks and decode rows
+ * ("Failed Star / fs — Milestones", M4 KV cache: cached K/V per layer, so a
+ * sequence's new tokens cost one token of work each, whichever call they
+ * arrive in). Segment i appends n_tokens[i] >= 1 ids of sequence seqs[i] at
+ * its current length (a prefill chunk when n_tokens[i] > 1, a decode row when
+ * 1); `seqs` and `n_tokens` are HOST arrays of n_seqs distinct sequences;
+ * `tokens` (host or device int32) holds the segments' ids back to back. Each
+ * row attends to its own sequence's cache and the rows before it in its
+ * segment. Writes the logits of each segment's LAST row to `logits_out`
+ * (device fp32 [n_seqs, vocab], row i for segment i; may be NULL) and their
+ * greedy ids to `argmax_out` (device int32 [n_seqs]; may be NULL). Runs the
+ * general (any rows) kernels. A debug capture armed for this call holds the
+ * rows in processing order: every segment's rows but the last, segment by
+ * segment, then the segments' last rows. 1 <= sum of n_tokens <= 64.
+ * Errors: FS_ERR_NULL, FS_ERR_EMPTY, FS_ERR_SEQ, FS_ERR_CONTEXT,
+ * FS_ERR_INVALID, FS_ERR_TOKEN, FS_ERR_ALIGN, FS_ERR_CUDA. */
+fs_status fs_forward_batch(fs_model* model, fs_kv* kv, const int32_t* seqs,
+                           const int32_t* n_tokens, int32_t n_seqs, const int32_t* tokens,
+                           float* logits_out, int32_t* argmax_out, void* stream);
 
 /* Greedy continuation of `prompt` (n_prompt ids, host or device) on sequence
  * `seq`, following "Coming back to Failed Star", "Next: one complete
@@ -258,14 +297,17 @@ fs_status fs_debug_block(fs_model* model, fs_kv* kv, int32_t seq, int32_t layer,
                          const float* h_in, int32_t rows, float* h_out, void* stream);
 
 /* Debug: the next decode step that runs on the persistent decode kernel
- * records %globaltimer stamps (ns) into `buf` (device uint64
- * [SMs][n_layers+1][16]): per CTA and block, slot 0 start of the QKV phase,
- * 1 its input (the residual) complete, 2 QKV rows done, 3 start of the
- * attention phase, 4 q/k/v of the first batch row ready, 5 attention done,
- * 6 O-projection share added, 7 start of the MLP phase, 8 its input
- * complete, 9 gate/up rows done, 10 down share added; row n_layers holds the
- * tail (0 start, 1 input complete, 2 LM-head rows done, 3 the producer's last
- * copy issued, 4 greedy ids folded). Slots a CTA never reaches are left as
+ * records timestamps into `buf` (device uint64 [SMs][n_layers+1][16]): per
+ * CTA and block the SM's cycle counter (clock64) at slot 0 start of the QKV
+ * phase, 11 this CTA's slice of its input reduced, 1 its input loaded, 2 QKV rows done,
+ * 3 start of the attention phase, 4 q/k/v of the first batch row ready, 13
+ * its keys done, 5 attention merged, 6 O-projection share added, 7 start of
+ * the MLP phase, 12 this CTA's slice of its input reduced, 8 its input loaded, 9 gate/up
+ * rows done, 10 down share added. Row n_layers holds the tail (0 start, 11
+ * slice of its input reduced, 1 input loaded, 2 LM-head rows done, 3 the producer's
+ * last copy issued, 4 greedy ids folded) and the CTA's %globaltimer (ns) and
+ * cycle counter at kernel start (12, 13) and end (14, 15), which place the
+ * cycle stamps on a common time base. Slots a CTA never reaches are left as
  * they were. One-shot; NULL disarms. Timing only: no work changes. */
 fs_status fs_debug_trace(fs_model* model, uint64_t* buf);
 
@@ -275,11 +317,26 @@ fs_status fs_debug_trace(fs_model* model, uint64_t* buf);
  * the kernel stops waiting everywhere, returns, and sets the device error
  * word to 3 (fs_device_error, which also clears the kernel's exchange state;
  * fs_greedy reports FS_ERR_DEVICE). `withhold_layer` >= 0 makes the next
- * step on that kernel never publish block `withhold_layer`'s Q/K/V
- * projections, so the waits for them run out (a test of that path; the step's
- * outputs are then undefined); -1 withholds nothing.
- * Errors: FS_ERR_NULL, FS_ERR_INVALID. */
+ * step on that kernel never publish one of block `withhold_layer`'s hand-offs
+ * between CTAs (the cooperative kernel: its Q/K/V projections; the cluster
+ * kernel: its output-projection shares), so the waits for them run out (a
+ * test of that path; the step's outputs are then undefined); -1 withholds
+ * nothing. Errors: FS_ERR_NULL, FS_ERR_INVALID. */
 fs_status fs_debug_wait_limit(fs_model* model, uint64_t wait_ns, int32_t withhold_layer);
+
+/* Debug: which decode path later steps of 1..4 rows take. 0 (default): the
+ * cluster kernel (one 16-CTA cluster per kv head; bf16 weights, on shapes and
+ * devices it covers), else the cooperative persistent kernel, else the
+ * general kernel sequence; 1: the cooperative kernel, else general; 2: the
+ * general sequence only. For comparing the paths in tests and benchmarks;
+ * every path computes the same forward. Errors: FS_ERR_NULL, FS_ERR_INVALID. */
+fs_status fs_debug_decode_path(fs_model* model, int32_t path);
+
+/* Debug: the kernel a decode step of `batch` rows would use under the current
+ * path: *kind = 2 the cluster kernel, 1 the cooperative kernel (if it covers
+ * the shape; else the general sequence runs), 0 the general sequence.
+ * Errors: FS_ERR_NULL, FS_ERR_INVALID. */
+fs_status fs_debug_decode_kernel(const fs_model* model, int32_t batch, int32_t* kind);
 
 /* Debug: dequantise Q8_0 blocks to fp32, out[n*k] = codes[n*k] * scales[n*(k/32)]
  * (all device, row-major). Bit-exact by construction. k % 32 == 0. */
@@ -322,9 +379,11 @@ fs_status fs_set_prefill_split(fs_model* model, int32_t split);
  * exits. A call needs rows*hidden*4 (rounded up to 256) + rows*4*SMs*8 bytes
  * of it (148 SMs: 16 rows of hidden 1024 fit, 64 rows do not); larger calls
  * are rejected with FS_ERR_INVALID before anything runs.
- * The first call on a device looks up the array's device address (a one-time
- * set-up per device, done with that device current); make that first call
- * before any stream capture. All calls share the one array: two calls whose
+ * Each call made outside a stream capture looks up the array's device
+ * address afresh (so it stays right after cudaDeviceReset); a call captured
+ * into a graph uses the address of the last uncaptured call on that device,
+ * so make one uncaptured call (after any reset) before capturing. All calls
+ * share the one array: two calls whose
  * work overlaps on the GPU (different streams, or different host threads on
  * one device) race on it and may return wrong results; serialise them.
  * Requirements: hidden % 64 == 0, 1 <= rows <= 64, rms_eps > 0, pointers

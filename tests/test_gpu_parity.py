@@ -658,3 +658,45 @@ def test_decode_wait_timeout_is_reported_and_recovers(tiny):
     rl = tiny.oracle.forward([5], cache)[0]
     assert_logits_close(oracle_tensor(logits), rl, what="step after a timeout")
     check_greedy_step(int(am.item()), oracle_tensor(logits), rl)
+
+
+def test_tiny_mixed_prefill_and_decode_batch(tiny):
+    """One fs_forward_batch call with a fresh 20-token prefill chunk, a decode
+    row, a 7-token chunk onto a 60-position sequence (crossing the page
+    boundary at 64) and a decode row at position 1: per segment the last-row
+    logits and greedy id, the appended K/V and the per-block hidden states of
+    every row against the oracle."""
+    m, s = tiny.model, tiny.shape
+    kv = m.kv(4, 128)
+    hist = {1: synth.token_ids(37, s.vocab, seed=81).tolist(),
+            2: synth.token_ids(60, s.vocab, seed=82).tolist(),
+            3: synth.token_ids(1, s.vocab, seed=83).tolist()}
+    caches = {0: None}
+    for q, toks in hist.items():
+        m.prefill(kv, q, _dev_i32(toks))
+        caches[q] = tiny.oracle.forward(toks)[2]
+    segs = [(0, synth.token_ids(20, s.vocab, seed=84).tolist()), (1, [123]),
+            (2, synth.token_ids(7, s.vocab, seed=85).tolist()), (3, [4000])]
+    rows = sum(len(t) for _, t in segs)
+    hidden = torch.zeros((s.n_layers + 1, rows, s.hidden), device=DEV)
+    logits = torch.empty((len(segs), s.vocab), device=DEV)
+    am = torch.empty(len(segs), dtype=torch.int32, device=DEV)
+    m.capture(hidden, rows)
+    m.forward_batch(kv, segs, logits, am)
+    torch.cuda.synchronize()
+    gh = oracle_tensor(hidden)
+    # processing order: all rows but each segment's last, then the last rows
+    order = [(i, t) for i, (_, ts) in enumerate(segs) for t in range(len(ts) - 1)]
+    order += [(i, len(ts) - 1) for i, (_, ts) in enumerate(segs)]
+    for i, (q, toks) in enumerate(segs):
+        rl, rh, cache = tiny.oracle.forward(toks, caches[q])
+        assert_logits_close(oracle_tensor(logits[i]), rl, what=f"mixed batch segment {i}")
+        check_greedy_step(int(am[i]), oracle_tensor(logits[i]), rl)
+        got = np.stack([gh[:, order.index((i, t))] for t in range(len(toks))], axis=1)
+        assert_blocks_close(got, rh, tol=E2E_BLOCK_REL_L2, what=f"mixed batch segment {i}")
+        n = len(hist.get(q, [])) + len(toks)
+        assert kv.length(q) == n
+        for l in range(s.n_layers):
+            k, v = kv.export(q, l, 0, n)
+            assert rel_l2(oracle_tensor(k), cache.k[l]) <= BLOCK_REL_L2
+            assert rel_l2(oracle_tensor(v), cache.v[l]) <= BLOCK_REL_L2
