@@ -57,7 +57,7 @@
 namespace fs {
 namespace clus {
 
-constexpr int kCS = 16;  // CTAs per cluster
+constexpr int kMaxCS = 16;  // CTAs per cluster (16, or 8 where 16-CTA clusters do not all fit)
 constexpr int kConsumerWarps = 11;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;  // + producer warp
@@ -65,12 +65,28 @@ constexpr int kMaxB = 4;
 constexpr int kStage = 17408;  // ring stage: 16 Q8_0 rows of K = 1024 with their scales
 constexpr int kMaxStages = 14;
 constexpr int kTraceSlots = 16;
-constexpr int kMaxRows = 64;   // rows of one tensor-core pass
+constexpr int kMaxRows = 128;  // rows of one tensor-core pass
 constexpr int kMaxH = 1024;
+
+// How the work of a block is split. Clusters: `split` per kv head, each
+// taking rep / split of the head's query heads (and the head's k and v
+// rows, so with split > 1 the k and v projections run in every cluster of
+// the head); CTAs: `cs` per cluster.
+struct Geo {
+  int cs, split, ncl, repc;
+  int nA;      // QKV rows per CTA: (repc + 2) d / cs
+  int nO;      // O and down rows per CTA: H / cs
+  int nc;      // intermediate columns per CTA: I / (ncl cs)
+  int Kc;      // intermediate columns per cluster (the down product's K): I / ncl
+  int RDc;     // attention outputs per cluster: repc d (the O product's K)
+  int F;       // attention outputs merged by one CTA: RDc / cs
+  int n[4], K[4];  // rows and K of the four weight phases
+};
 
 struct Params {
   int L, H, nq, nkv, d, I, V;
   float eps;
+  Geo geo;
   const LayerDev* layers;
   const __nv_bfloat16* embed;
   const __nv_bfloat16* final_norm;
@@ -80,8 +96,8 @@ struct Params {
   int seq[kMaxB];
   int pos[kMaxB];
   const int32_t* tokens;
-  unsigned long long* po;  // [n_kv][kMaxB][H] O-projection shares (tagged)
-  unsigned long long* pd;  // [n_kv][kMaxB][H] down-projection shares (tagged)
+  unsigned long long* po;  // [clusters][kMaxB][H] O-projection shares (tagged)
+  unsigned long long* pd;  // [clusters][kMaxB][H] down-projection shares (tagged)
   uint32_t tag0;
   int l0, l1;
   const float* h_in;
@@ -102,7 +118,7 @@ struct Params {
   int lm_owners, lm_rows;
   int bt_in_smem;
   int q8;
-  const unsigned char* packed;  // [L][n_kv][16] per-CTA weight images of stream_bytes each
+  const unsigned char* packed;  // [L][clusters][cs] per-CTA weight images of stream_bytes each
   int stream_bytes;
   int pofs[4];                  // offsets of the four phases in an image
   // shared-memory carve-up (byte offsets)
@@ -199,6 +215,20 @@ __device__ __forceinline__ bool consumer_sync_or(bool v) {
 }
 __device__ __forceinline__ bool aborted(const int* flag) {
   return *reinterpret_cast<const volatile int*>(flag) != 0;
+}
+// Whether a wait first stamped at t0 (0: stamp it now) must stop: it ran
+// past `limit`, or, once it has lasted 20 us, another CTA raised the abort
+// flag. Only waits that already took long read the one shared flag, so the
+// many short waits of a step do not all poll the same word.
+__device__ __forceinline__ bool wait_expired(unsigned long long& t0, unsigned long long limit,
+                                             const int* abort_flag) {
+  const unsigned long long t = now_ns();
+  if (t0 == 0) {
+    t0 = t;
+    return false;
+  }
+  const unsigned long long dt = t - t0;
+  return dt > 20000ull && (dt > limit || aborted(abort_flag));
 }
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -337,22 +367,32 @@ __device__ __forceinline__ size_t kv_off(const Params& p, int layer, int b, int 
          (((size_t)page * p.kv.n_kv_heads + g) * kPage + (pos % kPage)) * p.kv.head_dim;
 }
 
-// Row counts of one CTA (rank r of the cluster of kv head g).
-__host__ __device__ inline int rows_qkv(int rep, int d) { return (rep + 2) * d / kCS; }
-__host__ __device__ inline int rows_out(int H) { return H / kCS; }
-__host__ __device__ inline int cols_mlp(int I, int nkv) { return I / (nkv * kCS); }
-// Rows and K of each phase (the same for every CTA).
-__host__ __device__ inline void phase_geometry(int H, int nq, int nkv, int d, int I, int (&n)[4],
-                                               int (&K)[4]) {
-  const int rep = nq / nkv;
-  n[kPA] = rows_qkv(rep, d);
-  K[kPA] = H;
-  n[kPO] = rows_out(H);
-  K[kPO] = rep * d;
-  n[kPGU] = 2 * cols_mlp(I, nkv);
-  K[kPGU] = H;
-  n[kPD] = rows_out(H);
-  K[kPD] = I / nkv;
+__host__ __device__ inline Geo make_geo(int H, int nq, int nkv, int d, int I, int cs, int split) {
+  Geo g{};
+  g.cs = cs;
+  g.split = split;
+  g.ncl = nkv * split;
+  g.repc = nq / nkv / split;
+  g.nA = (g.repc + 2) * d / cs;
+  g.nO = H / cs;
+  g.nc = I / (g.ncl * cs);
+  g.Kc = I / g.ncl;
+  g.RDc = g.repc * d;
+  g.F = g.RDc / cs;
+  g.n[kPA] = g.nA;
+  g.K[kPA] = H;
+  g.n[kPO] = g.nO;
+  g.K[kPO] = g.RDc;
+  g.n[kPGU] = 2 * g.nc;
+  g.K[kPGU] = H;
+  g.n[kPD] = g.nO;
+  g.K[kPD] = g.Kc;
+  return g;
+}
+// The 16-byte unit u of packed row j sits at unit u ^ (j mod 8), within each
+// whole group of 8 units (a row's last partial group stays in place).
+__host__ __device__ inline int swz(int u, int j, int units) {
+  return (u | 7) < units ? (u ^ (j & 7)) : u;
 }
 
 // ---------------------------------------------------------------------------
@@ -376,8 +416,7 @@ struct Producer {
     int spins = 0;
     while (!mbar_test(&r.empty[s], parity)) {
       if ((++spins & 15) == 0) {
-        if (t0 == 0) t0 = now_ns();
-        if (aborted(p.abort_flag) || now_ns() - t0 > p.wait_ns) {
+        if (wait_expired(t0, p.wait_ns, p.abort_flag)) {
           if (!aborted(p.abort_flag)) {
             atomicExch(p.abort_flag, 1);
             atomicCAS(p.err, 0, kErrTimeout);
@@ -412,17 +451,16 @@ struct Producer {
     }
   }
 
-  __device__ void layer(int l, int g, int rk) {
-    int n[4], K[4];
-    phase_geometry(p.H, p.nq, p.nkv, p.d, p.I, n, K);
+  __device__ void layer(int l, int c, int g, int rk) {
+    const Geo& G = p.geo;
     const unsigned char* img =
-        p.packed + ((size_t)(l * p.nkv + g) * kCS + rk) * (size_t)p.stream_bytes;
-    weights(img + p.pofs[kPA], n[kPA], K[kPA]);
+        p.packed + ((size_t)(l * G.ncl + c) * G.cs + rk) * (size_t)p.stream_bytes;
+    weights(img + p.pofs[kPA], G.n[kPA], G.K[kPA]);
     // B: the CTA's key range of each batch row, K then V per page segment
     const int d = p.d;
     for (int b = 0; b < p.B && !quit; ++b) {
       int k0, k1;
-      slice(p.pos[b], kCS, rk, k0, k1);
+      slice(p.pos[b], G.cs, rk, k0, k1);
       for (int j0 = k0; j0 < k1 && !quit;) {
         const int je = min(k1, (j0 / kPage + 1) * kPage), nk = je - j0;
         const size_t off = kv_off(p, l, b, j0, g);
@@ -437,9 +475,9 @@ struct Producer {
         j0 = je;
       }
     }
-    weights(img + p.pofs[kPO], n[kPO], K[kPO]);
-    weights(img + p.pofs[kPGU], n[kPGU], K[kPGU]);
-    weights(img + p.pofs[kPD], n[kPD], K[kPD]);
+    weights(img + p.pofs[kPO], G.n[kPO], G.K[kPO]);
+    weights(img + p.pofs[kPGU], G.n[kPGU], G.K[kPGU]);
+    weights(img + p.pofs[kPD], G.n[kPD], G.K[kPD]);
   }
 
   // LM head: runs of lm_rows whole embedding rows, one bulk copy each.
@@ -470,7 +508,7 @@ struct Consumer {
   uint32_t parity = 0;
   bool quit = false;
   unsigned int xk = 0;  // exchanges done
-  int tid, warp, lane, cta, g, rk, G;
+  int tid, warp, lane, cta, cl, g, hs, rk, G;
   float inv[NB];
   unsigned long long wbest[kMaxB] = {0ull, 0ull, 0ull, 0ull};
   static constexpr int kEPT = (NB * kMaxH + kConsumers - 1) / kConsumers;
@@ -482,7 +520,9 @@ struct Consumer {
     cta = blockIdx.x;
     G = gridDim.x;
     rk = (int)cluster_rank();
-    g = cta / kCS;
+    cl = cta / p.geo.cs;      // cluster
+    g = cl / p.geo.split;     // its kv head
+    hs = cl % p.geo.split;    // its share of the head's query heads
   }
 
   // ---- shared-memory regions ---------------------------------------------
@@ -491,29 +531,31 @@ struct Consumer {
   __device__ __nv_bfloat16* zt() { return reinterpret_cast<__nv_bfloat16*>(sm + p.off_zt); }
   __device__ int zt_stride() const { return p.H + 8; }  // [2B][H + 8]: hi, lo rows of each batch row
   __device__ __nv_bfloat16* zo() { return reinterpret_cast<__nv_bfloat16*>(sm + p.off_zo); }
-  __device__ int zo_stride() const { return (p.nq / p.nkv) * p.d + 8; }
+  __device__ int zo_stride() const { return p.geo.RDc + 8; }
   __device__ __nv_bfloat16* za() { return reinterpret_cast<__nv_bfloat16*>(sm + p.off_za); }
-  __device__ int za_stride() const { return p.I / p.nkv + 8; }
-  __device__ float* raw() { return reinterpret_cast<float*>(sm + p.off_raw); }  // [B][(rep+2)d]
-  __device__ float* qs() { return reinterpret_cast<float*>(sm + p.off_q); }     // [B][rep][d]
+  __device__ int za_stride() const { return p.geo.Kc + 8; }
+  __device__ float* raw() { return reinterpret_cast<float*>(sm + p.off_raw); }  // [B][(repc+2)d]
+  __device__ float* qs() { return reinterpret_cast<float*>(sm + p.off_q); }     // [B][repc][d]
   __device__ __nv_bfloat16* kcur() { return reinterpret_cast<__nv_bfloat16*>(sm + p.off_kv); }
   __device__ __nv_bfloat16* vcur() { return kcur() + kMaxB * p.d; }
-  __device__ float* att() { return reinterpret_cast<float*>(sm + p.off_att); }  // [16][B][2 + F]
+  __device__ float* att() { return reinterpret_cast<float*>(sm + p.off_att); }  // [cs][kMaxB][2 + F]
   __device__ float* cmb() { return reinterpret_cast<float*>(sm + p.off_cmb); }  // [B][F]
   __device__ float* act() { return reinterpret_cast<float*>(sm + p.off_act); }  // [B][nc]
   __device__ float* ssc() { return reinterpret_cast<float*>(sm + p.off_ssc); }  // [rep][64] + run state
-  __device__ float* ys() { return reinterpret_cast<float*>(sm + p.off_ys); }    // [64][4]
+  __device__ float* ys() { return reinterpret_cast<float*>(sm + p.off_ys); }    // [128][4]
   __device__ float* red() { return reinterpret_cast<float*>(sm + p.off_red); }
   __device__ float* ssp() { return reinterpret_cast<float*>(sm + p.off_ss); }   // [11][kMaxB]
-  // [64] shared address of each row of a phase's product (| row mod 8: its swizzle)
-  __device__ uint32_t* rowaddr() { return reinterpret_cast<uint32_t*>(sm + p.off_misc); }
-  // [64] Q8_0: shared address of each row's scales
-  __device__ uint32_t* scaleaddr() { return reinterpret_cast<uint32_t*>(sm + p.off_misc + 512); }
-  __device__ uint32_t zero_addr() { return su32(sm + p.off_misc + 256); }  // 64 zero bytes
+  // misc (bytes): zero bytes 0..64, greedy keys 64..96, flag 96, counts 104,
+  // the row tables from 128.
+  __device__ uint32_t zero_addr() { return su32(sm + p.off_misc); }  // 64 zero bytes
   __device__ unsigned long long* best() {
-    return reinterpret_cast<unsigned long long*>(sm + p.off_misc + 320);
+    return reinterpret_cast<unsigned long long*>(sm + p.off_misc + 64);
   }
-  __device__ int* flag() { return reinterpret_cast<int*>(sm + p.off_misc + 352); }
+  __device__ int* flag() { return reinterpret_cast<int*>(sm + p.off_misc + 96); }
+  // [128] shared address of each row of a phase's product (| row mod 8: its swizzle)
+  __device__ uint32_t* rowaddr() { return reinterpret_cast<uint32_t*>(sm + p.off_misc + 128); }
+  // [128] Q8_0: shared address of each row's scales
+  __device__ uint32_t* scaleaddr() { return reinterpret_cast<uint32_t*>(sm + p.off_misc + 640); }
   __device__ uint64_t* xbar() { return r.empty + kMaxStages; }  // [2] exchange barriers
 
   // ---- ring --------------------------------------------------------------
@@ -529,6 +571,10 @@ struct Consumer {
     }
     quit = true;
   }
+  // `quit` of any lane of this warp: the guard of warp-collective work
+  // (shuffles, ldmatrix, mma), which every lane must execute or skip
+  // together; per-thread quit alone may differ between lanes.
+  __device__ __forceinline__ bool warp_quit() const { return __any_sync(0xffffffffu, quit); }
   // Wait (whole warp) for the chunk `ahead` places after the oldest one this
   // warp has not released (every chunk before it waited for by this warp).
   __device__ __noinline__ const unsigned char* chunk_wait(int ahead = 0) {
@@ -546,8 +592,7 @@ struct Consumer {
       if ((++spins & 15) == 0) {
         int bad = 0;
         if (lane == 0) {
-          if (t0 == 0) t0 = now_ns();
-          bad = aborted(p.abort_flag) || now_ns() - t0 > p.wait_ns;
+          bad = wait_expired(t0, p.wait_ns, p.abort_flag);
         }
         if (__shfl_sync(0xffffffffu, bad, 0)) give_up();
       }
@@ -581,8 +626,7 @@ struct Consumer {
       if ((++spins & 15) == 0) {
         int bad = 0;
         if (lane == 0) {
-          if (t0 == 0) t0 = now_ns();
-          bad = aborted(p.abort_flag) || now_ns() - t0 > p.wait_ns;
+          bad = wait_expired(t0, p.wait_ns, p.abort_flag);
         }
         if (__shfl_sync(0xffffffffu, bad, 0)) give_up();
       }
@@ -609,12 +653,7 @@ struct Consumer {
     while (!mbar_test_cluster(bar, par)) {
       if (quit) break;
       if ((++spins & 15) == 0) {
-        bool stop = aborted(p.abort_flag);
-        if (!stop) {
-          if (t0 == 0) t0 = now_ns();
-          stop = now_ns() - t0 > p.wait_ns;
-        }
-        if (stop) {
+        if (wait_expired(t0, p.wait_ns, p.abort_flag)) {
           give_up();
           break;
         }
@@ -632,13 +671,8 @@ struct Consumer {
     do {
       __nanosleep(20);
       x = ld_word(w);
-      if ((++spins & 7) == 0) {
-        bool stop = aborted(p.abort_flag);
-        if (!stop && (spins & 63) == 0) {
-          if (t0 == 0) t0 = now_ns();
-          stop = now_ns() - t0 > p.wait_ns;
-        }
-        if (stop) {
+      if ((++spins & 15) == 0) {
+        if (wait_expired(t0, p.wait_ns, p.abort_flag)) {
           give_up();
           break;
         }
@@ -658,7 +692,7 @@ struct Consumer {
   // Ends with the exchange complete.
   __device__ __noinline__ void exchange_sum(const unsigned long long* src, uint32_t tag,
                                             const float* base, float* dst) {
-    const int H = p.H, E = H / kCS, e0 = rk * E, n = p.B * E, total = p.nkv * n;
+    const int H = p.H, E = H / p.geo.cs, e0 = rk * E, n = p.B * E, total = p.geo.ncl * n;
     float* buf = red();
     float* sums = buf + total;
     for (int f0 = tid; f0 < total; f0 += 4 * kConsumers) {
@@ -678,14 +712,14 @@ struct Consumer {
       }
     }
     consumer_sync();
-    if (tid < n) {
+    for (int v = tid; v < n; v += kConsumers) {
       float s = 0.f;
-      for (int c = 0; c < p.nkv; ++c) s += buf[c * n + tid];
-      sums[tid] = base[(tid / E) * H + e0 + tid % E] + s;
+      for (int c = 0; c < p.geo.ncl; ++c) s += buf[c * n + v];
+      sums[v] = base[(v / E) * H + e0 + v % E] + s;
     }
     consumer_sync();
     xarm((uint32_t)(p.B * H * 4));
-    for (int w = tid; w < n * kCS; w += kConsumers) {
+    for (int w = tid; w < n * p.geo.cs; w += kConsumers) {
       const int dest = w / n, v = w % n;
       xsend(dst + (v / E) * H + e0 + v % E, dest, __float_as_uint(sums[v]));
     }
@@ -756,21 +790,21 @@ struct Consumer {
     return v;
   }
 
-  // ys[j * 4 + b] = sum_k W[j][k] x_b[k] for the R rows (R <= 64) of a phase,
-  // K a multiple of 128, row j's data at rowaddr()[j] (16-byte units stored
-  // at u ^ (j mod 8)): A = the rows (16-row tiles), B = the 2B operand rows at
-  // `ob` (stride `ostride` bytes): column 2b + t of the product is term t of
-  // batch row b. Work items are (row tile, block of 128 columns), warp w
-  // taking items w, w + 11, ...; the items' partial sums are added in a fixed
-  // order. Ends on a barrier.
-  __device__ __noinline__ void mma_rows(int R, int K, uint32_t ob, uint32_t ostride) {
+  // ys[j * 4 + b] = sum_k W[j][k] x_b[k] for the R rows (R <= 128) of a
+  // phase, K a multiple of 64, row j's data at rowaddr()[j] (16-byte units
+  // stored as swz() places them): A = the rows (16-row tiles), B = the 2B
+  // operand rows at `ob` (stride `ostride` bytes): column 2b + t of the
+  // product is term t of batch row b. Work items are (row tile, block of 64
+  // columns), warp w taking items w, w + 11, ...; the items' partial sums are
+  // added in a fixed order. Ends on a barrier.
+  __device__ __noinline__ void mma_rows(int R, int K, uint32_t ob, uint32_t ostride, int y0) {
     const uint32_t* ra = rowaddr();
     float* part = red();
-    const int nkb = K / 128, mt = (R + 15) / 16, items = mt * nkb, twoB = 2 * p.B;
+    const int nkb = K / 64, mt = (R + 15) / 16, items = mt * nkb, twoB = 2 * p.B;
     const uint32_t zero = zero_addr();
     const int gq = lane >> 2, q = lane & 3;
     for (int it = warp; it < items; it += kConsumerWarps) {
-      const int m = it / nkb, kb0 = (it % nkb) * 8;
+      const int m = it / nkb, kb0 = (it % nkb) * 4;  // first k-step of the item
       float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
       if constexpr (!Q8) {
         const int row = m * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
@@ -781,7 +815,7 @@ struct Consumer {
         uint32_t baddr = brow ? ob + n * ostride + (((lane >> 3) & 1) << 4) + kb0 * 32 : zero;
         const uint32_t bstep = brow ? 32u : 0u;
 #pragma unroll
-        for (int ks = 0; ks < 8; ks += 2) {
+        for (int ks = 0; ks < 4; ks += 2) {
           const uint32_t u = (uint32_t)((kb0 + ks) * 2 + (lane >> 4));
           uint32_t a[4], b[2], a2[4], b2[2];
           ldsm_x4(arow ? rb + ((u ^ sw) << 4) : zero, a);
@@ -793,7 +827,7 @@ struct Consumer {
           baddr += 2 * bstep;
         }
       } else {
-        // Q8_0: 4 blocks of 32 columns; each thread takes 8 consecutive codes
+        // Q8_0: 2 blocks of 32 columns; each thread takes 8 consecutive codes
         // of rows gq and gq + 8 (columns 32 blk + 8 q ..) and the same 8
         // operand columns, a column order that both operands share. Each
         // block's product is scaled by its rows' scales.
@@ -801,14 +835,15 @@ struct Consumer {
         const bool h0 = r0 < R, h1 = r1 < R, hb = gq < twoB;
         const uint32_t v0 = h0 ? ra[r0] : 0u, v1 = h1 ? ra[r1] : 0u;
         const uint32_t s0a = h0 ? scaleaddr()[r0] : 0u, s1a = h1 ? scaleaddr()[r1] : 0u;
-        const uint32_t sw = (uint32_t)gq;  // rows r0 and r1 are both gq mod 8
+        const int units = K / 16;  // rows r0 and r1 are both gq mod 8
         const uint32_t bb = ob + gq * ostride;
 #pragma unroll
-        for (int bi = 0; bi < 4; ++bi) {
+        for (int bi = 0; bi < 2; ++bi) {
           const int blk = kb0 / 2 + bi;
-          const uint32_t u = (uint32_t)(blk * 2 + (q >> 1)), half = (uint32_t)(q & 1) * 8u;
-          const uint2 c0 = h0 ? lds64((v0 & ~15u) + ((u ^ sw) << 4) + half) : make_uint2(0u, 0u);
-          const uint2 c1 = h1 ? lds64((v1 & ~15u) + ((u ^ sw) << 4) + half) : make_uint2(0u, 0u);
+          const uint32_t u = (uint32_t)swz(blk * 2 + (q >> 1), gq, units);
+          const uint32_t half = (uint32_t)(q & 1) * 8u;
+          const uint2 c0 = h0 ? lds64((v0 & ~15u) + (u << 4) + half) : make_uint2(0u, 0u);
+          const uint2 c1 = h1 ? lds64((v1 & ~15u) + (u << 4) + half) : make_uint2(0u, 0u);
           const uint4 z = hb ? lds128(bb + (uint32_t)(blk * 64 + q * 16)) : make_uint4(0u, 0u, 0u, 0u);
           const uint32_t a0[4] = {i8x2_bf16(c0.x, 0), i8x2_bf16(c1.x, 0), i8x2_bf16(c0.x, 1),
                                   i8x2_bf16(c1.x, 1)};
@@ -830,7 +865,7 @@ struct Consumer {
       part[(it * 16 + gq + 8) * 4 + q] = (d0[2] + d1[2]) + (d0[3] + d1[3]);
     }
     consumer_sync();
-    float* y = ys();
+    float* y = ys() + y0 * 4;
     for (int t = tid; t < R * 4; t += kConsumers) {
       const int rr = (t >> 2) & 15, q2 = t & 3, m = t >> 6;
       float sum = 0.f;
@@ -840,25 +875,27 @@ struct Consumer {
     consumer_sync();
   }
 
-  // The rows of phase `ph` (spread over the next chunks): waits for them,
-  // fills the row tables and runs the product; the chunks are released
-  // after it.
+  // The rows of phase `ph` (spread over the next chunks) into ys: in passes
+  // of as many chunks as the ring holds, each pass waiting for its chunks,
+  // filling the row tables, running the product of its rows and releasing
+  // the chunks.
   __device__ void rows_product(int ph, uint32_t ob, uint32_t ostride) {
-    int n[4], K[4];
-    phase_geometry(p.H, p.nq, p.nkv, p.d, p.I, n, K);
-    const int R = n[ph], Kp = K[ph], cap = cap_rows(Kp, Q8), nch = (R + cap - 1) / cap;
-    const int rb = Q8 ? Kp : 2 * Kp;
-    for (int c = 0; c < nch; ++c) chunk_wait(c);
-    if (warp == 0)
-      for (int j = lane; j < R; j += 32) {
-        const int c = j / cap, slot = j - c * cap;
-        const uint32_t st = stage_addr(c);
-        rowaddr()[j] = (st + slot * rb) | (uint32_t)(j & 7);
-        if (Q8) scaleaddr()[j] = st + min(cap, R - c * cap) * Kp + slot * (Kp / 16);
-      }
-    consumer_sync();
-    mma_rows(R, Kp, ob, ostride);
-    for (int c = 0; c < nch; ++c) chunk_release();
+    const int R = p.geo.n[ph], Kp = p.geo.K[ph], cap = cap_rows(Kp, Q8), nch = (R + cap - 1) / cap;
+    const int rb = Q8 ? Kp : 2 * Kp, pass = min(nch, r.n);
+    for (int c0 = 0; c0 < nch; c0 += pass) {
+      const int np = min(pass, nch - c0), j0 = c0 * cap, rows = min(R, (c0 + np) * cap) - j0;
+      for (int c = 0; c < np; ++c) chunk_wait(c);
+      if (warp == 0)
+        for (int jj = lane; jj < rows; jj += 32) {
+          const int j = j0 + jj, c = j / cap, slot = j - c * cap;  // chunk and row slot
+          const uint32_t st = stage_addr(c - c0);
+          rowaddr()[jj] = (st + slot * rb) | (uint32_t)(j & 7);
+          if (Q8) scaleaddr()[jj] = st + min(cap, R - c * cap) * Kp + slot * (Kp / 16);
+        }
+      consumer_sync();
+      mma_rows(rows, Kp, ob, ostride, j0);
+      for (int c = 0; c < np; ++c) chunk_release();
+    }
   }
 
   __device__ __noinline__ void tr(int layer, int k) {
@@ -900,7 +937,8 @@ struct Consumer {
   // cache. Ends on a barrier.
   __device__ __noinline__ void prep_heads(int l) {
     const LayerDev& Lw = layer_s(p, l);
-    const int d = p.d, rep = p.nq / p.nkv, nroles = rep + 2, rowlen = nroles * d;
+    const int d = p.d, rep = p.geo.repc, nroles = rep + 2, rowlen = nroles * d;
+    const bool owner = rk == 0 && hs == 0;  // appends the head's k and v
     float* tmp = ssc();  // [11][128] scratch of the k rows
     for (int u = warp; u < p.B * nroles; u += kConsumerWarps) {
       const int b = u / nroles, role = u % nroles, pos = p.pos[b];
@@ -915,14 +953,14 @@ struct Consumer {
         for (int i2 = lane; i2 < d; i2 += 32) {
           const __nv_bfloat16 kb = __float2bfloat16_rn(kt[i2]);
           kcur()[b * d + i2] = kb;
-          if (rk == 0 && !quit) p.kv.k[off + i2] = kb;
+          if (owner && !quit) p.kv.k[off + i2] = kb;
         }
       } else {
         const size_t off = kv_off(p, l, b, pos, g);
         for (int i2 = lane; i2 < d; i2 += 32) {
           const __nv_bfloat16 vb = __float2bfloat16_rn(x[i2]);
           vcur()[b * d + i2] = vb;
-          if (rk == 0 && !quit) p.kv.v[off + i2] = vb;
+          if (owner && !quit) p.kv.v[off + i2] = vb;
         }
       }
     }
@@ -932,7 +970,7 @@ struct Consumer {
   __device__ __noinline__ void phase_a(int l) {
     tr(l, 0);
     const LayerDev& Lw = layer_s(p, l);
-    const int d = p.d, rep = p.nq / p.nkv;
+    const int d = p.d, rep = p.geo.repc;
     if (l == p.l0)
       first_input();
     else
@@ -940,12 +978,12 @@ struct Consumer {
     tr(l, 1);
     capture_rows(l, ha());
     norm_operand(ha(), Lw.attn_norm);
-    const int nA = rows_qkv(rep, d), rowlen = (rep + 2) * d;
+    const int nA = p.geo.nA, rowlen = (rep + 2) * d, cs = p.geo.cs;
     rows_product(kPA, su32(zt()), (uint32_t)zt_stride() * 2);
     tr(l, 2);
     // the raw q | k | v rows to every CTA of the cluster
     xarm((uint32_t)(p.B * rowlen * 4));
-    for (int w = tid; w < nA * p.B * kCS; w += kConsumers) {
+    for (int w = tid; w < nA * p.B * cs; w += kConsumers) {
       const int dest = w / (nA * p.B), v = w % (nA * p.B), j = v / p.B, b = v % p.B;
       xsend(raw() + b * rowlen + rk * nA + j, dest, __float_as_uint(ys()[j * 4 + b] * inv_of(b)));
     }
@@ -966,7 +1004,7 @@ struct Consumer {
   // output (t / d, t % d)). Ends on a barrier.
   __device__ void attend(int b, const __nv_bfloat16* Kp, const __nv_bfloat16* Vp, int nk,
                          float& o) {
-    const int d = p.d, rep = p.nq / p.nkv;
+    const int d = p.d, rep = p.geo.repc;
     float* s = ssc();  // [rep][64]
     const float* q = qs() + b * rep * d;
     for (int pr = warp; pr < nk * rep; pr += kConsumerWarps) {
@@ -1011,8 +1049,8 @@ struct Consumer {
   }
 
   __device__ __noinline__ void phase_b(int l) {
-    const int H = p.H, d = p.d, rep = p.nq / p.nkv, RD = rep * d, F = RD / kCS;
-    xarm((uint32_t)(kCS * p.B * (2 + F) * 4));
+    const int H = p.H, d = p.d, rep = p.geo.repc, RD = p.geo.RDc, F = p.geo.F, cs = p.geo.cs;
+    xarm((uint32_t)(cs * p.B * (2 + F) * 4));
     for (int b = 0; b < p.B; ++b) {
       if (tid < rep) {
         run_m()[tid] = -INFINITY;
@@ -1021,7 +1059,7 @@ struct Consumer {
       consumer_sync();
       float o = 0.f;
       int k0, k1;
-      slice(p.pos[b], kCS, rk, k0, k1);
+      slice(p.pos[b], cs, rk, k0, k1);
       for (int j0 = k0; j0 < k1;) {
         const int je = min(k1, (j0 / kPage + 1) * kPage);
         const __nv_bfloat16* Kp = reinterpret_cast<const __nv_bfloat16*>(chunk_wait(0));
@@ -1046,13 +1084,13 @@ struct Consumer {
     }
     tr(l, 4);
     xwait();
-    // merge the 16 states of the F outputs this CTA owns
+    // merge the cs states of the F outputs this CTA owns
     if (tid < p.B * F) {
       const int b = tid / F, f = tid % F;
       float M = -INFINITY;
-      for (int s2 = 0; s2 < kCS; ++s2) M = fmaxf(M, att()[(s2 * kMaxB + b) * (2 + F)]);
+      for (int s2 = 0; s2 < cs; ++s2) M = fmaxf(M, att()[(s2 * kMaxB + b) * (2 + F)]);
       float Ls = 0.f, Os = 0.f;
-      for (int s2 = 0; s2 < kCS; ++s2) {
+      for (int s2 = 0; s2 < cs; ++s2) {
         const float* e = att() + (s2 * kMaxB + b) * (2 + F);
         const float w = (e[0] == -INFINITY) ? 0.f : expf(e[0] - M);
         Ls = fmaf(e[1], w, Ls);
@@ -1064,7 +1102,7 @@ struct Consumer {
     // the merged outputs (hi and lo bf16 terms, pairs of columns) to every CTA
     xarm((uint32_t)(p.B * RD * 2 * 2));
     const int F2 = F / 2;
-    for (int w = tid; w < p.B * F2 * kCS; w += kConsumers) {
+    for (int w = tid; w < p.B * F2 * cs; w += kConsumers) {
       const int dest = w / (p.B * F2), v = w % (p.B * F2), b = v / F2, f = 2 * (v % F2);
       __nv_bfloat16 h0, l0, h1, l1;
       split_bf16(cmb()[b * F + f], h0, l0);
@@ -1076,13 +1114,13 @@ struct Consumer {
     xwait();
     tr(l, 5);
     // O projection rows of this CTA
-    const int nO = rows_out(H);
+    const int nO = p.geo.nO;
     rows_product(kPO, su32(zo()), (uint32_t)zo_stride() * 2);
     const uint32_t tag = tag_of(p.tag0, l, p.l0, 0);
     if (l != p.withhold_layer && !quit)
       for (int t = tid; t < nO * p.B; t += kConsumers) {
         const int j = t / p.B, b = t % p.B;
-        st_tag(p.po + ((size_t)g * kMaxB + b) * H + rk * nO + j, ys()[j * 4 + b], tag);
+        st_tag(p.po + ((size_t)cl * kMaxB + b) * H + rk * nO + j, ys()[j * 4 + b], tag);
       }
     tr(l, 6);
   }
@@ -1091,7 +1129,7 @@ struct Consumer {
 
   __device__ __noinline__ void phase_c(int l) {
     const LayerDev& Lw = layer_s(p, l);
-    const int H = p.H, nc = cols_mlp(p.I, p.nkv), Kc = p.I / p.nkv;
+    const int H = p.H, nc = p.geo.nc, Kc = p.geo.Kc, cs = p.geo.cs;
     exchange_sum(p.po, tag_of(p.tag0, l, p.l0, 0), ha(), hm());
     tr(l, 7);
     norm_operand(hm(), Lw.ffn_norm);
@@ -1105,7 +1143,7 @@ struct Consumer {
     tr(l, 8);
     xarm((uint32_t)(p.B * Kc * 2 * 2));
     const int n2 = nc / 2;
-    for (int w = tid; w < p.B * n2 * kCS; w += kConsumers) {
+    for (int w = tid; w < p.B * n2 * cs; w += kConsumers) {
       const int dest = w / (p.B * n2), v = w % (p.B * n2), b = v / n2, j = 2 * (v % n2);
       __nv_bfloat16 h0, l0, h1, l1;
       split_bf16(act()[b * nc + j], h0, l0);
@@ -1116,13 +1154,13 @@ struct Consumer {
     }
     xwait();
     tr(l, 9);
-    const int nO = rows_out(H);
+    const int nO = p.geo.nO;
     rows_product(kPD, su32(za()), (uint32_t)za_stride() * 2);
     const uint32_t tag = tag_of(p.tag0, l, p.l0, 1);
     if (!quit)
       for (int t = tid; t < nO * p.B; t += kConsumers) {
         const int j = t / p.B, b = t % p.B;
-        st_tag(p.pd + ((size_t)g * kMaxB + b) * H + rk * nO + j, ys()[j * 4 + b], tag);
+        st_tag(p.pd + ((size_t)cl * kMaxB + b) * H + rk * nO + j, ys()[j * 4 + b], tag);
       }
     tr(l, 10);
   }
@@ -1217,7 +1255,7 @@ struct Consumer {
       const int e = min(b, n + cap), nr = e - n;
       if ((int)(i % p.lm_owners) == warp) {
         const unsigned char* st = chunk_wait_owned();
-        if (!quit) lm_rows(st, n, nr);
+        if (!warp_quit()) lm_rows(st, n, nr);
         __syncwarp();
         if (lane == 0 && !quit) mbar_arrive_n(&r.empty[stage], kConsumerWarps);
       }
@@ -1260,7 +1298,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_cluster_kernel(const __gri
         bt[k] = p.kv.block_table[(size_t)p.seq[k / pps] * pps + k % pps];
     }
     if (threadIdx.x < 16)  // zero bytes read by the tensor-core loads of padding rows
-      reinterpret_cast<uint32_t*>(smem + p.off_misc + 256)[threadIdx.x] = 0u;
+      reinterpret_cast<uint32_t*>(smem + p.off_misc)[threadIdx.x] = 0u;
   }
   // every CTA's barriers are initialised before any peer may signal them
   cluster_sync_all();
@@ -1271,13 +1309,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_cluster_kernel(const __gri
     trow[12] = now_ns();
     trow[13] = clock64();
   }
-  volatile unsigned int* counts = reinterpret_cast<volatile unsigned int*>(smem + p.off_misc + 360);
+  volatile unsigned int* counts = reinterpret_cast<volatile unsigned int*>(smem + p.off_misc + 104);
   bool quit_any = false;
   if (warp == kConsumerWarps) {
     if (lane == 0) {
       Producer pr(p, ring);
-      const int g = c / kCS, rk = (int)cluster_rank();
-      for (int l = p.l0; l < p.l1 && !pr.quit; ++l) pr.layer(l, g, rk);
+      const int cl = c / p.geo.cs, rk = (int)cluster_rank();
+      for (int l = p.l0; l < p.l1 && !pr.quit; ++l) pr.layer(l, cl, cl / p.geo.split, rk);
       int a, b;
       slice(p.V, gridDim.x, c, a, b);
       if (!pr.quit) pr.tail(a, b);
@@ -1333,19 +1371,22 @@ struct PackArgs {
   const void* w[kNumLin];
   const __half* s[kNumLin];
   int H, nq, nkv, d, I;
+  Geo geo;
   int q8;
-  unsigned char* dst;  // this block's images: [n_kv][16][stream_bytes]
+  unsigned char* dst;  // this block's images: [clusters][cs][stream_bytes]
   int stream_bytes;
   int pofs[4];
 };
 
 __global__ void pack_kernel(const PackArgs a) {
+  const Geo& G = a.geo;
   const int cta = blockIdx.x, j = blockIdx.y, ph = blockIdx.z;
-  int n[4], K[4];
-  phase_geometry(a.H, a.nq, a.nkv, a.d, a.I, n, K);
+  const int* n = G.n;
   if (j >= n[ph]) return;
   const bool q8 = a.q8 != 0;
-  const int g = cta / kCS, r = cta % kCS, Kp = K[ph], rep = a.nq / a.nkv, RD = rep * a.d;
+  const int cl = cta / G.cs, r = cta % G.cs, g = cl / G.split, hs = cl % G.split;
+  const int Kp = G.K[ph], RD = G.RDc;
+  const int q0 = (g * (a.nq / a.nkv) + hs * G.repc) * a.d;  // first q row / Wo column of the cluster
   int lin, kfull, col0;
   size_t row;
   if (ph == kPA) {
@@ -1354,7 +1395,7 @@ __global__ void pack_kernel(const PackArgs a) {
     col0 = 0;
     if (rho < RD) {
       lin = kWq;
-      row = (size_t)g * RD + rho;
+      row = (size_t)q0 + rho;
     } else if (rho < RD + a.d) {
       lin = kWk;
       row = (size_t)g * a.d + rho - RD;
@@ -1366,9 +1407,9 @@ __global__ void pack_kernel(const PackArgs a) {
     lin = kWo;
     row = (size_t)r * n[kPO] + j;
     kfull = a.nq * a.d;
-    col0 = g * RD;
+    col0 = q0;
   } else if (ph == kPGU) {
-    const int nc = n[kPGU] / 2, c0 = g * (a.I / a.nkv) + r * nc;
+    const int nc = G.nc, c0 = cl * G.Kc + r * nc;
     lin = j < nc ? kWg : kWu;
     row = (size_t)c0 + (j < nc ? j : j - nc);
     kfull = a.H;
@@ -1377,24 +1418,23 @@ __global__ void pack_kernel(const PackArgs a) {
     lin = kWd;
     row = (size_t)r * n[kPD] + j;
     kfull = a.I;
-    col0 = g * (a.I / a.nkv);
+    col0 = cl * G.Kc;
   }
   const int cap = cap_rows(Kp, q8), c = j / cap, slot = j - c * cap;
   const int nr = min(cap, n[ph] - c * cap);
   unsigned char* chunk = a.dst + (size_t)cta * a.stream_bytes + a.pofs[ph] +
                          (size_t)c * chunk_bytes(cap, Kp, q8);
-  const int sw = j & 7;
   if (!q8) {
     const unsigned short* src =
         static_cast<const unsigned short*>(a.w[lin]) + row * kfull + col0;
     unsigned short* dst = reinterpret_cast<unsigned short*>(chunk + (size_t)slot * 2 * Kp);
     for (int e = threadIdx.x; e < Kp; e += blockDim.x)
-      dst[(((e >> 3) ^ sw) << 3) | (e & 7)] = src[e];
+      dst[(swz(e >> 3, j, Kp / 8) << 3) | (e & 7)] = src[e];
   } else {
     const unsigned char* src = static_cast<const unsigned char*>(a.w[lin]) + row * kfull + col0;
     unsigned char* dst = chunk + (size_t)slot * Kp;
     for (int e = threadIdx.x; e < Kp; e += blockDim.x)
-      dst[(((e >> 4) ^ sw) << 4) | (e & 15)] = src[e];
+      dst[(swz(e >> 4, j, Kp / 16) << 4) | (e & 15)] = src[e];
     const __half* ssrc = a.s[lin] + row * (kfull / 32) + col0 / 32;
     __half* sdst = reinterpret_cast<__half*>(chunk + (size_t)nr * Kp + (size_t)slot * (Kp / 16));
     for (int t = threadIdx.x; t < Kp / 32; t += blockDim.x) sdst[t] = ssrc[t];
@@ -1418,6 +1458,7 @@ struct ClusterState {
   unsigned char* packed = nullptr;
   int stream_bytes = 0;
   int pofs[4] = {0, 0, 0, 0};
+  clus::Geo geo{};
   uint32_t next_tag = 1;
   bool eligible = false;
   unsigned long long wait_ns = 1000000000ull;
@@ -1426,17 +1467,16 @@ struct ClusterState {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-bool shape_ok(const fs_model* m) {
-  const Shape& s = m->s;
-  if (s.nkv < 1 || s.nq % s.nkv) return false;
-  const int rep = s.nq / s.nkv, RD = rep * s.d;
-  if (s.H > clus::kMaxH || s.H % 128 || s.d % 32 || s.d > 128) return false;
-  if ((rep + 2) * s.d % clus::kCS || clus::rows_qkv(rep, s.d) > clus::kMaxRows) return false;
-  if (RD % 128 || RD > 256 || (RD / clus::kCS) % 2) return false;  // O-product K; pairs of outputs
-  if (s.H % clus::kCS || clus::rows_out(s.H) > clus::kMaxRows) return false;
-  if (s.I % (s.nkv * clus::kCS)) return false;
-  const int nc = clus::cols_mlp(s.I, s.nkv);
-  if (nc % 2 || 2 * nc > clus::kMaxRows || (s.I / s.nkv) % 128) return false;
+// The split (cs CTAs per cluster, split clusters per kv head) covers the
+// shape: every per-CTA share is whole and fits the kernel's buffers.
+bool geo_ok(const Shape& s, const clus::Geo& g) {
+  if (g.cs > clus::kMaxCS || s.nkv < 1 || s.nq % s.nkv || (s.nq / s.nkv) % g.split) return false;
+  if (s.H > clus::kMaxH || s.H % 64 || s.d % 64 || s.d > 128) return false;
+  if ((g.repc + 2) * s.d % g.cs || g.nA > clus::kMaxRows || g.nA < 1) return false;
+  if (g.RDc % 64 || g.RDc > 256 || g.RDc % g.cs || g.F % 2 || s.d % g.F) return false;
+  if (s.H % g.cs || g.nO > clus::kMaxRows) return false;
+  if (s.I % (g.ncl * g.cs) || g.nc < 1 || g.nc % 2 || 2 * g.nc > clus::kMaxRows) return false;
+  if (g.Kc % 64) return false;
   if (s.L > 64 || s.V >= 0x7fffffff) return false;
   return true;
 }
@@ -1460,37 +1500,53 @@ const void* kernel_for(int B, bool q8) {
 fs_status cluster_init(fs_model* m) {
   ClusterState* st = new ClusterState();
   m->cl_extras = st;
-  st->eligible = shape_ok(m);
-  if (!st->eligible) return FS_OK;
   const Shape& s = m->s;
-  // one cluster of 16 CTAs per kv head, every cluster resident at once
-  for (int nb : {1, 4}) {
-    const void* k = kernel_for(nb, m->q8);
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
-      cudaGetLastError();
-      st->eligible = false;
-      return FS_OK;
+  // The first split whose clusters all fit on the device at once: 16-CTA
+  // clusters, one per kv head; 8-CTA clusters, two per kv head; 8-CTA
+  // clusters, one per kv head.
+  st->eligible = false;
+  const int splits[3][2] = {{16, 1}, {8, 2}, {8, 1}};
+  for (const auto& sp : splits) {
+    const int cs = sp[0];
+    const clus::Geo g = clus::make_geo(s.H, s.nq, s.nkv, s.d, s.I, cs, sp[1]);
+    if (!geo_ok(s, g)) continue;
+    bool fits = true;
+    for (int nb : {1, 4}) {
+      const void* k = kernel_for(nb, m->q8);
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448) !=
+              cudaSuccess ||
+          cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+              cudaSuccess) {
+        cudaGetLastError();
+        fits = false;
+        break;
+      }
+      cudaLaunchConfig_t cfg{};
+      cfg.gridDim = dim3(g.ncl * cs);
+      cfg.blockDim = dim3(clus::kThreads);
+      cfg.dynamicSmemBytes = 232448;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = cs;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, k, &cfg) != cudaSuccess || n < g.ncl) {
+        cudaGetLastError();
+        fits = false;
+        break;
+      }
     }
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(s.nkv * clus::kCS);
-    cfg.blockDim = dim3(clus::kThreads);
-    cfg.dynamicSmemBytes = 232448;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = clus::kCS;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, k, &cfg) != cudaSuccess || n < s.nkv) {
-      cudaGetLastError();
-      st->eligible = false;
-      return FS_OK;
+    if (fits) {
+      st->geo = g;
+      st->eligible = true;
+      break;
     }
   }
+  if (!st->eligible) return FS_OK;
+  const clus::Geo& G = st->geo;
   auto alloc = [&](void** p, size_t bytes) {
     if (cudaMalloc(p, bytes) != cudaSuccess) {
       cudaGetLastError();
@@ -1500,16 +1556,14 @@ fs_status cluster_init(fs_model* m) {
     cudaMemset(*p, 0, bytes);
     return true;
   };
-  int n[4], K[4];
-  clus::phase_geometry(s.H, s.nq, s.nkv, s.d, s.I, n, K);
   int acc = 0;
   for (int ph = 0; ph < clus::kPhases; ++ph) {
     st->pofs[ph] = acc;
-    acc += clus::phase_bytes(n[ph], K[ph], m->q8);
+    acc += clus::phase_bytes(G.n[ph], G.K[ph], m->q8);
   }
   st->stream_bytes = acc;
-  const size_t image = (size_t)s.nkv * clus::kCS * acc;  // one block's images
-  const size_t words = (size_t)s.nkv * clus::kMaxB * s.H * sizeof(unsigned long long);
+  const size_t image = (size_t)G.ncl * G.cs * acc;  // one block's images
+  const size_t words = (size_t)G.ncl * clus::kMaxB * s.H * sizeof(unsigned long long);
   bool ok = alloc((void**)&st->po, words) && alloc((void**)&st->pd, words) &&
             alloc((void**)&st->am_key, clus::kMaxB * sizeof(unsigned long long)) &&
             alloc((void**)&st->am_cnt, 64) && alloc((void**)&st->abort_flag, 64) &&
@@ -1523,11 +1577,12 @@ fs_status cluster_init(fs_model* m) {
         a.s[t] = m->layers[l].s[t];
       }
       a.H = s.H; a.nq = s.nq; a.nkv = s.nkv; a.d = s.d; a.I = s.I;
+      a.geo = G;
       a.q8 = m->q8 ? 1 : 0;
       a.dst = st->packed + image * l;
       a.stream_bytes = acc;
       for (int ph = 0; ph < 4; ++ph) a.pofs[ph] = st->pofs[ph];
-      clus::pack_kernel<<<dim3(s.nkv * clus::kCS, clus::kMaxRows, clus::kPhases), 128>>>(a);
+      clus::pack_kernel<<<dim3(G.ncl * G.cs, clus::kMaxRows, clus::kPhases), 128>>>(a);
     }
     ok = cudaDeviceSynchronize() == cudaSuccess;
     if (!ok) cudaGetLastError();
@@ -1580,7 +1635,9 @@ fs_status decode_cluster(fs_model* m, const fs_kv* kv, const RowMap& map, int B,
   if (!st || !st->eligible || B > clus::kMaxB || B < 1) return FS_ERR_UNSUPPORTED;
   const Shape& s = m->s;
   clus::Params p{};
+  const clus::Geo& G = st->geo;
   p.L = s.L; p.H = s.H; p.nq = s.nq; p.nkv = s.nkv; p.d = s.d; p.I = s.I; p.V = s.V;
+  p.geo = G;
   p.eps = s.eps;
   p.layers = st->layers;
   p.embed = m->embed;
@@ -1621,7 +1678,7 @@ fs_status decode_cluster(fs_model* m, const fs_kv* kv, const RowMap& map, int B,
   if (st->next_tag > 0xF0000000u) {
     // wrap: clear the tags so the numbering can restart
     cudaStreamSynchronize(stream);
-    const size_t words = (size_t)s.nkv * clus::kMaxB * s.H * sizeof(unsigned long long);
+    const size_t words = (size_t)G.ncl * clus::kMaxB * s.H * sizeof(unsigned long long);
     cudaMemsetAsync(st->po, 0, words, stream);
     cudaMemsetAsync(st->pd, 0, words, stream);
     st->next_tag = 1;
@@ -1629,17 +1686,18 @@ fs_status decode_cluster(fs_model* m, const fs_kv* kv, const RowMap& map, int B,
   p.tag0 = st->next_tag;
   st->next_tag += 2u * (uint32_t)(l1 - l0) + 1u;
   // shared memory carve-up
-  const int rep = s.nq / s.nkv, RD = rep * s.d, F = RD / clus::kCS, nc = clus::cols_mlp(s.I, s.nkv);
-  const int Kc = s.I / s.nkv;
+  const int rep = G.repc, RD = G.RDc, F = G.F, nc = G.nc, Kc = G.Kc;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
     off += align_up(bytes, 128);
     return (int)o;
   };
-  const int n_items = 4 * std::max(std::max(s.H, Kc) / 128, 1);  // row tiles x k-blocks
+  int n_items = 0;  // tensor-core work items of the largest product
+  for (int ph = 0; ph < clus::kPhases; ++ph)
+    n_items = std::max(n_items, (G.n[ph] + 15) / 16 * (G.K[ph] / 64));
   const size_t red = std::max((size_t)n_items * 64 * 4,
-                              ((size_t)s.nkv + 1) * B * (s.H / clus::kCS) * 4);
+                              ((size_t)G.ncl + 1) * B * (s.H / G.cs) * 4);
   const size_t tab_ptrs = (size_t)s.L * sizeof(LayerDev);
   const size_t bt_bytes = (size_t)B * kv->pages_per_seq * sizeof(int32_t);
   const bool bt_smem = bt_bytes <= 8192;
@@ -1655,14 +1713,14 @@ fs_status decode_cluster(fs_model* m, const fs_kv* kv, const RowMap& map, int B,
     take((size_t)B * (rep + 2) * s.d * 4);          // raw
     take((size_t)B * RD * 4);                       // q
     take((size_t)2 * clus::kMaxB * s.d * 2);        // kcur, vcur
-    take((size_t)clus::kCS * clus::kMaxB * (2 + F) * 4);  // att
+    take((size_t)G.cs * clus::kMaxB * (2 + F) * 4);  // att
     take((size_t)B * F * 4);                        // cmb
     take((size_t)B * nc * 4);                       // act
     take((size_t)std::max(2 * kPage + 8, clus::kConsumerWarps * 128) * 4);  // ssc
     take((size_t)clus::kMaxRows * 4 * 4);           // ys
     take(red);
     take((size_t)clus::kConsumerWarps * clus::kMaxB * 4);  // ss
-    take(1024);                                     // misc
+    take(1152);                                     // misc
     take((size_t)(2 * clus::kMaxStages + 2) * 8);   // barriers
     take(tab_ptrs + (bt_smem ? bt_bytes : 0));      // tables
     fixed = off;
@@ -1671,16 +1729,9 @@ fs_status decode_cluster(fs_model* m, const fs_kv* kv, const RowMap& map, int B,
   int n_stages = (int)((budget - std::min(fixed, budget)) / clus::kStage);
   n_stages = std::min(n_stages, clus::kMaxStages);
   // the most chunks one phase holds at once
-  int need = 2;  // K and V of an attention segment
-  {
-    int n[4], K[4];
-    clus::phase_geometry(s.H, s.nq, s.nkv, s.d, s.I, n, K);
-    for (int ph = 0; ph < clus::kPhases; ++ph) {
-      const int cap = clus::cap_rows(K[ph], m->q8);
-      need = std::max(need, (n[ph] + cap - 1) / cap);
-    }
-  }
-  if (n_stages < 4 || n_stages < need) return FS_ERR_UNSUPPORTED;
+  // products take their chunks in passes of at most a ring; an attention
+  // segment holds 2 chunks
+  if (n_stages < 4) return FS_ERR_UNSUPPORTED;
   off = (size_t)n_stages * clus::kStage;
   p.off_ha = take((size_t)B * s.H * 4);
   p.off_hm = take((size_t)B * s.H * 4);
@@ -1690,14 +1741,14 @@ fs_status decode_cluster(fs_model* m, const fs_kv* kv, const RowMap& map, int B,
   p.off_raw = take((size_t)B * (rep + 2) * s.d * 4);
   p.off_q = take((size_t)B * RD * 4);
   p.off_kv = take((size_t)2 * clus::kMaxB * s.d * 2);
-  p.off_att = take((size_t)clus::kCS * clus::kMaxB * (2 + F) * 4);
+  p.off_att = take((size_t)G.cs * clus::kMaxB * (2 + F) * 4);
   p.off_cmb = take((size_t)B * F * 4);
   p.off_act = take((size_t)B * nc * 4);
   p.off_ssc = take((size_t)std::max(2 * kPage + 8, clus::kConsumerWarps * 128) * 4);
   p.off_ys = take((size_t)clus::kMaxRows * 4 * 4);
   p.off_red = take(red);
   p.off_ss = take((size_t)clus::kConsumerWarps * clus::kMaxB * 4);
-  p.off_misc = take(1024);
+  p.off_misc = take(1152);
   p.off_bar = take((size_t)(2 * clus::kMaxStages + 2) * 8);
   p.off_tab = take(tab_ptrs + (bt_smem ? bt_bytes : 0));
   if (off > budget) return FS_ERR_UNSUPPORTED;
@@ -1706,13 +1757,13 @@ fs_status decode_cluster(fs_model* m, const fs_kv* kv, const RowMap& map, int B,
   p.lm_owners = std::min(clus::kConsumerWarps, n_stages);
   p.lm_rows = std::min(8, clus::kStage / (2 * s.H));
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(s.nkv * clus::kCS);
+  cfg.gridDim = dim3(G.ncl * G.cs);
   cfg.blockDim = dim3(clus::kThreads);
   cfg.dynamicSmemBytes = off;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = clus::kCS;
+  attr[0].val.clusterDim.x = G.cs;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;

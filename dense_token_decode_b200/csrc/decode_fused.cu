@@ -54,7 +54,7 @@ constexpr int kMaxB = 4;
 constexpr int kData = 16384;   // main area of a Q8_0 stage
 constexpr int kExtra = 2048;   // Q8_0 scale area after it
 constexpr int kStageQ8 = kData + kExtra;
-constexpr int kStageBf16 = 8 * (2 * 1024 + 16);  // eight padded bf16 rows of K = 1024
+constexpr int kStageBf16 = 8 * 2 * 1024;  // eight bf16 rows of K = 1024
 constexpr int kMaxStages = 16;
 constexpr int kSlice = 8;      // head-dimension slice of one attention unit
 constexpr int kMaxRep = 2;     // query heads per kv head
@@ -189,6 +189,20 @@ __device__ __forceinline__ bool __syncthreads_or_consumers(bool v) {
 __device__ __forceinline__ bool aborted(const int* flag) {
   return *reinterpret_cast<const volatile int*>(flag) != 0;
 }
+// Whether a wait first stamped at t0 (0: stamp it now) must stop: it ran
+// past `limit`, or, once it has lasted 20 us, another CTA raised the abort
+// flag. Only waits that already took long read the one shared flag, so the
+// many short waits of a step do not all poll the same word.
+__device__ __forceinline__ bool wait_expired(unsigned long long& t0, unsigned long long limit,
+                                             const int* abort_flag) {
+  const unsigned long long t = now_ns();
+  if (t0 == 0) {
+    t0 = t;
+    return false;
+  }
+  const unsigned long long dt = t - t0;
+  return dt > 20000ull && (dt > limit || aborted(abort_flag));
+}
 __device__ __forceinline__ float lo16(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float hi16(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
 __device__ __forceinline__ float warp_sum(float v) {
@@ -234,12 +248,13 @@ __host__ __device__ inline void slice(int N, int G, int c, int& a, int& b) {
 }
 
 // Layout of weight rows in a stage (the consumers and the producer agree on
-// it). bf16 rows (K = H) sit 2H + 16 bytes apart, so the rows an ldmatrix
-// reads together fall in different shared-memory banks; Q8_0 code rows are
-// packed (H bytes apart) with their scales at kData.
-__host__ __device__ inline int row_stride(int H, bool q8) { return q8 ? H : 2 * H + 16; }
+// it): rows packed as in memory (bf16 2H bytes apart, Q8_0 codes H bytes
+// apart with their scales at kData), so a chunk of consecutive rows is one
+// bulk copy. (A bulk copy per row, to pad the rows against bank conflicts of
+// the ldmatrix reads, made the producer's copy issue the bottleneck.)
+__host__ __device__ inline int row_stride(int H, bool q8) { return q8 ? H : 2 * H; }
 __host__ __device__ inline int rows_cap(int H, bool q8) {  // rows of K = H per chunk
-  const int r = q8 ? kData / H : kStageBf16 / (2 * H + 16);
+  const int r = q8 ? kData / H : kStageBf16 / (2 * H);
   return r < 16 ? r : 16;
 }
 __host__ __device__ inline int pairs_cap(int H, bool q8) {
@@ -321,8 +336,7 @@ struct Producer {
     int spins = 0;
     while (!mbar_test(&r.empty[s], parity)) {
       if ((++spins & 15) == 0) {
-        if (t0 == 0) t0 = now_ns();
-        if (aborted(p.abort_flag) || now_ns() - t0 > p.wait_ns) {
+        if (wait_expired(t0, p.wait_ns, p.abort_flag)) {
           if (!aborted(p.abort_flag)) {
             atomicExch(p.abort_flag, 1);
             atomicCAS(p.err, 0, kErrTimeout);
@@ -344,19 +358,12 @@ struct Producer {
     }
   }
 
-  // Rows [n, e) of a [N][K = H] matrix into `st` from row slot `slot` on:
-  // bf16 rows one copy each at the padded stride, Q8_0 codes packed.
+  // Rows [n, n + nr) of a [N][K = H] matrix into `st` from row slot `slot`
+  // on, one bulk copy.
   __device__ void copy_rows(unsigned char* st, int slot, const void* w, int n, int nr, bool q8) {
-    const int H = p.H;
-    const uint32_t rb = q8 ? H : 2 * H;
+    const uint32_t rb = q8 ? p.H : 2 * p.H;
     const unsigned char* src = static_cast<const unsigned char*>(w) + (size_t)n * rb;
-    if (q8) {
-      bulk_load(st + slot * rb, src, nr * rb, bar(), policy);
-    } else {
-      const int rs = row_stride(H, false);
-      for (int i = 0; i < nr; ++i)
-        bulk_load(st + (slot + i) * rs, src + (size_t)i * rb, rb, bar(), policy);
-    }
+    bulk_load(st + slot * rb, src, nr * rb, bar(), policy);
   }
   // Rows [n, e) of a [N][K = H] matrix (bf16, or Q8_0 codes + scales).
   __device__ void rows(const void* w, const __half* s, int n, int e, bool q8) {
@@ -541,6 +548,10 @@ struct Consumer {
     }
     quit = true;
   }
+  // `quit` of any lane of this warp: the guard of warp-collective work
+  // (shuffles, ldmatrix, mma), which every lane must execute or skip
+  // together; per-thread quit alone may differ between lanes.
+  __device__ __forceinline__ bool warp_quit() const { return __any_sync(0xffffffffu, quit); }
 
   // Wait (whole warp) for the chunk `ahead` places after the oldest one this
   // warp has not released; returns its stage. Every chunk before it has been
@@ -565,8 +576,7 @@ struct Consumer {
       if ((++spins & 15) == 0) {
         int bad = 0;
         if (lane == 0) {
-          if (t0 == 0) t0 = now_ns();
-          bad = aborted(p.abort_flag) || now_ns() - t0 > p.wait_ns;
+          bad = wait_expired(t0, p.wait_ns, p.abort_flag);
         }
         if (__shfl_sync(0xffffffffu, bad, 0)) give_up();
       }
@@ -604,8 +614,7 @@ struct Consumer {
       if ((++spins & 15) == 0) {
         int bad = 0;
         if (lane == 0) {
-          if (t0 == 0) t0 = now_ns();
-          bad = aborted(p.abort_flag) || now_ns() - t0 > p.wait_ns;
+          bad = wait_expired(t0, p.wait_ns, p.abort_flag);
         }
         if (__shfl_sync(0xffffffffu, bad, 0)) give_up();
       }
@@ -650,15 +659,8 @@ struct Consumer {
     do {
       __nanosleep(20);
       x = ld_word(w);
-      if ((++spins & 7) == 0) {
-        // another CTA's abort ends the wait within a few polls; the time
-        // limit is read less often
-        bool stop = aborted(p.abort_flag);
-        if (!stop && (spins & 63) == 0) {
-          if (t0 == 0) t0 = now_ns();
-          stop = now_ns() - t0 > p.wait_ns;
-        }
-        if (stop) {
+      if ((++spins & 15) == 0) {
+        if (wait_expired(t0, p.wait_ns, p.abort_flag)) {
           give_up();
           break;
         }
@@ -1011,7 +1013,7 @@ struct Consumer {
       const unsigned char* st = chunk_wait();
       int r0 = (warp - (n - a)) % kConsumerWarps;
       if (r0 < 0) r0 += kConsumerWarps;
-      if (!quit) {
+      if (!warp_quit()) {
         for (int rr = r0; rr < nr; rr += kConsumerWarps) {
           float acc[NB];
           row_dot(st + rr * rb,
@@ -1234,7 +1236,7 @@ struct Consumer {
       const int nk = min(kPage, old - j0);
       const __nv_bfloat16* Kp = reinterpret_cast<const __nv_bfloat16*>(chunk_wait(0));
       const __nv_bfloat16* Vp = reinterpret_cast<const __nv_bfloat16*>(chunk_wait(1));
-      if (!quit) {
+      if (!warp_quit()) {
         const int g0 = j0 / 8, g1 = (j0 + nk + 7) / 8;
         int gi = g0 + ((warp - g0) % kConsumerWarps + kConsumerWarps) % kConsumerWarps;
         for (; gi < g1; gi += kConsumerWarps) {
@@ -1254,7 +1256,7 @@ struct Consumer {
   // the warps' states into o_s[b][h][t]. Ends on a barrier.
   __device__ __noinline__ void attn_finish(int b, int j, AttnState& S) {
     const int rep = p.nq / p.nkv, d = 4 * DQ, qq = lane & 3, kk = lane >> 2;
-    if (warp == 0 && !quit) {
+    if (warp == 0 && !warp_quit()) {
       float s[kMaxRep];
 #pragma unroll
       for (int h = 0; h < kMaxRep; ++h) {
@@ -1432,7 +1434,7 @@ struct Consumer {
     tr(l, 12);
     gather_norm(0, tag_of(p.tag0, l, p.l0, 2), gr, 1);
     tr(l, 8);
-    const int H = p.H, pc = pairs_cap(H, Q8W), rb = Q8W ? H : 2 * H, sb = Q8W ? H / 32 : 0;
+    const int H = p.H, pc = pairs_cap(H, Q8W);
     if constexpr (!Q8W) {
       // gate/up rows: all chunks resident, one tensor-core pass over 2P rows
       const int P = b - a, rs2 = row_stride(H, false);
@@ -1468,14 +1470,20 @@ struct Consumer {
       });
       for (int c = 0; c < nd; ++c) chunk_release();
       tr(l, 10);
-      return;
+    } else {
+      phase_c_q8(l, a, b);
     }
+  }
+
+  // Phase C with Q8_0 weights on the CUDA cores (codes widened in registers).
+  __device__ void phase_c_q8(int l, int a, int b) {
+    const int H = p.H, pc = pairs_cap(H, Q8W), rb = Q8W ? H : 2 * H, sb = Q8W ? H / 32 : 0;
     for (int n = a; n < b;) {
       const int e = min(b, n + pc), nr = e - n;
       const unsigned char* st = chunk_wait();
       int r0 = (warp - (n - a)) % kConsumerWarps;
       if (r0 < 0) r0 += kConsumerWarps;
-      if (!quit) {
+      if (!warp_quit()) {
         for (int rr = r0; rr < nr; rr += kConsumerWarps) {
           float gv[NB], uv[NB];
           const __half* sg = reinterpret_cast<const __half*>(st + kData) + rr * sb;
@@ -1555,7 +1563,7 @@ struct Consumer {
       const int e = min(b, n + cap), nr = e - n;
       if ((int)(i % p.lm_owners) == warp) {
         const unsigned char* st = chunk_wait_owned();
-        if (!quit) lm_rows_mma(st, n, nr);
+        if (!warp_quit()) lm_rows_mma(st, n, nr);
         __syncwarp();
         if (lane == 0 && !quit) mbar_arrive_n(&r.empty[stage], kConsumerWarps);
       }
