@@ -117,6 +117,7 @@ struct Params {
   int n_stages;
   int lm_owners, lm_rows;
   int bt_in_smem;
+  int off_par;  // a copy of these parameters in shared memory (see the kernel)
   int q8;
   const unsigned char* packed;  // [L][clusters][cs] per-CTA weight images of stream_bytes each
   int stream_bytes;
@@ -396,6 +397,52 @@ __host__ __device__ inline int swz(int u, int j, int units) {
 }
 
 // ---------------------------------------------------------------------------
+// Out-of-line waiting loops. They are free functions taking plain values, not
+// members: a member function that is not inlined takes the object's address,
+// which moves the whole object (ring cursor, flags, ...) to the stack, and
+// with shared memory taking most of L1 every member access then waits on
+// memory.
+
+// Warp-wide wait until bar1 (if not null) shows phase par1 and bar0 phase
+// par0, or the wait runs out; true if it ran out. `quit`: this lane gave up.
+__device__ __noinline__ bool warp_wait_slow(uint64_t* bar0, uint32_t par0, uint64_t* bar1,
+                                            uint32_t par1, bool quit, unsigned long long limit,
+                                            const int* abort_flag) {
+  unsigned long long t0 = 0;
+  int spins = 0;
+  const int lane = threadIdx.x & 31;
+  while (true) {
+    const bool ok = quit || ((bar1 == nullptr || mbar_test(bar1, par1)) && mbar_test(bar0, par0));
+    if (__all_sync(0xffffffffu, ok)) return false;
+    __nanosleep(32);
+    if ((++spins & 15) == 0) {
+      int bad = 0;
+      if (lane == 0) bad = wait_expired(t0, limit, abort_flag);
+      if (__shfl_sync(0xffffffffu, bad, 0)) return true;
+    }
+  }
+}
+// Polls one tagged word until its tag is `want`, backing off; *gave_up is set
+// when the wait runs out (the last value read is returned).
+__device__ __noinline__ unsigned long long poll_slow(const unsigned long long* w, uint32_t want,
+                                                     unsigned long long limit,
+                                                     const int* abort_flag, bool* gave_up) {
+  unsigned long long x = 0, t0 = 0;
+  int spins = 0;
+  unsigned int ns = 32;  // many waiting threads must not flood L2 with loads
+  do {
+    __nanosleep(ns);
+    ns = ns < 256 ? 2 * ns : 256;
+    x = ld_word(w);
+    if ((++spins & 15) == 0 && wait_expired(t0, limit, abort_flag)) {
+      *gave_up = true;
+      break;
+    }
+  } while (word_tag(x) != want);
+  return x;
+}
+
+// ---------------------------------------------------------------------------
 // Producer: issues the bulk copies of every chunk, in consumption order.
 
 struct Producer {
@@ -415,6 +462,9 @@ struct Producer {
     unsigned long long t0 = 0;
     int spins = 0;
     while (!mbar_test(&r.empty[s], parity)) {
+      // a spinning lane takes issue slots from the consumer warps of its
+      // scheduler: sleep between tests
+      __nanosleep(128);
       if ((++spins & 15) == 0) {
         if (wait_expired(t0, p.wait_ns, p.abort_flag)) {
           if (!aborted(p.abort_flag)) {
@@ -508,6 +558,7 @@ struct Consumer {
   uint32_t parity = 0;
   bool quit = false;
   unsigned int xk = 0;  // exchanges done
+  int cur_layer = 0;    // for trace stamps
   int tid, warp, lane, cta, cl, g, hs, rk, G;
   float inv[NB];
   unsigned long long wbest[kMaxB] = {0ull, 0ull, 0ull, 0ull};
@@ -564,7 +615,7 @@ struct Consumer {
     if (s >= r.n) s -= r.n;
     return su32(r.stages + (size_t)s * kStage);
   }
-  __device__ __noinline__ void give_up() {
+  __device__ __forceinline__ void give_up() {
     if (!aborted(p.abort_flag)) {
       atomicExch(p.abort_flag, 1);
       atomicCAS(p.err, 0, kErrTimeout);
@@ -577,26 +628,20 @@ struct Consumer {
   __device__ __forceinline__ bool warp_quit() const { return __any_sync(0xffffffffu, quit); }
   // Wait (whole warp) for the chunk `ahead` places after the oldest one this
   // warp has not released (every chunk before it waited for by this warp).
-  __device__ __noinline__ const unsigned char* chunk_wait(int ahead = 0) {
+  //
+  // The common case (the chunk is in) is inline; the waiting loop is not, so
+  // loops over chunks make no function call (calls spill registers to the
+  // stack, and with shared memory taking most of L1 those spills go to L2).
+  __device__ __forceinline__ const unsigned char* chunk_wait(int ahead = 0) {
     int s = stage + ahead;
     uint32_t par = parity;
     if (s >= r.n) {
       s -= r.n;
       par ^= 1u;
     }
-    unsigned long long t0 = 0;
-    int spins = 0;
-    while (true) {
-      const bool ok = quit || mbar_test(&r.full[s], par);
-      if (__all_sync(0xffffffffu, ok)) break;
-      if ((++spins & 15) == 0) {
-        int bad = 0;
-        if (lane == 0) {
-          bad = wait_expired(t0, p.wait_ns, p.abort_flag);
-        }
-        if (__shfl_sync(0xffffffffu, bad, 0)) give_up();
-      }
-    }
+    if (!__all_sync(0xffffffffu, quit || mbar_test(&r.full[s], par)) &&
+        warp_wait_slow(&r.full[s], par, nullptr, 0u, quit, p.wait_ns, p.abort_flag))
+      give_up();
     return r.stages + (size_t)s * kStage;
   }
   __device__ void cursor_advance() {
@@ -615,22 +660,13 @@ struct Consumer {
   }
   // Owner-mode wait of the LM head (this warp alone consumes the chunk): the
   // release of the chunk a ring earlier in the same stage, then the chunk.
-  __device__ __noinline__ const unsigned char* chunk_wait_owned() {
+  __device__ __forceinline__ const unsigned char* chunk_wait_owned() {
     const int s = stage;
-    unsigned long long t0 = 0;
-    int spins = 0;
-    while (true) {
-      const bool ok =
-          quit || (mbar_test(&r.empty[s], parity ^ 1u) && mbar_test(&r.full[s], parity));
-      if (__all_sync(0xffffffffu, ok)) break;
-      if ((++spins & 15) == 0) {
-        int bad = 0;
-        if (lane == 0) {
-          bad = wait_expired(t0, p.wait_ns, p.abort_flag);
-        }
-        if (__shfl_sync(0xffffffffu, bad, 0)) give_up();
-      }
-    }
+    if (!__all_sync(0xffffffffu, quit || (mbar_test(&r.empty[s], parity ^ 1u) &&
+                                          mbar_test(&r.full[s], parity))) &&
+        warp_wait_slow(&r.full[s], parity, &r.empty[s], parity ^ 1u, quit, p.wait_ns,
+                       p.abort_flag))
+      give_up();
     return r.stages + (size_t)s * kStage;
   }
 
@@ -645,12 +681,13 @@ struct Consumer {
   __device__ __forceinline__ void xsend(const void* local_dst, int dest, uint32_t v) {
     st_async(mapa(su32(local_dst), (uint32_t)dest), v, mapa(su32(&xbar()[xk & 1]), (uint32_t)dest));
   }
-  __device__ __noinline__ void xwait() {
+  __device__ __forceinline__ void xwait() {
     uint64_t* bar = &xbar()[xk & 1];
     const uint32_t par = (xk >> 1) & 1u;
     unsigned long long t0 = 0;
     int spins = 0;
     while (!mbar_test_cluster(bar, par)) {
+      __nanosleep(32);
       if (quit) break;
       if ((++spins & 15) == 0) {
         if (wait_expired(t0, p.wait_ns, p.abort_flag)) {
@@ -663,38 +700,35 @@ struct Consumer {
     consumer_sync();  // the received data are read by every thread after this
   }
 
-  // Polls one tagged word until its tag is `want` (bounded).
-  __device__ __noinline__ unsigned long long poll_word_slow(const unsigned long long* w,
-                                                            uint32_t want) {
-    unsigned long long x = 0, t0 = 0;
-    int spins = 0;
-    do {
-      __nanosleep(20);
-      x = ld_word(w);
-      if ((++spins & 15) == 0) {
-        if (wait_expired(t0, p.wait_ns, p.abort_flag)) {
-          give_up();
-          break;
-        }
-      }
-    } while (word_tag(x) != want);
-    return x;
-  }
+  // Polls one tagged word until its tag is `want` (bounded); x: the value
+  // already loaded.
   __device__ __forceinline__ unsigned long long poll_word(const unsigned long long* w,
                                                           unsigned long long x, uint32_t want) {
     if (word_tag(x) == want || quit) return x;
-    return poll_word_slow(w, want);
+    bool gave_up = false;
+    x = poll_slow(w, want, p.wait_ns, p.abort_flag, &gave_up);
+    if (gave_up) give_up();
+    return x;
   }
 
   // dst = base + sum over clusters of the tagged shares src[c][B][H], for the
-  // whole rows: this CTA sums its slice (elements [rk H/16, (rk+1) H/16) of
-  // each row, clusters in order) and sends it to every CTA of the cluster.
-  // Ends with the exchange complete.
-  __device__ __noinline__ void exchange_sum(const unsigned long long* src, uint32_t tag,
+  // whole rows: this CTA sums its slice (elements [rk E, (rk+1) E) of each
+  // row, E = H / cs, clusters in order) and sends it to every CTA of the
+  // cluster. The slice of cluster c is what rank rk of cluster c published.
+  // One thread per cluster first waits for that CTA's last word, so only a
+  // few threads poll while the shares are still coming; then every thread
+  // loads its words once (a word still stale is polled on its own). Ends
+  // with the exchange complete.
+  __device__ __forceinline__ void exchange_sum(const unsigned long long* src, uint32_t tag,
                                             const float* base, float* dst) {
     const int H = p.H, E = H / p.geo.cs, e0 = rk * E, n = p.B * E, total = p.geo.ncl * n;
     float* buf = red();
     float* sums = buf + total;
+    if (tid < p.geo.ncl) {
+      const unsigned long long* last = src + ((size_t)tid * kMaxB + p.B - 1) * H + e0 + E - 1;
+      poll_word(last, ld_word(last), tag);
+    }
+    consumer_sync();
     for (int f0 = tid; f0 < total; f0 += 4 * kConsumers) {
       unsigned long long w[4];
       const unsigned long long* ptr[4];
@@ -728,7 +762,7 @@ struct Consumer {
 
   // The block input of the first block: embedding rows of the tokens (or
   // h_in), whole rows, computed by every CTA. Ends on a barrier.
-  __device__ __noinline__ void first_input() {
+  __device__ __forceinline__ void first_input() {
     const int H = p.H;
     for (int k = tid; k < p.B * H; k += kConsumers) {
       const int b = k / H;
@@ -751,7 +785,7 @@ struct Consumer {
   // RMSNorm operand of the tensor-core products: zt rows (2b, 2b + 1) = the
   // hi and lo bf16 terms of gain * x_b, and inv[b] = 1/rms(x_b). Ends on a
   // barrier.
-  __device__ __noinline__ void norm_operand(const float* x, const __nv_bfloat16* gain) {
+  __device__ __forceinline__ void norm_operand(const float* x, const __nv_bfloat16* gain) {
     const int H = p.H;
     float ss[NB];
 #pragma unroll
@@ -797,7 +831,8 @@ struct Consumer {
   // product is term t of batch row b. Work items are (row tile, block of 64
   // columns), warp w taking items w, w + 11, ...; the items' partial sums are
   // added in a fixed order. Ends on a barrier.
-  __device__ __noinline__ void mma_rows(int R, int K, uint32_t ob, uint32_t ostride, int y0) {
+  __device__ __forceinline__ void mma_rows(int R, int K, uint32_t ob, uint32_t ostride, int y0,
+                                        bool stamp = false) {
     const uint32_t* ra = rowaddr();
     float* part = red();
     const int nkb = K / 64, mt = (R + 15) / 16, items = mt * nkb, twoB = 2 * p.B;
@@ -864,7 +899,9 @@ struct Consumer {
       part[(it * 16 + gq) * 4 + q] = (d0[0] + d1[0]) + (d0[1] + d1[1]);
       part[(it * 16 + gq + 8) * 4 + q] = (d0[2] + d1[2]) + (d0[3] + d1[3]);
     }
+    if (stamp) tr(cur_layer, 14);
     consumer_sync();
+    if (stamp) tr(cur_layer, 15);
     float* y = ys() + y0 * 4;
     for (int t = tid; t < R * 4; t += kConsumers) {
       const int rr = (t >> 2) & 15, q2 = t & 3, m = t >> 6;
@@ -876,15 +913,17 @@ struct Consumer {
   }
 
   // The rows of phase `ph` (spread over the next chunks) into ys: in passes
-  // of as many chunks as the ring holds, each pass waiting for its chunks,
-  // filling the row tables, running the product of its rows and releasing
-  // the chunks.
+  // of the chunks that hold two 16-row tiles (at least one chunk), each pass
+  // waiting for its chunks, filling the row tables, running the product of
+  // its rows and releasing the chunks at once, so the producer refills the
+  // ring while the later passes run.
   __device__ void rows_product(int ph, uint32_t ob, uint32_t ostride) {
     const int R = p.geo.n[ph], Kp = p.geo.K[ph], cap = cap_rows(Kp, Q8), nch = (R + cap - 1) / cap;
-    const int rb = Q8 ? Kp : 2 * Kp, pass = min(nch, r.n);
+    const int rb = Q8 ? Kp : 2 * Kp, pass = min(min(nch, r.n - 2), max(1, 32 / cap));
     for (int c0 = 0; c0 < nch; c0 += pass) {
       const int np = min(pass, nch - c0), j0 = c0 * cap, rows = min(R, (c0 + np) * cap) - j0;
       for (int c = 0; c < np; ++c) chunk_wait(c);
+      if (ph == kPGU && c0 == 0) tr(cur_layer, 12);
       if (warp == 0)
         for (int jj = lane; jj < rows; jj += 32) {
           const int j = j0 + jj, c = j / cap, slot = j - c * cap;  // chunk and row slot
@@ -893,16 +932,19 @@ struct Consumer {
           if (Q8) scaleaddr()[jj] = st + min(cap, R - c * cap) * Kp + slot * (Kp / 16);
         }
       consumer_sync();
-      mma_rows(rows, Kp, ob, ostride, j0);
+      const bool stamp = ph == kPGU && c0 == 0;
+      if (stamp) tr(cur_layer, 11);
+      mma_rows(rows, Kp, ob, ostride, j0, stamp);
+      if (stamp) tr(cur_layer, 13);
       for (int c = 0; c < np; ++c) chunk_release();
     }
   }
 
-  __device__ __noinline__ void tr(int layer, int k) {
+  __device__ __forceinline__ void tr(int layer, int k) {
     if (p.trace && tid == 0)
       p.trace[((size_t)cta * (p.L + 1) + layer) * kTraceSlots + k] = clock64();
   }
-  __device__ __noinline__ void capture_rows(int slot, const float* x) {
+  __device__ __forceinline__ void capture_rows(int slot, const float* x) {
     if (!p.capture || cta != 0) return;
     for (int k = tid; k < p.B * p.H; k += kConsumers) {
       const int b = k / p.H, e = k % p.H;
@@ -935,7 +977,7 @@ struct Consumer {
   // rotated, rounded to bf16 as the cache stores it) and v (bf16) of every
   // batch row from the exchanged raw rows; rank 0 appends k and v to the
   // cache. Ends on a barrier.
-  __device__ __noinline__ void prep_heads(int l) {
+  __device__ __forceinline__ void prep_heads(int l) {
     const LayerDev& Lw = layer_s(p, l);
     const int d = p.d, rep = p.geo.repc, nroles = rep + 2, rowlen = nroles * d;
     const bool owner = rk == 0 && hs == 0;  // appends the head's k and v
@@ -967,7 +1009,7 @@ struct Consumer {
     consumer_sync();
   }
 
-  __device__ __noinline__ void phase_a(int l) {
+  __device__ __forceinline__ void phase_a(int l) {
     tr(l, 0);
     const LayerDev& Lw = layer_s(p, l);
     const int d = p.d, rep = p.geo.repc;
@@ -1048,7 +1090,7 @@ struct Consumer {
     consumer_sync();
   }
 
-  __device__ __noinline__ void phase_b(int l) {
+  __device__ __forceinline__ void phase_b(int l) {
     const int H = p.H, d = p.d, rep = p.geo.repc, RD = p.geo.RDc, F = p.geo.F, cs = p.geo.cs;
     xarm((uint32_t)(cs * p.B * (2 + F) * 4));
     for (int b = 0; b < p.B; ++b) {
@@ -1127,7 +1169,7 @@ struct Consumer {
 
   // ---- phase C -------------------------------------------------------------
 
-  __device__ __noinline__ void phase_c(int l) {
+  __device__ __forceinline__ void phase_c(int l) {
     const LayerDev& Lw = layer_s(p, l);
     const int H = p.H, nc = p.geo.nc, Kc = p.geo.Kc, cs = p.geo.cs;
     exchange_sum(p.po, tag_of(p.tag0, l, p.l0, 0), ha(), hm());
@@ -1183,7 +1225,7 @@ struct Consumer {
   // thread loads 8 consecutive columns (32 blk + 8 q ..) of row gq and of
   // operand row gq, a column order both operands share; rows 8..15 of the
   // tile are zero.
-  __device__ __noinline__ void lm_rows(const unsigned char* st, int n0, int nr) {
+  __device__ __forceinline__ void lm_rows(const unsigned char* st, int n0, int nr) {
     const int gq = lane >> 2, q = lane & 3, H = p.H;
     const bool ha = gq < nr, hb = gq < 2 * p.B;
     const uint32_t ab = su32(st) + gq * 2 * H + q * 16;
@@ -1200,7 +1242,7 @@ struct Consumer {
     if (ha && q < p.B) fold_logit(q, n0 + gq, ((d0[0] + d1[0]) + (d0[1] + d1[1])) * inv_of(q));
   }
 
-  __device__ __noinline__ void finish_head() {
+  __device__ __forceinline__ void finish_head() {
     unsigned long long* bst = best();
     if (tid < kMaxB) bst[tid] = 0ull;
     consumer_sync();
@@ -1238,7 +1280,7 @@ struct Consumer {
     }
   }
 
-  __device__ __noinline__ void tail() {
+  __device__ __forceinline__ void tail() {
     const int L = p.L;
     tr(L, 0);
     exchange_sum(p.pd, tag_of(p.tag0, p.l1 - 1, p.l0, 1), hm(), ha());
@@ -1276,6 +1318,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_cluster_kernel(const __gri
   ring.n = p.n_stages;
   ring.full = reinterpret_cast<uint64_t*>(smem + p.off_bar);
   ring.empty = ring.full + kMaxStages;
+  // The phases read the parameters through a reference; a reference to the
+  // kernel's parameter space makes every such read a long-latency generic
+  // load, so they read a copy in shared memory instead.
+  Params* ps = reinterpret_cast<Params*>(smem + p.off_par);
+  for (int k = threadIdx.x; k < (int)(sizeof(Params) / 4); k += blockDim.x)
+    reinterpret_cast<unsigned*>(ps)[k] = reinterpret_cast<const unsigned*>(&p)[k];
   uint64_t* xbar = ring.empty + kMaxStages;
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.n_stages; ++s) {
@@ -1313,7 +1361,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_cluster_kernel(const __gri
   bool quit_any = false;
   if (warp == kConsumerWarps) {
     if (lane == 0) {
-      Producer pr(p, ring);
+      Producer pr(*ps, ring);
       const int cl = c / p.geo.cs, rk = (int)cluster_rank();
       for (int l = p.l0; l < p.l1 && !pr.quit; ++l) pr.layer(l, cl, cl / p.geo.split, rk);
       int a, b;
@@ -1323,11 +1371,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_cluster_kernel(const __gri
       counts[0] = pr.i;
     }
   } else {
-    Consumer<NB, Q8> cs(p, ring, smem);
+    Consumer<NB, Q8> cs(*ps, ring, smem);
     // `quit` is per thread, so it steers no path that holds a barrier: after
     // an abort every thread still walks all phases (waits return at once, no
     // global stores), and every exchange still sends its bytes.
     for (int l = p.l0; l < p.l1; ++l) {
+      cs.cur_layer = l;
       cs.phase_a(l);
       cs.phase_b(l);
       cs.phase_c(l);
@@ -1723,6 +1772,7 @@ fs_status decode_cluster(fs_model* m, const fs_kv* kv, const RowMap& map, int B,
     take(1152);                                     // misc
     take((size_t)(2 * clus::kMaxStages + 2) * 8);   // barriers
     take(tab_ptrs + (bt_smem ? bt_bytes : 0));      // tables
+    take(sizeof(clus::Params));                     // parameter copy
     fixed = off;
   }
   const size_t budget = 232448;
@@ -1751,6 +1801,7 @@ fs_status decode_cluster(fs_model* m, const fs_kv* kv, const RowMap& map, int B,
   p.off_misc = take(1152);
   p.off_bar = take((size_t)(2 * clus::kMaxStages + 2) * 8);
   p.off_tab = take(tab_ptrs + (bt_smem ? bt_bytes : 0));
+  p.off_par = take(sizeof(clus::Params));
   if (off > budget) return FS_ERR_UNSUPPORTED;
   p.bt_in_smem = bt_smem ? 1 : 0;
   p.n_stages = n_stages;

@@ -108,6 +108,7 @@ struct Params {
   int n_stages;
   int off_r, off_z, off_misc, off_attn, off_tab, off_bar, off_red;
   int bt_in_smem;
+  int off_par;  // a copy of these parameters in shared memory (see the kernel)
   int stage_bytes;
   int off_zt;     // [2 slots][2B rows: hi, lo of each batch row][H + 8] bf16 GEMV operands
   int lm_owners;  // warps that consume LM-head chunks (chunk i: warp i % lm_owners)
@@ -316,6 +317,51 @@ __host__ __device__ __forceinline__ uint32_t tag_of(uint32_t tag0, int l, int l0
 }
 
 // ---------------------------------------------------------------------------
+// Out-of-line waiting loops, as free functions taking plain values: a member
+// function that is not inlined takes the object's address, which moves the
+// whole consumer state (ring cursor, flags, ...) to the stack, and with shared
+// memory taking most of L1 every access to it then waits on memory.
+
+// Warp-wide wait until bar1 (if not null) shows phase par1 and bar0 phase
+// par0, or the wait runs out; true if it ran out.
+__device__ __noinline__ bool warp_wait_slow(uint64_t* bar0, uint32_t par0, uint64_t* bar1,
+                                            uint32_t par1, bool quit, unsigned long long limit,
+                                            const int* abort_flag) {
+  unsigned long long t0 = 0;
+  int spins = 0;
+  const int lane = threadIdx.x & 31;
+  while (true) {
+    const bool ok = quit || ((bar1 == nullptr || mbar_test(bar1, par1)) && mbar_test(bar0, par0));
+    if (__all_sync(0xffffffffu, ok)) return false;
+    __nanosleep(32);
+    if ((++spins & 15) == 0) {
+      int bad = 0;
+      if (lane == 0) bad = wait_expired(t0, limit, abort_flag);
+      if (__shfl_sync(0xffffffffu, bad, 0)) return true;
+    }
+  }
+}
+// Polls one tagged word until its tag is `want`, backing off; *gave_up is set
+// when the wait runs out.
+__device__ __noinline__ unsigned long long poll_slow(const unsigned long long* w, uint32_t want,
+                                                     unsigned long long limit,
+                                                     const int* abort_flag, bool* gave_up) {
+  unsigned long long x = 0, t0 = 0;
+  int spins = 0;
+  unsigned int ns = 32;  // many waiting threads must not flood L2 with loads
+  do {
+    __nanosleep(ns);
+    ns = ns < 256 ? 2 * ns : 256;
+    x = ld_word(w);
+    if ((++spins & 15) == 0 && wait_expired(t0, limit, abort_flag)) {
+      *gave_up = true;
+      break;
+    }
+  } while (word_tag(x) != want);
+  return x;
+}
+
+// ---------------------------------------------------------------------------
 // Producer: issues the bulk copies of every chunk, in consumption order.
 
 struct Producer {
@@ -335,6 +381,9 @@ struct Producer {
     unsigned long long t0 = 0;
     int spins = 0;
     while (!mbar_test(&r.empty[s], parity)) {
+      // a spinning lane takes issue slots from the consumer warps of its
+      // scheduler: sleep between tests
+      __nanosleep(128);
       if ((++spins & 15) == 0) {
         if (wait_expired(t0, p.wait_ns, p.abort_flag)) {
           if (!aborted(p.abort_flag)) {
@@ -537,11 +586,11 @@ struct Consumer {
 
   // Trace stamp k of (this CTA, layer): the SM's cycle counter (converted on
   // the host with the CTA's own globaltimer / clock pairs at start and end).
-  __device__ __noinline__ void tr(int layer, int k) {
+  __device__ __forceinline__ void tr(int layer, int k) {
     if (p.trace && tid == 0)
       p.trace[((size_t)cta * (p.L + 1) + layer) * kTraceSlots + k] = clock64();
   }
-  __device__ __noinline__ void give_up() {
+  __device__ __forceinline__ void give_up() {
     if (!aborted(p.abort_flag)) {
       atomicExch(p.abort_flag, 1);
       atomicCAS(p.err, 0, kErrTimeout);
@@ -564,23 +613,9 @@ struct Consumer {
       s -= r.n;
       par ^= 1u;
     }
-    if (__all_sync(0xffffffffu, mbar_test(&r.full[s], par))) return r.stages + (size_t)s * p.stage_bytes;
-    return chunk_wait_slow(s, par);
-  }
-  __device__ __noinline__ const unsigned char* chunk_wait_slow(int s, uint32_t par) {
-    unsigned long long t0 = 0;
-    int spins = 0;
-    while (true) {
-      const bool ok = quit || mbar_test(&r.full[s], par);
-      if (__all_sync(0xffffffffu, ok)) break;
-      if ((++spins & 15) == 0) {
-        int bad = 0;
-        if (lane == 0) {
-          bad = wait_expired(t0, p.wait_ns, p.abort_flag);
-        }
-        if (__shfl_sync(0xffffffffu, bad, 0)) give_up();
-      }
-    }
+    if (!__all_sync(0xffffffffu, quit || mbar_test(&r.full[s], par)) &&
+        warp_wait_slow(&r.full[s], par, nullptr, 0u, quit, p.wait_ns, p.abort_flag))
+      give_up();
     return r.stages + (size_t)s * p.stage_bytes;
   }
   __device__ void cursor_advance() {
@@ -603,24 +638,16 @@ struct Consumer {
   // the chunk itself. With n >= W the release test cannot see an older phase:
   // this warp waited on a chunk W places back, so every chunk 2n places back
   // has been released.
-  __device__ __noinline__ const unsigned char* chunk_wait_owned() {
+  __device__ __forceinline__ const unsigned char* chunk_wait_owned() {
     const int s = stage;
-    unsigned long long t0 = 0;
-    int spins = 0;
-    while (true) {
-      const bool ok =
-          quit || (mbar_test(&r.empty[s], parity ^ 1u) && mbar_test(&r.full[s], parity));
-      if (__all_sync(0xffffffffu, ok)) break;
-      if ((++spins & 15) == 0) {
-        int bad = 0;
-        if (lane == 0) {
-          bad = wait_expired(t0, p.wait_ns, p.abort_flag);
-        }
-        if (__shfl_sync(0xffffffffu, bad, 0)) give_up();
-      }
-    }
+    if (!__all_sync(0xffffffffu, quit || (mbar_test(&r.empty[s], parity ^ 1u) &&
+                                          mbar_test(&r.full[s], parity))) &&
+        warp_wait_slow(&r.full[s], parity, &r.empty[s], parity ^ 1u, quit, p.wait_ns,
+                       p.abort_flag))
+      give_up();
     return r.stages + (size_t)s * p.stage_bytes;
   }
+
 
   // ---- residual input of a phase -----------------------------------------
 
@@ -649,38 +676,32 @@ struct Consumer {
   __device__ __forceinline__ unsigned long long poll_word(const unsigned long long* w,
                                                           unsigned long long x, uint32_t want) {
     if (word_tag(x) == want || quit) return x;
-    return poll_word_slow(w, want);
-  }
-  __device__ __noinline__ unsigned long long poll_word_slow(const unsigned long long* w,
-                                                            uint32_t want) {
-    unsigned long long x = 0;
-    unsigned long long t0 = 0;
-    int spins = 0;
-    do {
-      __nanosleep(20);
-      x = ld_word(w);
-      if ((++spins & 15) == 0) {
-        if (wait_expired(t0, p.wait_ns, p.abort_flag)) {
-          give_up();
-          break;
-        }
-      }
-    } while (word_tag(x) != want);
+    bool gave_up = false;
+    x = poll_slow(w, want, p.wait_ns, p.abort_flag, &gave_up);
+    if (gave_up) give_up();
     return x;
   }
+
 
   // This CTA's slice of a residual sum: elements [e0, e1) of the flattened
   // [B][H] rows, each = base[e] (rs: the residual the half started from) plus
   // the partials of contributors 0..n_contrib-1 (slot c at src + c*B*H,
   // tagged tag_in), summed in a fixed order; published to dst with tag_out.
   // Ends on a barrier.
-  __device__ __noinline__ void reduce_slice(const unsigned long long* src, int n_contrib, uint32_t tag_in,
+  __device__ __forceinline__ void reduce_slice(const unsigned long long* src, int n_contrib, uint32_t tag_in,
                                unsigned long long* dst, uint32_t tag_out) {
     const int n = p.B * p.H;
     int e0, e1;
     slice(n, G, cta, e0, e1);
     const int E = e1 - e0, total = n_contrib * E;
     float* buf = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(rs) - p.off_r + p.off_red);
+    // one thread per contributor first waits for the slice's last word, so
+    // only a few threads poll while the partials are still coming
+    for (int c = tid; c < n_contrib && E > 0; c += kConsumers) {
+      const unsigned long long* last = src + (size_t)c * n + e1 - 1;
+      poll_word(last, ld_word(last), tag_in);
+    }
+    consumer_sync();
     for (int f0 = tid; f0 < total; f0 += 4 * kConsumers) {
       unsigned long long w[4];
       const unsigned long long* ptr[4];
@@ -720,7 +741,7 @@ struct Consumer {
   // `slot` (0: phase A and the LM head, 1: phase C) picks the buffers of zs and
   // of the partial sums, so a warp that runs ahead into the next phase never
   // writes what a slower warp still reads.
-  __device__ __noinline__ void gather_norm(int kind, uint32_t tag, const float (&gr)[kEPT], int slot) {
+  __device__ __forceinline__ void gather_norm(int kind, uint32_t tag, const float (&gr)[kEPT], int slot) {
     const int H = p.H, n = p.B * H;
     zs = zs_base + (size_t)slot * n;
     zt = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<unsigned char*>(misc) - p.off_misc +
@@ -733,6 +754,13 @@ struct Consumer {
     unsigned long long w[kEPT];
     const unsigned long long* src = kind >= 0 ? p.rsum + (size_t)kind * n : nullptr;
     if (kind >= 0) {
+      // one thread per reducing CTA first waits for the last word of its slice
+      for (int c = tid; c < G; c += kConsumers) {
+        int a, b;
+        slice(n, G, c, a, b);
+        if (b > a) poll_word(src + b - 1, ld_word(src + b - 1), tag);
+      }
+      consumer_sync();
 #pragma unroll
       for (int e = 0; e < kEPT; ++e) {
         const int k = tid + e * kConsumers;
@@ -839,7 +867,7 @@ struct Consumer {
   // (row tile, block of 8 k-steps), warp w taking items w, w + 11, ...; the
   // items' partial sums meet in shared memory and are added in a fixed order.
   // Ends on a barrier.
-  __device__ __noinline__ void mma_rows(int R) {
+  __device__ __forceinline__ void mma_rows(int R) {
     const uint32_t* ra = rowaddr();
     float* part = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(rs) - p.off_r + p.off_red);
     const int nkb = p.H / 128, mt = (R + 15) / 16, items = mt * nkb, twoB = 2 * p.B;
@@ -928,7 +956,7 @@ struct Consumer {
 
   // One LM-head chunk (nr <= 8 rows of the embedding at the padded stride) on
   // this warp: logits of every batch row, folded into the greedy keys.
-  __device__ __noinline__ void lm_rows_mma(const unsigned char* st, int n0, int nr) {
+  __device__ __forceinline__ void lm_rows_mma(const unsigned char* st, int n0, int nr) {
     const uint32_t rs2 = (uint32_t)row_stride(p.H, false), zero = zero_addr();
     const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
     const bool arow = row < nr;
@@ -955,7 +983,7 @@ struct Consumer {
 
   // ---- phase A: RMSNorm + QKV rows --------------------------------------
 
-  __device__ __noinline__ void capture_rows(int slot) {
+  __device__ __forceinline__ void capture_rows(int slot) {
     if (!p.capture || cta != 0) return;
     for (int k = tid; k < p.B * p.H; k += kConsumers) {
       const int b = k / p.H, e = k % p.H;
@@ -963,7 +991,7 @@ struct Consumer {
     }
   }
 
-  __device__ __noinline__ void phase_a(int l, int a, int b) {
+  __device__ __forceinline__ void phase_a(int l, int a, int b) {
     tr(l, 0);
     const LayerDev& Lw = layer_s(p, l);
     float gr[kEPT];
@@ -1101,7 +1129,7 @@ struct Consumer {
 
   // q heads, k and v of (row b, group g) into shared memory; the j = 0 unit
   // also appends k and v (bf16) to the cache. Ends on a barrier.
-  __device__ __noinline__ void attn_prep(int l, int b, int g, int j) {
+  __device__ __forceinline__ void attn_prep(int l, int b, int g, int j) {
     const int d = p.d, rep = p.nq / p.nkv, qd = p.nq * d, kvd = p.nkv * d;
     const int qkvd = qd + 2 * kvd, pos = p.pos[b];
     const LayerDev& Lw = layer_s(p, l);
@@ -1210,7 +1238,7 @@ struct Consumer {
     }
   }
 
-  __device__ __noinline__ void attn_keys(int l, int b, int g, int j, AttnState& S) {
+  __device__ __forceinline__ void attn_keys(int l, int b, int g, int j, AttnState& S) {
     const int rep = p.nq / p.nkv, old = p.pos[b];
     float q[kMaxRep][DQ];
     const int qq = lane & 3;
@@ -1254,7 +1282,7 @@ struct Consumer {
 
   // The new key (position pos, from k_sm / v_sm) on warp 0, then the merge of
   // the warps' states into o_s[b][h][t]. Ends on a barrier.
-  __device__ __noinline__ void attn_finish(int b, int j, AttnState& S) {
+  __device__ __forceinline__ void attn_finish(int b, int j, AttnState& S) {
     const int rep = p.nq / p.nkv, d = 4 * DQ, qq = lane & 3, kk = lane >> 2;
     if (warp == 0 && !warp_quit()) {
       float s[kMaxRep];
@@ -1361,7 +1389,7 @@ struct Consumer {
       for (int e = 0; e < 4; ++e) acc4[b][e] = fmaf(s[b], w[e], acc4[b][e]);
   }
 
-  __device__ __noinline__ void phase_b(int l) {
+  __device__ __forceinline__ void phase_b(int l) {
     tr(l, 3);
     const int d = p.d, ds = d / kSlice, rep = p.nq / p.nkv, H = p.H;
     for (int u = cta; u < p.n_units; u += G) {
@@ -1424,7 +1452,7 @@ struct Consumer {
 
   // ---- phase C: RMSNorm + gate/up + SwiGLU + down share ------------------
 
-  __device__ __noinline__ void phase_c(int l, int a, int b) {
+  __device__ __forceinline__ void phase_c(int l, int a, int b) {
     tr(l, 7);
     const LayerDev& Lw = layer_s(p, l);
     float gr[kEPT];
@@ -1533,7 +1561,7 @@ struct Consumer {
 
   // ---- tail: final norm + LM head + greedy, or the block output -----------
 
-  __device__ __noinline__ void tail(int a, int b) {
+  __device__ __forceinline__ void tail(int a, int b) {
     const int L = p.L;
     tr(L, 0);
     float gr[kEPT];
@@ -1589,7 +1617,7 @@ struct Consumer {
   }
 
   // Fold this CTA's greedy keys; the last CTA to finish writes the ids.
-  __device__ __noinline__ void finish_head() {
+  __device__ __forceinline__ void finish_head() {
     if (tid < kMaxB) best[tid] = 0ull;
     consumer_sync();
 #pragma unroll
@@ -1636,6 +1664,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   ring.n = p.n_stages;
   ring.full = reinterpret_cast<uint64_t*>(smem + p.off_bar);
   ring.empty = ring.full + kMaxStages;
+  // The phases read the parameters through a reference; a reference to the
+  // kernel's parameter space makes every such read a long-latency generic
+  // load, so they read a copy in shared memory instead.
+  Params* ps = reinterpret_cast<Params*>(smem + p.off_par);
+  for (int k = threadIdx.x; k < (int)(sizeof(Params) / 4); k += blockDim.x)
+    reinterpret_cast<unsigned*>(ps)[k] = reinterpret_cast<const unsigned*>(&p)[k];
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.n_stages; ++s) {
       mbar_init(&ring.full[s], 1);
@@ -1676,7 +1710,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
       reinterpret_cast<volatile unsigned int*>(smem + p.off_misc + 4096 + 8 * kMaxB + 8);
   if (warp == kConsumerWarps) {
     if (lane == 0) {
-      Producer pr(p, ring);
+      Producer pr(*ps, ring);
       for (int l = p.l0; l < p.l1 && !pr.quit; ++l) {
         int a, b;
         slice(qkvd, G, c, a, b);
@@ -1692,7 +1726,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
       counts[0] = pr.i;
     }
   } else {
-    Consumer<NB, Q8W, IT, DQ> cs(p, ring, smem);
+    Consumer<NB, Q8W, IT, DQ> cs(*ps, ring, smem);
     // `quit` is per thread (a wait that gave up), so it must not steer any
     // path that holds a consumer barrier: after an abort every thread still
     // walks all phases, with each wait returning at once and no stores.
@@ -2018,7 +2052,8 @@ fs_status decode_fused(fs_model* m, const fs_kv* kv, const RowMap& map, int B, c
   const size_t red = align_up(std::max((size_t)(std::max(p.n_units, st->sms) + 4) * emax * 4,
                                        (size_t)3 * (s.H / 128) * 64 * 4),
                               128);
-  const size_t fixed = rows_bytes + zs_bytes + zt_bytes + misc + attn + tab + bars + red;
+  const size_t par = align_up(sizeof(fused::Params), 128);
+  const size_t fixed = rows_bytes + zs_bytes + zt_bytes + misc + attn + tab + bars + red + par;
   const size_t budget = 232448;
   p.stage_bytes = m->q8 ? fused::kStageQ8 : fused::kStageBf16;
   int n_stages = (int)((budget - fixed) / (size_t)p.stage_bytes);
@@ -2033,6 +2068,7 @@ fs_status decode_fused(fs_model* m, const fs_kv* kv, const RowMap& map, int B, c
   p.off_bar = (int)off; off += bars;
   p.off_tab = (int)off; off += tab;
   p.off_red = (int)off; off += red;
+  p.off_par = (int)off; off += par;
   p.bt_in_smem = bt_smem ? 1 : 0;
   p.n_stages = n_stages;
   // A warp that consumes only every lm_owners-th chunk tests the release of

@@ -29,7 +29,10 @@ SLOTS = {  # cooperative kernel
     2: [(0, "block begins"), (1, "block input exchanged"), (2, "QKV rows done"),
         (3, "q/k/v exchanged, normed, rotated"), (4, "keys done, states sent"),
         (5, "attention merged and exchanged"), (6, "O shares published"),
-        (7, "MLP input exchanged"), (8, "gate/up + SwiGLU done"),
+        (7, "MLP input exchanged"), (12, "first gate/up pass: chunks in"),
+        (11, "  product starts"), (14, "  warp 0 items done"), (15, "  all items done"),
+        (13, "first gate/up pass: product done"),
+        (8, "gate/up + SwiGLU done"),
         (9, "activations exchanged"), (10, "down shares published")],
 }
 HOPS = {
