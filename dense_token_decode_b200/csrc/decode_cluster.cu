@@ -559,6 +559,7 @@ struct Consumer {
   bool quit = false;
   unsigned int xk = 0;  // exchanges done
   int cur_layer = 0;    // for trace stamps
+  unsigned int grp = 0;  // owner-mode chunk groups so far (the owner of the next one is grp % W)
   int tid, warp, lane, cta, cl, g, hs, rk, G;
   float inv[NB];
   unsigned long long wbest[kMaxB] = {0ull, 0ull, 0ull, 0ull};
@@ -594,19 +595,14 @@ struct Consumer {
   __device__ float* act() { return reinterpret_cast<float*>(sm + p.off_act); }  // [B][nc]
   __device__ float* ssc() { return reinterpret_cast<float*>(sm + p.off_ssc); }  // [rep][64] + run state
   __device__ float* ys() { return reinterpret_cast<float*>(sm + p.off_ys); }    // [128][4]
-  __device__ float* red() { return reinterpret_cast<float*>(sm + p.off_red); }
+  __device__ float* red() { return reinterpret_cast<float*>(sm + p.off_red); }  // exchange sums
   __device__ float* ssp() { return reinterpret_cast<float*>(sm + p.off_ss); }   // [11][kMaxB]
-  // misc (bytes): zero bytes 0..64, greedy keys 64..96, flag 96, counts 104,
-  // the row tables from 128.
+  // misc (bytes): zero bytes 0..64, greedy keys 64..96, flag 96, counts 104.
   __device__ uint32_t zero_addr() { return su32(sm + p.off_misc); }  // 64 zero bytes
   __device__ unsigned long long* best() {
     return reinterpret_cast<unsigned long long*>(sm + p.off_misc + 64);
   }
   __device__ int* flag() { return reinterpret_cast<int*>(sm + p.off_misc + 96); }
-  // [128] shared address of each row of a phase's product (| row mod 8: its swizzle)
-  __device__ uint32_t* rowaddr() { return reinterpret_cast<uint32_t*>(sm + p.off_misc + 128); }
-  // [128] Q8_0: shared address of each row's scales
-  __device__ uint32_t* scaleaddr() { return reinterpret_cast<uint32_t*>(sm + p.off_misc + 640); }
   __device__ uint64_t* xbar() { return r.empty + kMaxStages; }  // [2] exchange barriers
 
   // ---- ring --------------------------------------------------------------
@@ -660,14 +656,25 @@ struct Consumer {
   }
   // Owner-mode wait of the LM head (this warp alone consumes the chunk): the
   // release of the chunk a ring earlier in the same stage, then the chunk.
-  __device__ __forceinline__ const unsigned char* chunk_wait_owned() {
-    const int s = stage;
-    if (!__all_sync(0xffffffffu, quit || (mbar_test(&r.empty[s], parity ^ 1u) &&
-                                          mbar_test(&r.full[s], parity))) &&
-        warp_wait_slow(&r.full[s], parity, &r.empty[s], parity ^ 1u, quit, p.wait_ns,
-                       p.abort_flag))
+  __device__ __forceinline__ const unsigned char* chunk_wait_owned(int ahead = 0) {
+    int s = stage + ahead;
+    uint32_t par = parity;
+    if (s >= r.n) {
+      s -= r.n;
+      par ^= 1u;
+    }
+    if (!__all_sync(0xffffffffu, quit || (mbar_test(&r.empty[s], par ^ 1u) &&
+                                          mbar_test(&r.full[s], par))) &&
+        warp_wait_slow(&r.full[s], par, &r.empty[s], par ^ 1u, quit, p.wait_ns, p.abort_flag))
       give_up();
     return r.stages + (size_t)s * kStage;
+  }
+  // Owner-mode release of the chunk `ahead` places after the cursor.
+  __device__ __forceinline__ void chunk_release_owned(int ahead) {
+    int s = stage + ahead;
+    if (s >= r.n) s -= r.n;
+    __syncwarp();
+    if (lane == 0 && !quit) mbar_arrive_n(&r.empty[s], kConsumerWarps);
   }
 
   // ---- cluster exchanges ---------------------------------------------------
@@ -824,62 +831,64 @@ struct Consumer {
     return v;
   }
 
-  // ys[j * 4 + b] = sum_k W[j][k] x_b[k] for the R rows (R <= 128) of a
-  // phase, K a multiple of 64, row j's data at rowaddr()[j] (16-byte units
-  // stored as swz() places them): A = the rows (16-row tiles), B = the 2B
-  // operand rows at `ob` (stride `ostride` bytes): column 2b + t of the
-  // product is term t of batch row b. Work items are (row tile, block of 64
-  // columns), warp w taking items w, w + 11, ...; the items' partial sums are
-  // added in a fixed order. Ends on a barrier.
-  __device__ __forceinline__ void mma_rows(int R, int K, uint32_t ob, uint32_t ostride, int y0,
-                                        bool stamp = false) {
-    const uint32_t* ra = rowaddr();
-    float* part = red();
-    const int nkb = K / 64, mt = (R + 15) / 16, items = mt * nkb, twoB = 2 * p.B;
+  // All rows of one or two chunks (nr rows of K, phase rows j0 ..; rows
+  // [0, cap) at shared address st, the rest at st2 (bf16 only); j0 a multiple
+  // of 8, so row r has swizzle r mod 8) on this warp,
+  // over the whole K: ys[(j0 + r) * 4 + b] = sum_k W[r][k] x_b[k]. A = 16-row
+  // tiles of the chunk (rows past nr read zeros), B = the 2B operand rows at
+  // `ob` (column 2b + t = term t of batch row b); loads of 4 k-steps are
+  // issued before their products.
+  __device__ __forceinline__ void chunk_rows(uint32_t st, uint32_t st2, int cap, int j0, int nr,
+                                             int K, uint32_t ob, uint32_t ostride) {
+    const int gq = lane >> 2, q = lane & 3, twoB = 2 * p.B;
     const uint32_t zero = zero_addr();
-    const int gq = lane >> 2, q = lane & 3;
-    for (int it = warp; it < items; it += kConsumerWarps) {
-      const int m = it / nkb, kb0 = (it % nkb) * 4;  // first k-step of the item
-      float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+    float* y = ys();
+    for (int t0 = 0; t0 < nr; t0 += 16) {
+      float d[4][4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) d[c][0] = d[c][1] = d[c][2] = d[c][3] = 0.f;
       if constexpr (!Q8) {
-        const int row = m * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-        const bool arow = row < R;
-        const uint32_t rv = arow ? ra[row] : 0u, rb = rv & ~15u, sw = rv & 7u;
+        const int row = t0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const bool arow = row < nr;
+        const uint32_t rb = (row < cap ? st + (uint32_t)row * 2u * K
+                                       : st2 + (uint32_t)(row - cap) * 2u * K),
+                       sw = (uint32_t)(row & 7);
         const int n = lane & 7;
         const bool brow = n < twoB;
-        uint32_t baddr = brow ? ob + n * ostride + (((lane >> 3) & 1) << 4) + kb0 * 32 : zero;
+        const uint32_t bb = brow ? ob + n * ostride + (((lane >> 3) & 1) << 4) : zero;
         const uint32_t bstep = brow ? 32u : 0u;
+        for (int ks = 0; ks < K / 16; ks += 4) {
+          uint32_t a[4][4], b[4][2];
 #pragma unroll
-        for (int ks = 0; ks < 4; ks += 2) {
-          const uint32_t u = (uint32_t)((kb0 + ks) * 2 + (lane >> 4));
-          uint32_t a[4], b[2], a2[4], b2[2];
-          ldsm_x4(arow ? rb + ((u ^ sw) << 4) : zero, a);
-          ldsm_x2(baddr, b);
-          ldsm_x4(arow ? rb + (((u + 2) ^ sw) << 4) : zero, a2);
-          ldsm_x2(baddr + bstep, b2);
-          mma16816(d0, a, b);
-          mma16816(d1, a2, b2);
-          baddr += 2 * bstep;
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t u = (uint32_t)((ks + j) * 2 + (lane >> 4));
+            ldsm_x4(arow ? rb + ((u ^ sw) << 4) : zero, a[j]);
+            ldsm_x2(bb + (uint32_t)(ks + j) * bstep, b[j]);
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) mma16816(d[j], a[j], b[j]);
         }
       } else {
-        // Q8_0: 2 blocks of 32 columns; each thread takes 8 consecutive codes
-        // of rows gq and gq + 8 (columns 32 blk + 8 q ..) and the same 8
-        // operand columns, a column order that both operands share. Each
-        // block's product is scaled by its rows' scales.
-        const int r0 = m * 16 + gq, r1 = r0 + 8;
-        const bool h0 = r0 < R, h1 = r1 < R, hb = gq < twoB;
-        const uint32_t v0 = h0 ? ra[r0] : 0u, v1 = h1 ? ra[r1] : 0u;
-        const uint32_t s0a = h0 ? scaleaddr()[r0] : 0u, s1a = h1 ? scaleaddr()[r1] : 0u;
+        // Q8_0: each thread takes 8 consecutive codes of rows gq and gq + 8
+        // (columns 32 blk + 8 q ..) and the same 8 operand columns, a column
+        // order both operands share; each 32-column block's product is scaled
+        // by its rows' scales.
+        const int r0 = t0 + gq, r1 = r0 + 8;
+        const bool h0 = r0 < nr, h1 = r1 < nr, hb = gq < twoB;
+        const uint32_t c0a = st + (uint32_t)r0 * K, c1a = st + (uint32_t)r1 * K;
+        const uint32_t sca = st + (uint32_t)nr * K;  // the chunk's scales follow its codes
+        const uint32_t s0a = sca + (uint32_t)r0 * (K / 16), s1a = sca + (uint32_t)r1 * (K / 16);
         const int units = K / 16;  // rows r0 and r1 are both gq mod 8
-        const uint32_t bb = ob + gq * ostride;
+        const uint32_t bbq = ob + gq * ostride + q * 16;
+        const uint32_t half = (uint32_t)(q & 1) * 8u;
+        for (int blk0 = 0; blk0 < K / 32; blk0 += 2) {  // K / 32 is even
 #pragma unroll
-        for (int bi = 0; bi < 2; ++bi) {
-          const int blk = kb0 / 2 + bi;
+        for (int jb = 0; jb < 2; ++jb) {
+          const int blk = blk0 + jb;
           const uint32_t u = (uint32_t)swz(blk * 2 + (q >> 1), gq, units);
-          const uint32_t half = (uint32_t)(q & 1) * 8u;
-          const uint2 c0 = h0 ? lds64((v0 & ~15u) + (u << 4) + half) : make_uint2(0u, 0u);
-          const uint2 c1 = h1 ? lds64((v1 & ~15u) + (u << 4) + half) : make_uint2(0u, 0u);
-          const uint4 z = hb ? lds128(bb + (uint32_t)(blk * 64 + q * 16)) : make_uint4(0u, 0u, 0u, 0u);
+          const uint2 c0 = h0 ? lds64(c0a + (u << 4) + half) : make_uint2(0u, 0u);
+          const uint2 c1 = h1 ? lds64(c1a + (u << 4) + half) : make_uint2(0u, 0u);
+          const uint4 z = hb ? lds128(bbq + (uint32_t)blk * 64u) : make_uint4(0u, 0u, 0u, 0u);
           const uint32_t a0[4] = {i8x2_bf16(c0.x, 0), i8x2_bf16(c1.x, 0), i8x2_bf16(c0.x, 1),
                                   i8x2_bf16(c1.x, 1)};
           const uint32_t a1[4] = {i8x2_bf16(c0.y, 0), i8x2_bf16(c1.y, 0), i8x2_bf16(c0.y, 1),
@@ -890,54 +899,53 @@ struct Consumer {
           mma16816(e, a1, b1);
           const float sc0 = h0 ? lds_half(s0a + blk * 2) : 0.f;
           const float sc1 = h1 ? lds_half(s1a + blk * 2) : 0.f;
-          d0[0] = fmaf(sc0, e[0], d0[0]);
-          d0[1] = fmaf(sc0, e[1], d0[1]);
-          d0[2] = fmaf(sc1, e[2], d0[2]);
-          d0[3] = fmaf(sc1, e[3], d0[3]);
+          d[jb][0] = fmaf(sc0, e[0], d[jb][0]);
+          d[jb][1] = fmaf(sc0, e[1], d[jb][1]);
+          d[jb][2] = fmaf(sc1, e[2], d[jb][2]);
+          d[jb][3] = fmaf(sc1, e[3], d[jb][3]);
+        }
         }
       }
-      part[(it * 16 + gq) * 4 + q] = (d0[0] + d1[0]) + (d0[1] + d1[1]);
-      part[(it * 16 + gq + 8) * 4 + q] = (d0[2] + d1[2]) + (d0[3] + d1[3]);
+      // rows gq (d[.][0..1]) and gq + 8 (d[.][2..3]); columns 2q (hi), 2q + 1 (lo)
+      const float lo_row = ((d[0][0] + d[1][0]) + (d[2][0] + d[3][0])) +
+                           ((d[0][1] + d[1][1]) + (d[2][1] + d[3][1]));
+      const float hi_row = ((d[0][2] + d[1][2]) + (d[2][2] + d[3][2])) +
+                           ((d[0][3] + d[1][3]) + (d[2][3] + d[3][3]));
+      if (q < p.B) {
+        if (t0 + gq < nr) y[(j0 + t0 + gq) * 4 + q] = lo_row;
+        if (t0 + gq + 8 < nr) y[(j0 + t0 + gq + 8) * 4 + q] = hi_row;
+      }
     }
-    if (stamp) tr(cur_layer, 14);
-    consumer_sync();
-    if (stamp) tr(cur_layer, 15);
-    float* y = ys() + y0 * 4;
-    for (int t = tid; t < R * 4; t += kConsumers) {
-      const int rr = (t >> 2) & 15, q2 = t & 3, m = t >> 6;
-      float sum = 0.f;
-      for (int kb = 0; kb < nkb; ++kb) sum += part[((m * nkb + kb) * 16 + rr) * 4 + q2];
-      y[t] = sum;
-    }
-    consumer_sync();
   }
 
-  // The rows of phase `ph` (spread over the next chunks) into ys: in passes
-  // of the chunks that hold two 16-row tiles (at least one chunk), each pass
-  // waiting for its chunks, filling the row tables, running the product of
-  // its rows and releasing the chunks at once, so the producer refills the
-  // ring while the later passes run.
+  // The rows of phase `ph` into ys, chunk by chunk: chunk i of the ring goes
+  // to warp i mod lm_owners, which waits for it, computes all its rows over
+  // the whole K and releases it at once; the other warps only advance their
+  // cursor. No CTA barrier until the phase's end, so the products overlap the
+  // copies of the next chunks. Ends on a barrier.
+  //
+  // Chunks of 8 rows go to their owner in pairs (one full 16-row tile); the
+  // owners of pairs are at most half a ring of warps, so a warp's owned
+  // chunks stay within a ring of each other (the condition under which the
+  // owner-mode wait cannot mistake an older phase of a barrier).
   __device__ void rows_product(int ph, uint32_t ob, uint32_t ostride) {
     const int R = p.geo.n[ph], Kp = p.geo.K[ph], cap = cap_rows(Kp, Q8), nch = (R + cap - 1) / cap;
-    const int rb = Q8 ? Kp : 2 * Kp, pass = min(min(nch, r.n - 2), max(1, 32 / cap));
-    for (int c0 = 0; c0 < nch; c0 += pass) {
-      const int np = min(pass, nch - c0), j0 = c0 * cap, rows = min(R, (c0 + np) * cap) - j0;
-      for (int c = 0; c < np; ++c) chunk_wait(c);
-      if (ph == kPGU && c0 == 0) tr(cur_layer, 12);
-      if (warp == 0)
-        for (int jj = lane; jj < rows; jj += 32) {
-          const int j = j0 + jj, c = j / cap, slot = j - c * cap;  // chunk and row slot
-          const uint32_t st = stage_addr(c - c0);
-          rowaddr()[jj] = (st + slot * rb) | (uint32_t)(j & 7);
-          if (Q8) scaleaddr()[jj] = st + min(cap, R - c * cap) * Kp + slot * (Kp / 16);
-        }
-      consumer_sync();
-      const bool stamp = ph == kPGU && c0 == 0;
-      if (stamp) tr(cur_layer, 11);
-      mma_rows(rows, Kp, ob, ostride, j0, stamp);
-      if (stamp) tr(cur_layer, 13);
-      for (int c = 0; c < np; ++c) chunk_release();
+    const int per = (!Q8 && cap < 16) ? 2 : 1;
+    const int W = per == 1 ? p.lm_owners : max(1, min(p.lm_owners, r.n / 2));
+    for (int c = 0; c < nch; c += per) {
+      const int ng = min(per, nch - c);
+      if ((int)(grp % (unsigned)W) == warp) {
+        const unsigned char* st = chunk_wait_owned(0);
+        const unsigned char* st2 = ng > 1 ? chunk_wait_owned(1) : st;
+        const int j0 = c * cap;
+        if (!warp_quit())
+          chunk_rows(su32(st), su32(st2), cap, j0, min(ng * cap, R - j0), Kp, ob, ostride);
+        for (int g2 = 0; g2 < ng; ++g2) chunk_release_owned(g2);
+      }
+      for (int g2 = 0; g2 < ng; ++g2) cursor_advance();
+      ++grp;
     }
+    consumer_sync();
   }
 
   __device__ __forceinline__ void tr(int layer, int k) {

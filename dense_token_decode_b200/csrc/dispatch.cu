@@ -8,11 +8,13 @@ namespace fs {
 fs_status init_extras(fs_model* m) {
   fs_status s = fused_init(m);
   if (s != FS_OK) return s;
+  if ((s = mega_init(m)) != FS_OK) return s;
   return cluster_init(m);
 }
 
 void release_extras(fs_model* m) {
   cluster_release(m);
+  mega_release(m);
   fused_release(m);
   tc_release(m);
 }
@@ -20,11 +22,17 @@ void release_extras(fs_model* m) {
 fs_status decode_persistent(fs_model* m, const fs_kv* kv, const RowMap& map, int B,
                             const int32_t* tok, const float* h_in, float* h_out, int l0, int l1,
                             bool run_head, float* logits, int32_t* argmax, cudaStream_t stream) {
-  if (m->decode_path == 2) return FS_ERR_UNSUPPORTED;
-  if (m->decode_path == 0) {
+  const int path = m->decode_path;
+  if (path == 2) return FS_ERR_UNSUPPORTED;
+  if (path == 3 || (path == 0 && B == 1)) {
+    fs_status s = decode_mega(m, kv, map, B, tok, h_in, h_out, l0, l1, run_head, logits, argmax,
+                              stream);
+    if (s != FS_ERR_UNSUPPORTED || path == 3) return s;
+  }
+  if (path == 0 || path == 4) {
     fs_status s = decode_cluster(m, kv, map, B, tok, h_in, h_out, l0, l1, run_head, logits,
                                  argmax, stream);
-    if (s != FS_ERR_UNSUPPORTED) return s;
+    if (s != FS_ERR_UNSUPPORTED || path == 4) return s;
   }
   return decode_fused(m, kv, map, B, tok, h_in, h_out, l0, l1, run_head, logits, argmax, stream);
 }

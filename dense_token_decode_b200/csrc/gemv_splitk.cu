@@ -1,108 +1,92 @@
 // Weight-streaming linear layer for 5..16 rows (batched decode, bf16
-// weights): y[r, n] (+)= sum_k x[r, k] W[n, k], on the tensor cores.
+// weights): y[r, n] (+)= sum_k x[r, k] W[n, k].
 //
-// A CTA (4 warps) owns 64 weight rows and a 256-column slice of the input
-// axis (many CTAs per SM keep HBM busy). It stages the slice of every batch
-// row in shared
-// memory as two bf16 terms (hi = bf16(x), lo = bf16(x - hi)), so each product
-// keeps about 16 bits of the fp32 activation; rows 2r and 2r + 1 of the
-// operand hold the terms of batch row r. Each warp then streams its 16
-// weight rows straight from global memory: per 32-column block a thread
-// loads 8 consecutive weights of rows g and g + 8 (g = lane / 4, at column
-// 32 blk + 8 (lane % 4)) and the same 8 columns of operand rows, an order of
-// the columns that both operands share, and issues mma.sync m16n8k16 (bf16
-// in, fp32 accumulate) for the four 8-column tiles of the 32 operand rows.
-// The first weight loads are issued before the staging, and loads run
-// several blocks ahead of the products. Slices of the input axis are
-// combined with fp32 atomics.
+// One warp owns 8 weight rows and a 256-wide slice of the input axis: every
+// lane loads 8 consecutive bf16 weights of each of the 8 rows (16-byte loads,
+// 512 contiguous bytes per row per warp) and the matching 8 activations of
+// each batch row, so an activation load serves 8 weight rows and a weight
+// load serves every batch row. The 8 x R partial sums are reduced across the
+// warp by a transposing butterfly (4 sums per lane at the end) and added
+// into y with fp32 atomics, which combine the slices of the input axis.
+// Many short warps keep enough weight bytes in flight to stream HBM.
 #include "fs_internal.h"
 
 namespace fs {
 
 namespace {
 
+constexpr int kRowsPerWarp = 8;
+constexpr int kSlice = 256;  // input-axis slice of one warp
 constexpr int kWarps = 4;
-constexpr int kRowsPerCta = 16 * kWarps;
-constexpr int kSlice = 256;   // input-axis slice of one CTA
-constexpr int kOpStride = kSlice + 8;  // bf16 per operand row in shared memory
-constexpr int kAhead = 4;     // 32-column blocks of weights in flight per thread
 
-__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4],
-                                         const uint32_t (&b)[2]) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
+__device__ __forceinline__ float lo16(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float hi16(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
 
-__global__ void __launch_bounds__(kWarps * 32) gemv_mma_kernel(
-    const float* __restrict__ x, int rows, int K, const __nv_bfloat16* __restrict__ W, int N,
-    float* __restrict__ out, int ldo) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(smem);  // [32][kOpStride]
-  const int k0 = blockIdx.y * kSlice, ks = min(kSlice, K - k0);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int g = lane >> 2, q = lane & 3;
-  const int n0 = blockIdx.x * kRowsPerCta + warp * 16;
-  const int ra = min(n0 + g, N - 1), rb = min(n0 + g + 8, N - 1);  // rows past N: dropped below
-  const uint4* wa = reinterpret_cast<const uint4*>(W + (size_t)ra * K + k0 + 8 * q);
-  const uint4* wb = reinterpret_cast<const uint4*>(W + (size_t)rb * K + k0 + 8 * q);
-  const int nblk = ks / 32;
-  uint4 pa[kAhead], pb[kAhead];
+// Transposing butterfly over the warp: 128 partial sums per lane in, the
+// warp totals of 4 of them per lane out. Rounds with masks 16, 8, 4, 2, 1
+// halve the values a lane keeps (64, 32, 16, 8, 4); afterwards lane l holds
+// in v[q] the total of index 64*b4 + 32*b3 + 16*b2 + 8*b1 + 4*b0 + q, with
+// b4..b0 the bits of l.
+__device__ __forceinline__ void reduce128(float (&v)[128], int lane) {
 #pragma unroll
-  for (int i = 0; i < kAhead; ++i) {
-    pa[i] = i < nblk ? __ldg(wa + i * 4) : make_uint4(0u, 0u, 0u, 0u);
-    pb[i] = i < nblk ? __ldg(wb + i * 4) : make_uint4(0u, 0u, 0u, 0u);
-  }
-  // stage the operand: 32 rows (hi, lo of 16 batch rows; absent rows zero)
-  for (int i = threadIdx.x; i < 16 * ks; i += blockDim.x) {
-    const int r = i / ks, k = i - r * ks;
-    const float v = r < rows ? x[(size_t)r * K + k0 + k] : 0.f;
-    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-    op[(2 * r) * kOpStride + k] = hi;
-    op[(2 * r + 1) * kOpStride + k] = __float2bfloat16_rn(v - __bfloat162float(hi));
-  }
-  __syncthreads();
-  if (n0 >= N) return;
-  const uint32_t opb = (uint32_t)__cvta_generic_to_shared(op) + (uint32_t)(g * kOpStride + 8 * q) * 2;
-  float acc[4][4];
+  for (int w = 64, mask = 16; w >= 4; w >>= 1, mask >>= 1) {
+    const bool upper = (lane & mask) != 0;
 #pragma unroll
-  for (int t = 0; t < 4; ++t)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
-  for (int blk0 = 0; blk0 < nblk; blk0 += kAhead) {
-#pragma unroll
-    for (int i = 0; i < kAhead; ++i) {
-      const int blk = blk0 + i;
-      if (blk >= nblk) break;
-      const uint4 a = pa[i], b = pb[i];
-      if (blk + kAhead < nblk) {
-        pa[i] = __ldg(wa + (blk + kAhead) * 4);
-        pb[i] = __ldg(wb + (blk + kAhead) * 4);
-      }
-      // k-step 0 takes columns 8q .. 8q+3 of the block, k-step 1 8q+4 .. 8q+7
-      const uint32_t a0[4] = {a.x, b.x, a.y, b.y}, a1[4] = {a.z, b.z, a.w, b.w};
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        uint4 z;
-        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(z.x), "=r"(z.y), "=r"(z.z), "=r"(z.w)
-                     : "r"(opb + (uint32_t)(t * 8 * kOpStride + blk * 32) * 2));
-        const uint32_t b0[2] = {z.x, z.y}, b1[2] = {z.z, z.w};
-        mma16816(acc[t], a0, b0);
-        mma16816(acc[t], a1, b1);
-      }
+    for (int i = 0; i < w; ++i) {
+      const float send = upper ? v[i] : v[i + w];
+      const float keep = upper ? v[i + w] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
     }
   }
-  // acc[t]: rows g (e 0, 1) and g + 8 (e 2, 3) of the warp's 16, operand
-  // columns 8t + 2q (hi) and 8t + 2q + 1 (lo): batch row 4t + q
+}
+
+template <int R>
+__global__ void __launch_bounds__(kWarps * 32) gemv_splitk_kernel(
+    const float* __restrict__ x, int rows, int K, const __nv_bfloat16* __restrict__ W, int N,
+    float* __restrict__ out, int ldo) {
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * kWarps + (threadIdx.x >> 5);
+  const int slices = K / kSlice;
+  const int n_groups = (N + kRowsPerWarp - 1) / kRowsPerWarp;
+  if (gw >= n_groups * slices) return;
+  const int grp = gw / slices, sl = gw % slices;
+  const int n0 = grp * kRowsPerWarp;
+  const int k = sl * kSlice + lane * 8;
+
+  uint4 w[kRowsPerWarp];
 #pragma unroll
-  for (int t = 0; t < 4; ++t) {
-    const int r = 4 * t + q;
-    if (r >= rows) continue;
-    if (n0 + g < N) atomicAdd(out + (size_t)r * ldo + n0 + g, acc[t][0] + acc[t][1]);
-    if (n0 + g + 8 < N) atomicAdd(out + (size_t)r * ldo + n0 + g + 8, acc[t][2] + acc[t][3]);
+  for (int j = 0; j < kRowsPerWarp; ++j) {
+    const int n = min(n0 + j, N - 1);  // rows past N repeat the last one; dropped below
+    w[j] = __ldg(reinterpret_cast<const uint4*>(W + (size_t)n * K + k));
+  }
+  float v[128];
+#pragma unroll
+  for (int i = 0; i < 128; ++i) v[i] = 0.f;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    if (r >= rows) break;
+    const float4 a = __ldg(reinterpret_cast<const float4*>(x + (size_t)r * K + k));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(x + (size_t)r * K + k + 4));
+#pragma unroll
+    for (int j = 0; j < kRowsPerWarp; ++j) {
+      float s = lo16(w[j].x) * a.x;
+      s = fmaf(hi16(w[j].x), a.y, s);
+      s = fmaf(lo16(w[j].y), a.z, s);
+      s = fmaf(hi16(w[j].y), a.w, s);
+      s = fmaf(lo16(w[j].z), b.x, s);
+      s = fmaf(hi16(w[j].z), b.y, s);
+      s = fmaf(lo16(w[j].w), b.z, s);
+      s = fmaf(hi16(w[j].w), b.w, s);
+      v[r * 8 + j] = s;
+    }
+  }
+  reduce128(v, lane);
+  const int base = ((lane >> 4) & 1) * 64 + ((lane >> 3) & 1) * 32 + ((lane >> 2) & 1) * 16 +
+                   ((lane >> 1) & 1) * 8 + (lane & 1) * 4;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int idx = base + q, r = idx >> 3, j = idx & 7;
+    if (r < rows && n0 + j < N) atomicAdd(out + (size_t)r * ldo + n0 + j, v[q]);
   }
 }
 
@@ -162,7 +146,7 @@ cudaError_t launch_argmax_rows(const float* logits, int rows, int V, int32_t* ar
 }
 
 bool gemv_splitk_ok(int rows, int K, const __half* scales) {
-  return scales == nullptr && rows >= 1 && rows <= 16 && K % 32 == 0;
+  return scales == nullptr && rows >= 1 && rows <= 16 && K % kSlice == 0;
 }
 
 // y (+)= x W^T over `rows` rows; out rows are ldo floats apart. Without
@@ -175,15 +159,10 @@ cudaError_t launch_gemv_splitk(const float* x, int rows, int K, const __nv_bfloa
                                       rows, st);
     if (e != cudaSuccess) return e;
   }
-  static bool attr = false;
-  const int smem = 32 * kOpStride * 2;
-  if (!attr) {
-    cudaFuncSetAttribute(gemv_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    attr = true;
-  }
-  const dim3 grid((N + kRowsPerCta - 1) / kRowsPerCta, (K + kSlice - 1) / kSlice);
+  const int warps = (N + kRowsPerWarp - 1) / kRowsPerWarp * (K / kSlice);
+  const int blocks = (warps + kWarps - 1) / kWarps;
   count_launches();
-  gemv_mma_kernel<<<grid, kWarps * 32, smem, st>>>(x, rows, K, W, N, out, ldo);
+  gemv_splitk_kernel<16><<<blocks, kWarps * 32, 0, st>>>(x, rows, K, W, N, out, ldo);
   return cudaGetLastError();
 }
 

@@ -227,6 +227,7 @@ extern "C" fs_status fs_device_error(fs_model* m, int32_t* code) {
   if (v) {
     fs::fused_reset(m);
     fs::cluster_reset(m);
+    fs::mega_reset(m);
   }
   *code = v;
   return FS_OK;
@@ -753,6 +754,7 @@ fs_status generate_impl(fs_model* m, fs_kv* kv, int32_t seq, const int32_t* prom
     cudaMemset(m->err, 0, sizeof(int));
     fs::fused_reset(m);
     fs::cluster_reset(m);
+    fs::mega_reset(m);
     return fail(FS_ERR_DEVICE, "a kernel reported device error " + std::to_string(derr));
   }
   *n_out = produced;
@@ -891,12 +893,13 @@ extern "C" fs_status fs_debug_wait_limit(fs_model* m, uint64_t wait_ns, int32_t 
     return fail(FS_ERR_INVALID, "withhold_layer must be -1 or a layer index");
   fs::fused_debug_wait(m, wait_ns, withhold_layer);
   fs::cluster_debug_wait(m, wait_ns, withhold_layer);
+  fs::mega_debug_wait(m, wait_ns, withhold_layer);
   return FS_OK;
 }
 
 extern "C" fs_status fs_debug_decode_path(fs_model* m, int32_t path) {
   if (!m) return fail(FS_ERR_NULL, "model is NULL");
-  if (path < 0 || path > 2) return fail(FS_ERR_INVALID, "path must be 0, 1 or 2");
+  if (path < 0 || path > 4) return fail(FS_ERR_INVALID, "path must be 0 .. 4");
   m->decode_path = path;
   return FS_OK;
 }
@@ -905,8 +908,17 @@ extern "C" fs_status fs_debug_decode_kernel(const fs_model* m, int32_t batch, in
   if (!m || !kind) return fail(FS_ERR_NULL, "model or kind is NULL");
   if (batch < 1 || batch > fs::kMaxBatch) return fail(FS_ERR_INVALID, "batch out of range");
   *kind = 0;
-  if (batch <= 4 && m->decode_path != 2)
-    *kind = (m->decode_path == 0 && fs::cluster_eligible(m)) ? 2 : 1;
+  const int path = m->decode_path;
+  if (batch > 4 || path == 2) return FS_OK;
+  if ((path == 3 || (path == 0 && batch == 1)) && fs::mega_eligible(m)) {
+    *kind = 3;
+  } else if (path == 3) {
+    *kind = 0;
+  } else if ((path == 0 || path == 4) && fs::cluster_eligible(m)) {
+    *kind = 2;
+  } else {
+    *kind = path == 4 ? 0 : 1;
+  }
   return FS_OK;
 }
 

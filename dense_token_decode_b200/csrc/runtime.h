@@ -42,6 +42,7 @@ struct fs_model {
   unsigned long long* trace = nullptr;  // armed fs_debug_trace buffer
   void* extras = nullptr;     // persistent decode kernel state
   void* cl_extras = nullptr;  // cluster decode kernel state
+  void* mega_extras = nullptr;  // row-split decode kernel state
   int decode_path = 0;        // fs_debug_decode_path: 0 auto, 1 cooperative kernel, 2 general
   void* tc_extras = nullptr;  // tensor-core prefill state
 };
@@ -94,6 +95,17 @@ void fused_debug_wait(fs_model* m, unsigned long long wait_ns, int withhold_laye
 fs_status decode_fused(fs_model* m, const fs_kv* kv, const RowMap& map, int B, const int32_t* tok,
                        const float* h_in, float* h_out, int l0, int l1, bool run_head,
                        float* logits, int32_t* argmax, cudaStream_t stream);
+
+// Row-split persistent decode kernel (decode_mega.cu): batch 1, the shapes
+// whose ring holds a stage per consumer warp.
+fs_status mega_init(fs_model* m);
+void mega_release(fs_model* m);
+void mega_reset(fs_model* m);
+void mega_debug_wait(fs_model* m, unsigned long long wait_ns, int withhold_layer);
+bool mega_eligible(const fs_model* m);
+fs_status decode_mega(fs_model* m, const fs_kv* kv, const RowMap& map, int B, const int32_t* tok,
+                      const float* h_in, float* h_out, int l0, int l1, bool run_head,
+                      float* logits, int32_t* argmax, cudaStream_t stream);
 
 // Cluster decode kernel (decode_cluster.cu): the same calls for the kernel
 // that runs one 16-CTA cluster per kv head (bf16 weights, 1..4 rows).

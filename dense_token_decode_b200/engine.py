@@ -169,11 +169,11 @@ class Model:
                   "fs_debug_wait_limit")
 
     def decode_path(self, path: int):
-        """0 auto (cluster kernel first), 1 cooperative kernel, 2 general sequence."""
+        """0 auto, 1 cooperative, 2 general sequence, 3 row-split, 4 cluster kernel."""
         abi.check(abi.fs_debug_decode_path(self.handle, path), "fs_debug_decode_path")
 
     def decode_kernel(self, batch: int = 1) -> int:
-        """2 cluster kernel, 1 cooperative kernel, 0 general sequence."""
+        """3 row-split kernel, 2 cluster kernel, 1 cooperative kernel, 0 general sequence."""
         kind = C.c_int32(0)
         abi.check(abi.fs_debug_decode_kernel(self.handle, batch, C.byref(kind)),
                   "fs_debug_decode_kernel")

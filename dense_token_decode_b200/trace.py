@@ -29,10 +29,7 @@ SLOTS = {  # cooperative kernel
     2: [(0, "block begins"), (1, "block input exchanged"), (2, "QKV rows done"),
         (3, "q/k/v exchanged, normed, rotated"), (4, "keys done, states sent"),
         (5, "attention merged and exchanged"), (6, "O shares published"),
-        (7, "MLP input exchanged"), (12, "first gate/up pass: chunks in"),
-        (11, "  product starts"), (14, "  warp 0 items done"), (15, "  all items done"),
-        (13, "first gate/up pass: product done"),
-        (8, "gate/up + SwiGLU done"),
+        (7, "MLP input exchanged"), (8, "gate/up + SwiGLU done"),
         (9, "activations exchanged"), (10, "down shares published")],
 }
 HOPS = {
@@ -64,15 +61,16 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--fmt", default="bf16", choices=["bf16", "q8_0"])
     ap.add_argument("--context", type=int, default=100)
-    ap.add_argument("--path", type=int, default=0, choices=[0, 1],
-                    help="0 the default decode kernel, 1 the cooperative kernel")
+    ap.add_argument("--path", type=int, default=0, choices=[0, 1, 3, 4],
+                    help="0 the default decode path, 1 the cooperative kernel, "
+                         "3 the row-split kernel, 4 the cluster kernel")
     args = ap.parse_args()
     dev = "cuda:0"
     shape = synth.QWEN3_0P6B
     m = Model(shape, synth.model_weights(shape, 1, args.fmt), dev, max_pos=4096)
     m.decode_path(args.path)
     kind = m.decode_kernel(1)
-    print("kernel:", {2: "cluster", 1: "cooperative", 0: "general"}[kind])
+    print("kernel:", {3: "row-split", 2: "cluster", 1: "cooperative", 0: "general"}[kind])
     n = args.context
     kv = m.kv(1, n + 128)
     prompt = synth.token_ids(8, shape.vocab, seed=1).to(dev)
@@ -87,32 +85,35 @@ def main():
     abi.check(abi.fs_debug_trace(m.handle, buf.data_ptr()), "fs_debug_trace")
     m.decode_step(kv, [0], gen[n:n + 1], None, gen[n + 1:n + 2])
     torch.cuda.synchronize()
-    raw = buf.cpu().numpy()
-    t, ghz = to_us(raw, sms, L)
-    print(f"context {n + 8}; SM clock {ghz:.3f} GHz; us from the first QKV start of the layer, "
-          f"median of layers 3..{L - 3}")
-    print(f"{'slot':34s} {'first':>7s} {'median':>7s} {'last':>7s}")
-    # the tail row's slots 12..15 hold the start / end pairs, not phases
-    for k, name in SLOTS.get(kind, []):
-        rows = []
-        for l in range(3, L - 2):
-            col = t[:, l, k]
-            if np.isnan(col).all():
-                continue
-            base = np.nanmin(t[:, l, 0])
-            rows.append((np.nanmin(col) - base, np.nanmedian(col) - base, np.nanmax(col) - base))
-        if rows:
-            a = np.median(np.array(rows), axis=0)
-            print(f"{name:34s} {a[0]:7.2f} {a[1]:7.2f} {a[2]:7.2f}")
-    # hand-offs: the last producer of a phase's input to the median consumer
-    for name, k_from, k_to, dl in HOPS.get(kind, []):
-        v = [np.nanmedian(t[:, l + dl, k_to]) - np.nanmax(t[:, l, k_from]) for l in range(3, L - 2)]
-        print(f"hand-off {name:40s} {np.median(v):6.2f} us")
-    ends = np.nanmax(t[:, :L, 10], axis=0)
-    total = np.nanmax(t[:, L, 4]) - np.nanmin(t[:, 0, 0])
-    print(f"layer time (median) {np.median(np.diff(ends)):.2f} us; tail (final norm, LM head, "
-          f"greedy) {np.nanmax(t[:, L, 4]) - ends[-1]:.2f} us; whole step in the kernel "
-          f"{total:.1f} us")
+    if kind in SLOTS:
+        raw = buf.cpu().numpy()
+        t, ghz = to_us(raw, sms, L)
+        print(f"context {n + 8}; SM clock {ghz:.3f} GHz; us from the first QKV start of the layer, "
+              f"median of layers 3..{L - 3}")
+        print(f"{'slot':34s} {'first':>7s} {'median':>7s} {'last':>7s}")
+        # the tail row's slots 12..15 hold the start / end pairs, not phases
+        for k, name in SLOTS.get(kind, []):
+            rows = []
+            for l in range(3, L - 2):
+                col = t[:, l, k]
+                if np.isnan(col).all():
+                    continue
+                base = np.nanmin(t[:, l, 0])
+                rows.append((np.nanmin(col) - base, np.nanmedian(col) - base, np.nanmax(col) - base))
+            if rows:
+                a = np.median(np.array(rows), axis=0)
+                print(f"{name:34s} {a[0]:7.2f} {a[1]:7.2f} {a[2]:7.2f}")
+        # hand-offs: the last producer of a phase's input to the median consumer
+        for name, k_from, k_to, dl in HOPS.get(kind, []):
+            v = [np.nanmedian(t[:, l + dl, k_to]) - np.nanmax(t[:, l, k_from]) for l in range(3, L - 2)]
+            print(f"hand-off {name:40s} {np.median(v):6.2f} us")
+        ends = np.nanmax(t[:, :L, 10], axis=0)
+        total = np.nanmax(t[:, L, 4]) - np.nanmin(t[:, 0, 0])
+        print(f"layer time (median) {np.median(np.diff(ends)):.2f} us; tail (final norm, LM head, "
+              f"greedy) {np.nanmax(t[:, L, 4]) - ends[-1]:.2f} us; whole step in the kernel "
+              f"{total:.1f} us")
+    else:
+        print("(no phase timeline for this kernel)")
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()

@@ -324,18 +324,22 @@ fs_status fs_debug_trace(fs_model* model, uint64_t* buf);
  * nothing. Errors: FS_ERR_NULL, FS_ERR_INVALID. */
 fs_status fs_debug_wait_limit(fs_model* model, uint64_t wait_ns, int32_t withhold_layer);
 
-/* Debug: which decode path later steps of 1..4 rows take. 0 (default): the
- * cluster kernel (one 16-CTA cluster per kv head; bf16 weights, on shapes and
- * devices it covers), else the cooperative persistent kernel, else the
- * general kernel sequence; 1: the cooperative kernel, else general; 2: the
- * general sequence only. For comparing the paths in tests and benchmarks;
- * every path computes the same forward. Errors: FS_ERR_NULL, FS_ERR_INVALID. */
+/* Debug: which decode path later steps of 1..4 rows take. 0 (default): a
+ * batch of 1 takes the row-split persistent kernel where its weight ring
+ * holds a stage per consumer warp; other batches (and shapes it does not
+ * cover) take the cluster kernel (clusters of 16 or 8 CTAs per kv head, on
+ * shapes and devices it covers), else the cooperative persistent kernel, else
+ * the general kernel sequence; 1: the cooperative kernel, else general; 2:
+ * the general sequence only; 3: the row-split kernel, else general; 4: the
+ * cluster kernel, else general. For comparing the paths in tests and
+ * benchmarks; every path computes the same forward.
+ * Errors: FS_ERR_NULL, FS_ERR_INVALID. */
 fs_status fs_debug_decode_path(fs_model* model, int32_t path);
 
 /* Debug: the kernel a decode step of `batch` rows would use under the current
- * path: *kind = 2 the cluster kernel, 1 the cooperative kernel (if it covers
- * the shape; else the general sequence runs), 0 the general sequence.
- * Errors: FS_ERR_NULL, FS_ERR_INVALID. */
+ * path: *kind = 3 the row-split kernel, 2 the cluster kernel, 1 the
+ * cooperative kernel (if it covers the shape; else the general sequence
+ * runs), 0 the general sequence. Errors: FS_ERR_NULL, FS_ERR_INVALID. */
 fs_status fs_debug_decode_kernel(const fs_model* model, int32_t batch, int32_t* kind);
 
 /* Debug: dequantise Q8_0 blocks to fp32, out[n*k] = codes[n*k] * scales[n*(k/32)]

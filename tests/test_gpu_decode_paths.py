@@ -1,10 +1,10 @@
 """GPU parity of both persistent decode kernels against the oracle.
 
-Decode steps of 1..4 rows run on the cluster kernel (one 16-CTA cluster per
-kv head) by default, and on the cooperative kernel when the cluster kernel
-does not cover the shape or fs_debug_decode_path selects it.
-Each test here runs on both, so neither path goes unchecked while the other
-is the default: teacher-forced decode against the oracle's logits and greedy
+A decode step of one row runs on the row-split persistent kernel by default,
+steps of 2..4 rows on the cluster kernel (clusters of 16 or 8 CTAs per kv
+head), and the cooperative kernel serves what neither covers;
+fs_debug_decode_path selects one. Each test here runs on every kernel that
+serves its batch, so no path goes unchecked while another is the default: teacher-forced decode against the oracle's logits and greedy
 ids, each block alone at a decode position (per-block relative L2 <= 1e-3),
 batches of 2 to 4 in one launch, random RMSNorm gains, Q8_0 weights and the
 bounded-wait error path.
@@ -25,13 +25,14 @@ from test_gpu_parity import (DEV, QWEN_SEED, Pair, _dev_i32, blocks_local_decode
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"cluster": 0, "cooperative": 1}
+PATHS = {"cluster": 4, "cooperative": 1, "row-split": 3}
+KIND = {"cluster": 2, "cooperative": 1, "row-split": 3}
+BATCH_PATHS = ["cluster", "cooperative"]  # the row-split kernel serves batch 1
 
 
 def _use(pair, path):
     pair.model.decode_path(PATHS[path])
-    want = 2 if path == "cluster" else 1
-    assert pair.model.decode_kernel(1) == want, "the decode path did not take the kernel asked for"
+    assert pair.model.decode_kernel(1) == KIND[path], "the decode path did not take its kernel"
 
 
 @pytest.fixture(scope="module")
@@ -85,7 +86,7 @@ def test_qwen_decode_both_kernels(qwen_pair, path):
     qwen_pair.model.decode_path(0)
 
 
-@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("path", BATCH_PATHS)
 @pytest.mark.parametrize("B", [2, 3, 4])
 def test_qwen_batches_both_kernels(qwen_pair, path, B):
     """Batches of 2..4 sequences of different lengths in one launch, rows in
