@@ -28,6 +28,16 @@
 #include "runtime.h"
 #include "tc_common.cuh"
 
+// Terms of the bf16 Q and P operands (2: hi + lo, 1: hi only). Two terms keep
+// about 16 bits of each fp32 value; one term keeps 8 and halves the MMAs of
+// the product it feeds.
+#ifndef FS_ATTN_Q_TERMS
+#define FS_ATTN_Q_TERMS 2
+#endif
+#ifndef FS_ATTN_P_TERMS
+#define FS_ATTN_P_TERMS 2
+#endif
+
 namespace fs {
 namespace attn_tc {
 
@@ -203,8 +213,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int c = kk >> 2, off = (kk & 3) * 32;
             const uint64_t bk = smem_desc(kst + c * 8192 + off);
             mma_f16(tmem + b * kKTile, smem_desc(sQ + c * 16384 + off), bk, id_s, kk > 0 ? 1u : 0u);
-            mma_f16(tmem + b * kKTile, smem_desc(sQ + (Lay::kChunks + c) * 16384 + off), bk, id_s,
-                    1u);
+            if (FS_ATTN_Q_TERMS == 2)
+              mma_f16(tmem + b * kKTile, smem_desc(sQ + (Lay::kChunks + c) * 16384 + off), bk,
+                      id_s, 1u);
           }
           mma_commit(&s_full[b]);
           mma_commit(&k_empty[sk]);
@@ -223,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < kKTile / 16; ++kk) {
             const uint64_t bv = smem_desc(vst + kk * 2048, 8192, 1024);
             mma_f16(t_o, smem_desc(pb + kk * 32), bv, id_pv, (i > 0 || kk > 0) ? 1u : 0u);
-            mma_f16(t_o, smem_desc(pb + 16384 + kk * 32), bv, id_pv, 1u);
+            if (FS_ATTN_P_TERMS == 2) mma_f16(t_o, smem_desc(pb + 16384 + kk * 32), bv, id_pv, 1u);
           }
           mma_commit(&p_free[b]);
           mma_commit(&v_empty[sv]);
