@@ -79,7 +79,7 @@ struct Params {
   int* abort_flag;  // set on a timeout: every wait gives up
   unsigned long long wait_ns;  // limit of every wait
   int withhold_layer;          // debug: the Q/K/V rows of this block are never published
-  unsigned long long* trace;  // optional: %globaltimer stamps [G][L+1][16]
+  unsigned long long* trace;  // optional: clock64 stamps [G][L+1][16]; tail row 12..15 time base
   int n_stages;
   // smem carve-up (bytes)
   int off_hs, off_xs, off_attn, off_bar, off_misc, off_tab;
@@ -416,7 +416,7 @@ struct Producer {
     if (quit) return;
     if (p.trace && phase == kLM) {
       unsigned long long* t = p.trace + ((size_t)blockIdx.x * (p.L + 1) + p.L) * 16;
-      if (!lm_started) t[2] = now_ns();
+      if (!lm_started) t[2] = clock64();
       lm_started = true;
     }
     const bool pair = phase == kGU;
@@ -502,7 +502,7 @@ struct Consumer {
 
   // Timestamp slot k of (this CTA, layer) into the optional trace.
   __device__ void tr(int layer, int k) {
-    if (p.trace && tid == 0) p.trace[((size_t)cta * (p.L + 1) + layer) * 16 + k] = now_ns();
+    if (p.trace && tid == 0) p.trace[((size_t)cta * (p.L + 1) + layer) * 16 + k] = clock64();
   }
 
   __device__ uint32_t tag(int layer, int ph) const {
@@ -870,7 +870,8 @@ struct Consumer {
       n = e;
     }
     if (p.trace && tid == 0 && (ph == kQKV || ph == kLM))
-      p.trace[((size_t)cta * (p.L + 1) + (ph == kLM ? p.L : layer)) * 16 + 8 + ph] = now_ns();
+      p.trace[((size_t)cta * (p.L + 1) + (ph == kLM ? p.L : layer)) * 16 + (ph == kLM ? 6 : 8)] =
+          clock64();
   }
 
   // Output of row n for batch row b (y = the dot product; u = the up row's
@@ -999,6 +1000,7 @@ struct Consumer {
       }
     }
     consumer_sync();
+    tr(layer, 13);
     const int E = d / 32;
     const float scale = 1.f / sqrtf((float)d);
 #pragma unroll
@@ -1158,6 +1160,7 @@ struct Consumer {
 
   __device__ __forceinline__ void attn_end(int layer, int, const Item& x) {
     // No early exit before the first barrier: threads may disagree on quit here.
+    tr(layer, 14);
     const int d = p.d, rep = p.nq / p.nkv, E = d / 32;
     if (x.owner && warp == 0 && !quit) {
       float kk[4] = {0.f, 0.f, 0.f, 0.f}, vv[4] = {0.f, 0.f, 0.f, 0.f};
@@ -1211,6 +1214,7 @@ struct Consumer {
         pp[2 + c] = O;
       }
     }
+    tr(layer, 15);
     if (ns > 1) {
       __threadfence();
       consumer_sync();
@@ -1319,6 +1323,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mega_kernel(const __grid_c
         bt[k] = p.kv.block_table[(size_t)p.seq[k / pps] * pps + k % pps];
     }
   }
+  unsigned long long* trow =
+      p.trace ? p.trace + ((size_t)blockIdx.x * (p.L + 1) + p.L) * 16 : nullptr;
+  if (trow && threadIdx.x == 0) {  // time base: (%globaltimer, clock64) at start and end
+    trow[12] = now_ns();
+    trow[13] = clock64();
+  }
   __syncthreads();
   const int warp = threadIdx.x >> 5;
   if (warp == kConsumerWarps) {
@@ -1326,7 +1336,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mega_kernel(const __grid_c
     if ((threadIdx.x & 31) == 0) {
       Producer pr(p, ring);
       walk(p, blockIdx.x, gridDim.x, pr);
-      if (p.trace) p.trace[((size_t)blockIdx.x * (p.L + 1) + p.L) * 16 + 3] = now_ns();
+      if (p.trace) p.trace[((size_t)blockIdx.x * (p.L + 1) + p.L) * 16 + 3] = clock64();
       reinterpret_cast<volatile unsigned int*>(smem + p.off_misc + 8 * kMaxB + 8)[0] = pr.i;
     }
   } else {
@@ -1350,6 +1360,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mega_kernel(const __grid_c
       const unsigned long long t0 = now_ns();
       while (!mbar_test(&ring.full[k % ring.n], (k / ring.n) & 1))
         if (now_ns() - t0 > 10000000ull) break;  // 10 ms
+    }
+    if (trow) {
+      trow[14] = now_ns();
+      trow[15] = clock64();
     }
   }
 }
@@ -1381,7 +1395,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Keys per attention item of a decode step (the items of a kv head are merged
 // by the last one to finish).
-int kKeysPerSplit = 64;
+constexpr int kKeysPerSplit = 64;
 
 }  // namespace
 

@@ -19,7 +19,15 @@ import torch
 from . import abi, synth
 from .engine import Model
 
-SLOTS = {  # cooperative kernel
+SLOTS = {
+    # row-split kernel
+    3: [(0, "QKV phase begins"), (1, "QKV input loaded"), (8, "QKV rows done"),
+        (12, "attention item begins"), (2, "q/k/v loaded"), (13, "q/k normed, roped, K/V appended"),
+        (14, "item's keys done"), (15, "warps merged"), (9, "attention merged"),
+        (3, "O phase begins"), (4, "O input loaded"), (10, "gate/up phase begins"),
+        (5, "gate/up input loaded"), (11, "down phase begins"), (6, "down input loaded"),
+        (7, "block done")],
+    # cooperative kernel
     1: [(0, "QKV phase begins"), (11, "QKV input slice reduced"), (1, "QKV input loaded"),
         (2, "QKV rows done"), (3, "attention phase begins"), (4, "q/k/v ready"),
         (13, "attention keys done"), (5, "attention merged"), (6, "O share added"),
@@ -33,6 +41,8 @@ SLOTS = {  # cooperative kernel
         (9, "activations exchanged"), (10, "down shares published")],
 }
 HOPS = {
+    3: [("QKV rows -> q/k/v loaded", 8, 2, 0), ("attention merged -> O input loaded", 9, 4, 0),
+        ("block done -> next QKV input loaded", 7, 1, 1)],
     1: [("QKV rows -> q/k/v ready", 2, 4, 0), ("O shares -> MLP slice reduced", 6, 12, 0),
         ("down shares -> next QKV slice reduced", 10, 11, 1)],
     2: [("O shares -> MLP input exchanged", 6, 7, 0),
@@ -61,6 +71,7 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--fmt", default="bf16", choices=["bf16", "q8_0"])
     ap.add_argument("--context", type=int, default=100)
+    ap.add_argument("--dump", default=None, help="save the raw stamps (.npy) to this path")
     ap.add_argument("--path", type=int, default=0, choices=[0, 1, 3, 4],
                     help="0 the default decode path, 1 the cooperative kernel, "
                          "3 the row-split kernel, 4 the cluster kernel")
@@ -87,6 +98,8 @@ def main():
     torch.cuda.synchronize()
     if kind in SLOTS:
         raw = buf.cpu().numpy()
+        if args.dump:
+            np.save(args.dump, raw)
         t, ghz = to_us(raw, sms, L)
         print(f"context {n + 8}; SM clock {ghz:.3f} GHz; us from the first QKV start of the layer, "
               f"median of layers 3..{L - 3}")
@@ -107,13 +120,14 @@ def main():
         for name, k_from, k_to, dl in HOPS.get(kind, []):
             v = [np.nanmedian(t[:, l + dl, k_to]) - np.nanmax(t[:, l, k_from]) for l in range(3, L - 2)]
             print(f"hand-off {name:40s} {np.median(v):6.2f} us")
-        ends = np.nanmax(t[:, :L, 10], axis=0)
-        total = np.nanmax(t[:, L, 4]) - np.nanmin(t[:, 0, 0])
+        end_slot, tail_slot = (7, 7) if kind == 3 else (10, 4)
+        ends = np.nanmax(t[:, :L, end_slot], axis=0)
+        total = np.nanmax(t[:, L, tail_slot]) - np.nanmin(t[:, 0, 0])
         print(f"layer time (median) {np.median(np.diff(ends)):.2f} us; tail (final norm, LM head, "
-              f"greedy) {np.nanmax(t[:, L, 4]) - ends[-1]:.2f} us; whole step in the kernel "
-              f"{total:.1f} us")
+              f"greedy) {np.nanmax(t[:, L, tail_slot]) - ends[-1]:.2f} us; whole step in the "
+              f"kernel {total:.1f} us")
     else:
-        print("(no phase timeline for this kernel)")
+        print("(no phase timeline for the general kernel sequence)")
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()

@@ -296,19 +296,36 @@ fs_status fs_debug_capture(fs_model* model, float* hidden, int32_t max_rows);
 fs_status fs_debug_block(fs_model* model, fs_kv* kv, int32_t seq, int32_t layer,
                          const float* h_in, int32_t rows, float* h_out, void* stream);
 
-/* Debug: the next decode step that runs on the persistent decode kernel
+/* Debug: the next decode step that runs on a persistent decode kernel
  * records timestamps into `buf` (device uint64 [SMs][n_layers+1][16]): per
- * CTA and block the SM's cycle counter (clock64) at slot 0 start of the QKV
- * phase, 11 this CTA's slice of its input reduced, 1 its input loaded, 2 QKV rows done,
- * 3 start of the attention phase, 4 q/k/v of the first batch row ready, 13
- * its keys done, 5 attention merged, 6 O-projection share added, 7 start of
- * the MLP phase, 12 this CTA's slice of its input reduced, 8 its input loaded, 9 gate/up
- * rows done, 10 down share added. Row n_layers holds the tail (0 start, 11
- * slice of its input reduced, 1 input loaded, 2 LM-head rows done, 3 the producer's
- * last copy issued, 4 greedy ids folded) and the CTA's %globaltimer (ns) and
- * cycle counter at kernel start (12, 13) and end (14, 15), which place the
- * cycle stamps on a common time base. Slots a CTA never reaches are left as
- * they were. One-shot; NULL disarms. Timing only: no work changes. */
+ * CTA and block, the SM's cycle counter (clock64) at points of the step. Row
+ * n_layers holds the tail and, in slots 12..15, the CTA's %globaltimer (ns)
+ * and cycle counter at kernel start (12, 13) and end (14, 15), which place the
+ * cycle stamps on a common time base. Slots per kernel (fs_debug_decode_kernel):
+ * cooperative (1): 0 start of the QKV phase, 11 this CTA's slice of its input
+ * reduced, 1 its input loaded, 2 QKV rows done, 3 start of the attention
+ * phase, 4 q/k/v of the first batch row ready, 13 its keys done, 5 attention
+ * merged, 6 O-projection share added, 7 start of the MLP phase, 12 this CTA's
+ * slice of its input reduced, 8 its input loaded, 9 gate/up rows done, 10
+ * down share added; tail 0 start, 11 slice of its input reduced, 1 input
+ * loaded, 2 LM-head rows done, 3 the producer's last copy issued, 4 greedy
+ * ids folded.
+ * cluster (2): 0 block begins, 1 block input exchanged, 2 QKV rows done, 3
+ * q/k/v exchanged, normed and rotated, 4 keys done and states sent, 5
+ * attention merged and exchanged, 6 O shares published, 7 MLP input
+ * exchanged, 8 gate/up and SwiGLU done, 9 activations exchanged, 10 down
+ * shares published; tail 0 start, 1 input exchanged, 2 LM-head rows done, 3
+ * the producer's last copy issued, 4 greedy ids folded.
+ * row-split (3): 0 start of the QKV phase, 1 its input loaded, 8 QKV rows
+ * done, 12 an attention item begins, 2 its q/k/v loaded, 13 q/k normed and
+ * rotated, K/V appended, 14 its keys done, 15 the warps' states merged, 9
+ * attention merged (across splits too), 3 start of the O phase, 4 its input
+ * loaded, 10 start of the gate/up phase, 5 its input loaded, 11 start of the
+ * down phase, 6 its input loaded, 7 block done; tail 0 start, 1 input
+ * loaded, 2 the producer's first LM-head copy, 3 its last copy issued, 6
+ * LM-head rows done, 7 greedy ids folded.
+ * Slots a CTA never reaches are left as they were. One-shot; NULL disarms.
+ * Timing only: no work changes. */
 fs_status fs_debug_trace(fs_model* model, uint64_t* buf);
 
 /* Debug: the time limit of every wait inside the persistent decode kernel
