@@ -29,6 +29,7 @@
 #include <algorithm>
 
 #include "runtime.h"
+#include "tc_common.cuh"
 
 namespace fs {
 namespace mega {
@@ -185,6 +186,35 @@ __device__ __forceinline__ void raise_timeout(const Params& p) {
 }
 __device__ __forceinline__ float lo16(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float hi16(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+// Tensor-core helpers of the attention items: ldmatrix (x4, plain and
+// transposed), mma.sync m16n8k16 bf16 -> fp32, and bf16 pairs.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// bf16 bits of x (round to nearest even), and of the remainder x - bf16(x)
+__device__ __forceinline__ uint32_t bf16_bits(float x) {
+  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+__device__ __forceinline__ uint32_t bf16_term(float x, bool lo) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(x);
+  return lo ? bf16_bits(x - __bfloat162float(h)) : (uint32_t)__bfloat16_as_ushort(h);
+}
 
 // ---------------------------------------------------------------------------
 // Shapes of the chunk stream (identical in producer and consumers)
@@ -371,7 +401,12 @@ struct Producer {
   bool quit = false;
   bool lm_started = false;
 
-  __device__ Producer(const Params& pp, Ring rr) : p(pp), r(rr) { policy = evict_first_policy(); }
+  const CUtensorMap* tm_k;  // the KV cache as [rows][d] bf16, 32 x 64 boxes, 128-byte swizzle
+  const CUtensorMap* tm_v;
+  __device__ Producer(const Params& pp, Ring rr, const CUtensorMap* mk, const CUtensorMap* mv)
+      : p(pp), r(rr), tm_k(mk), tm_v(mv) {
+    policy = evict_first_policy();
+  }
   __device__ bool stop() const { return quit; }
   __device__ __forceinline__ void advance() {
     ++i;
@@ -448,15 +483,25 @@ struct Producer {
     advance();
   }
 
+  // A KV chunk: keys [j, j + nk) of the item as K and V tiles in the 128-byte
+  // swizzled layout the tensor-core attention reads. TMA boxes of 32 rows x
+  // 64 dims: one per 32 keys and 64 dims of the chunk's kpc-key tile (rows
+  // past nk are loaded too: finite cache contents, masked by the consumer;
+  // rows past the cache read as zero).
   __device__ void kv(int layer, const Item& x, int j, int nk) {
     if (quit) return;
-    const uint32_t bytes = 2u * nk * p.d * 2;
-    unsigned char* st = acquire(bytes);
+    unsigned char* st = acquire(kWeightBytes);
     if (!st) return;
-    const size_t off = kv_off(p, layer, x.b, j, x.g);
+    const int row = (int)(kv_off(p, layer, x.b, j, x.g) / (size_t)p.d);
+    const int kpc = keys_per_chunk(p.d);
     uint64_t* bar = &r.full[stage];
-    bulk_load(st, p.kv.k + off, nk * p.d * 2, bar, policy);
-    bulk_load(st + kWeightBytes / 2, p.kv.v + off, nk * p.d * 2, bar, policy);
+    for (int cb = 0; cb < p.d / 64; ++cb)
+      for (int rb = 0; rb < kpc / 32; ++rb) {
+        const int off = cb * kpc * 128 + rb * 32 * 128;
+        tc::tma_load_2d(st + off, tm_k, cb * 64, row + rb * 32, bar);
+        tc::tma_load_2d(st + kWeightBytes / 2 + off, tm_v, cb * 64, row + rb * 32, bar);
+      }
+    (void)nk;
     advance();
   }
 };
@@ -482,8 +527,10 @@ struct Consumer {
   int tid, warp, lane;
   int G, cta;
   // attention state (per warp, registers)
-  float qreg[2][4];
-  float m[2], l[2], acc[2][4];
+  // attention state of the lane's head (lane % 4 < rep) on the tensor cores
+  uint32_t qb[8][2];  // B fragments of q (hi, lo terms per head) per 16-dim step
+  float mh, lh;       // running maximum and sum of the lane's head
+  float o[8][4];      // C fragments of O^T per 16-dim tile
 
   __device__ Consumer(const Params& pp, Ring rr, unsigned char* sm) : p(pp), r(rr), smem(sm) {
     hs = reinterpret_cast<float*>(sm + p.off_hs);
@@ -912,12 +959,16 @@ struct Consumer {
   }
 
   // ---- attention ---------------------------------------------------------
-  // Scratch (floats): q [rep][d] | knew [d] | vnew [d] | merge m,l [8][rep][2] | acc [8][rep][d]
+  // Scratch (floats): q [rep][d] | knew [d] | vnew [d] | merge m,l [12][rep][2] | O [12][rep][d]
+  // (a state per consumer warp, then the current position's key) | q fragments [512 words]
   __device__ float* q_s() { return at + 16; }
   __device__ float* k_s() { return q_s() + (p.nq / p.nkv) * p.d; }
   __device__ float* v_s() { return k_s() + p.d; }
   __device__ float* ml_s() { return v_s() + p.d; }
-  __device__ float* acc_s() { return ml_s() + kConsumerWarps * (p.nq / p.nkv) * 2; }
+  __device__ float* acc_s() { return ml_s() + (kConsumerWarps + 1) * (p.nq / p.nkv) * 2; }
+  __device__ uint32_t* qf_s() {  // q's B fragments [8 steps][2][32 lanes]
+    return reinterpret_cast<uint32_t*>(acc_s() + (kConsumerWarps + 1) * (p.nq / p.nkv) * p.d);
+  }
 
   // Per-lane constants of a head's RMSNorm + RoPE: gains of the lane's
   // elements of both halves and cos/sin at pos. Loaded before the wait for the
@@ -1001,206 +1052,210 @@ struct Consumer {
     }
     consumer_sync();
     tr(layer, 13);
-    const int E = d / 32;
+    // q as the B operand of S = K q^T: column g = lane / 4 holds head g / 2,
+    // term g % 2 (bf16 hi, then the lo remainder) of the scaled q; columns past
+    // 2 * rep are zero. k-step kk covers dims 16 kk .. 16 kk + 15.
+    // Built once per CTA into a table (word (kk, hf, lane)), then loaded by
+    // every warp.
     const float scale = 1.f / sqrtf((float)d);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      m[h] = -INFINITY;
-      l[h] = 0.f;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        acc[h][e] = 0.f;
-        qreg[h][e] = (h < rep && e < E) ? q_s()[h * d + lane * E + e] * scale : 0.f;
+    uint32_t* qf = qf_s();
+    for (int w = tid; w < 8 * 2 * 32; w += kConsumers) {
+      const int kk = w >> 6, hf = (w >> 5) & 1, ln = w & 31, g = ln >> 2, t4 = ln & 3;
+      uint32_t v = 0u;
+      if (kk * 16 < d && g < 2 * rep) {
+        const float* qh = q_s() + (g >> 1) * d + kk * 16 + hf * 8 + 2 * t4;
+        v = bf16_term(qh[0] * scale, g & 1) | (bf16_term(qh[1] * scale, g & 1) << 16);
       }
+      qf[w] = v;
     }
+    consumer_sync();
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) qb[kk][hf] = qf[(kk * 2 + hf) * 32 + lane];
+    mh = -INFINITY;
+    lh = 0.f;
+#pragma unroll
+    for (int dt = 0; dt < 8; ++dt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[dt][e] = 0.f;
   }
 
-  // Online-softmax update with one key (k, v given per lane: E elements).
-  __device__ __forceinline__ void attend(const float (&kk)[4], const float (&vv)[4], int rep) {
+  // One owner warp attends a whole KV chunk on the tensor cores and folds it
+  // into its online-softmax state, 32 keys at a time. The chunk's K and V
+  // tiles were loaded by TMA with the 128-byte swizzle: rows of 128 bytes
+  // (64 dims), 16-byte unit u of row r stored at u ^ (r % 8), one block of
+  // kpc rows per 64 dims. S = K q^T per 16 keys: A = 16 keys x 16 dims
+  // (ldmatrix), B = q (hi / lo terms of both heads). Lane (g, t) = (lane / 4,
+  // lane % 4) then holds the scores of keys g, g + 8, g + 16, g + 24 for head
+  // t (t < rep). P V: A = V^T (ldmatrix.trans), B = P (hi / lo terms),
+  // accumulated into O^T per 16-dim tile; the lane's columns 2t, 2t + 1
+  // belong to head t.
+  __device__ __forceinline__ void attend_chunk(const unsigned char* st, int nk) {
+    const int d = p.d, rep = p.nq / p.nkv;
+    const int nd = d >> 4;                         // 16-dim steps
+    const uint32_t cbs = keys_per_chunk(d) * 128;  // bytes per 64-dim block of a tile
+    const uint32_t kb = su32(st), vb = kb + kWeightBytes / 2;
+    const int g = lane >> 2, t4 = lane & 3, mi = lane >> 3, rr = lane & 7;
+    const int hn = g >> 1;  // head of this lane's B column
+    const bool col_ok = g < 2 * rep, lo = g & 1, hv = t4 < rep;
+    for (int kb0 = 0; kb0 < nk; kb0 += 32) {
+      float sa[2][4], sb[2][4];  // per 16-key half: two accumulation chains
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      if (h >= rep) break;
-      float s = 0.f;
+      for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) s = fmaf(qreg[h][e], kk[e], s);
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      const float mn = fmaxf(m[h], s);
-      const float c = expf(m[h] - mn), pr = expf(s - mn);
-      l[h] = l[h] * c + pr;
+        for (int e = 0; e < 4; ++e) sa[hf][e] = sb[hf][e] = 0.f;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[h][e] = acc[h][e] * c + pr * vv[e];
-      m[h] = mn;
-    }
-  }
-
-  // Transposing butterfly: NV partial sums per lane -> the full sum of value
-  // lane >> (5 - log2 NV) in every lane.
-  template <int NV>
-  __device__ __forceinline__ float reduce_transpose(float (&v)[NV]) {
-    int w = NV / 2, mask = 16;
+      for (int kk = 0; kk < 8; ++kk) {
+        if (kk < nd) {
+          const int dim = kk * 16 + (mi >> 1) * 8;
+          const uint32_t du = (uint32_t)(dim >> 6) * cbs, un = (dim & 63) >> 3;
 #pragma unroll
-    for (; w >= 1; w >>= 1, mask >>= 1) {
-      const bool upper = (lane & mask) != 0;
-#pragma unroll
-      for (int i = 0; i < w; ++i) {
-        const float send = upper ? v[i] : v[i + w];
-        const float keep = upper ? v[i + w] : v[i];
-        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+          for (int hf = 0; hf < 2; ++hf) {
+            const int ka = kb0 + hf * 16 + (mi & 1) * 8 + rr;  // key row addressed (A = K)
+            uint32_t a[4];
+            ldsm_x4(kb + du + ka * 128 + ((un ^ (ka & 7)) << 4), a);
+            if (kk & 1)
+              mma_bf16(sb[hf], a, qb[kk][0], qb[kk][1]);
+            else
+              mma_bf16(sa[hf], a, qb[kk][0], qb[kk][1]);
+          }
+        }
       }
-    }
-    float t = v[0];
+      float x[4];  // keys kb0 + g + 8 q
 #pragma unroll
-    for (; mask >= 1; mask >>= 1) t += __shfl_xor_sync(0xffffffffu, t, mask);
-    return t;
-  }
-
-  // Online-softmax update with this warp's keys of a KV chunk: keys warp,
-  // warp + 11, ... (at most KG). The KG x 2 partial dot products are reduced
-  // across the warp in one transposing butterfly; each lane pair / quad then
-  // holds one (key, head) score.
-  template <int E>
-  __device__ __forceinline__ void attend_group(const __nv_bfloat16* K, const __nv_bfloat16* Vv,
-                                               int nk) {
-    constexpr int KG = E == 4 ? 4 : 8;  // keys per warp: a chunk holds 32 (d=128) or 64 keys
-    constexpr int NV = 2 * KG;          // (key, head) pairs, head fastest
-    constexpr int SH = NV == 8 ? 2 : 1;
-    const int d = 32 * E;
-    uint32_t kr[KG][E / 2], vr[KG][E / 2];
-#pragma unroll
-    for (int i = 0; i < KG; ++i) {
-      const int j = warp + i * kConsumerWarps;
-#pragma unroll
-      for (int e = 0; e < E / 2; ++e) {
-        kr[i][e] = 0u;
-        vr[i][e] = 0u;
+      for (int q = 0; q < 4; ++q) {
+        const int hf = q >> 1, e = (q & 1) * 2;
+        const bool ok = hv && kb0 + g + 8 * q < nk;
+        x[q] = ok ? (sa[hf][e] + sb[hf][e]) + (sa[hf][e + 1] + sb[hf][e + 1]) : -INFINITY;
       }
-      if (j < nk) {
-        if constexpr (E == 4) {
-          const uint2 ku = *reinterpret_cast<const uint2*>(K + j * d + lane * 4);
-          const uint2 vu = *reinterpret_cast<const uint2*>(Vv + j * d + lane * 4);
-          kr[i][0] = ku.x; kr[i][1] = ku.y;
-          vr[i][0] = vu.x; vr[i][1] = vu.y;
-        } else {
-          kr[i][0] = *reinterpret_cast<const uint32_t*>(K + j * d + lane * 2);
-          vr[i][0] = *reinterpret_cast<const uint32_t*>(Vv + j * d + lane * 2);
+      float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+#pragma unroll
+      for (int o2 = 4; o2 < 32; o2 <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
+      const float mn = fmaxf(mh, mx);
+      const float alpha = (mn == -INFINITY) ? 1.f : expf(mh - mn);
+      float pr[4], sm = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        pr[q] = x[q] == -INFINITY ? 0.f : expf(x[q] - mn);
+        sm += pr[q];
+      }
+#pragma unroll
+      for (int o2 = 4; o2 < 32; o2 <<= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o2);
+      lh = lh * alpha + sm;
+      mh = mn;
+#pragma unroll
+      for (int dt = 0; dt < 8; ++dt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[dt][e] *= alpha;
+      // B = P per 16-key half: column g is head hn, term g % 2; keys 2t, 2t + 1
+      // (b0) and 2t + 8, 2t + 9 (b1). Key k's probability for head hn sits in
+      // lane (k % 8) * 4 + hn, value pr[k / 8].
+      uint32_t pb[2][2];
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const float q00 = __shfl_sync(0xffffffffu, pr[2 * hf], (2 * t4) * 4 + hn);
+        const float q01 = __shfl_sync(0xffffffffu, pr[2 * hf], (2 * t4 + 1) * 4 + hn);
+        const float q10 = __shfl_sync(0xffffffffu, pr[2 * hf + 1], (2 * t4) * 4 + hn);
+        const float q11 = __shfl_sync(0xffffffffu, pr[2 * hf + 1], (2 * t4 + 1) * 4 + hn);
+        pb[hf][0] = col_ok ? bf16_term(q00, lo) | (bf16_term(q01, lo) << 16) : 0u;
+        pb[hf][1] = col_ok ? bf16_term(q10, lo) | (bf16_term(q11, lo) << 16) : 0u;
+      }
+#pragma unroll
+      for (int dt = 0; dt < 8; ++dt) {
+        if (dt < nd) {
+          const int dim = dt * 16 + (mi & 1) * 8;
+          const uint32_t du = (uint32_t)(dim >> 6) * cbs, un = (dim & 63) >> 3;
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const int kv_ = kb0 + hf * 16 + (mi >> 1) * 8 + rr;  // key row (A = V^T)
+            uint32_t a[4];
+            ldsm_x4_t(vb + du + kv_ * 128 + ((un ^ (kv_ & 7)) << 4), a);
+            mma_bf16(o[dt], a, pb[hf][0], pb[hf][1]);
+          }
         }
       }
     }
-    float part[NV];
-#pragma unroll
-    for (int i = 0; i < KG; ++i)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float t = 0.f;
-#pragma unroll
-        for (int e = 0; e < E / 2; ++e) {
-          t = fmaf(qreg[h][2 * e], lo16(kr[i][e]), t);
-          t = fmaf(qreg[h][2 * e + 1], hi16(kr[i][e]), t);
-        }
-        part[i * 2 + h] = t;
-      }
-    float sc = reduce_transpose<NV>(part);
-    const int my_v = lane >> SH, my_k = my_v >> 1, my_h = my_v & 1;
-    if (warp + my_k * kConsumerWarps >= nk) sc = -INFINITY;
-    float gm = sc;
-#pragma unroll
-    for (int b = SH + 1; b < 5; ++b) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, 1 << b));
-    float m_new[2], alpha[2];
-    bool any = false;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const float gmh = __shfl_sync(0xffffffffu, gm, h << SH);
-      any |= gmh != -INFINITY;
-      m_new[h] = fmaxf(m[h], gmh);
-      alpha[h] = (m_new[h] == -INFINITY) ? 1.f : expf(m[h] - m_new[h]);
-    }
-    if (!any) return;  // no key of this chunk for this warp (warp-uniform)
-    const float mh = my_h ? m_new[1] : m_new[0];
-    const float pv = (sc == -INFINITY) ? 0.f : expf(sc - mh);
-    float gs = pv;
-#pragma unroll
-    for (int b = SH + 1; b < 5; ++b) gs += __shfl_xor_sync(0xffffffffu, gs, 1 << b);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      l[h] = l[h] * alpha[h] + __shfl_sync(0xffffffffu, gs, h << SH);
-      m[h] = m_new[h];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[h][e] *= alpha[h];
-    }
-#pragma unroll
-    for (int i = 0; i < KG; ++i)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const float pk = __shfl_sync(0xffffffffu, pv, (i * 2 + h) << SH);
-#pragma unroll
-        for (int e = 0; e < E / 2; ++e) {
-          acc[h][2 * e] = fmaf(pk, lo16(vr[i][e]), acc[h][2 * e]);
-          acc[h][2 * e + 1] = fmaf(pk, hi16(vr[i][e]), acc[h][2 * e + 1]);
-        }
-      }
   }
 
+  // A KV chunk of the item, owner mode like the weight chunks: chunk i is
+  // attended by warp i % (consumer warps) alone, which then releases it; the
+  // warps' states are merged once, in attn_end.
   __device__ __forceinline__ void kv(int, const Item&, int, int nk) {
-    // Contains a CTA barrier: no early exit; a thread that gave up skips the work.
-    const unsigned char* st = stage_wait();
-    const __nv_bfloat16* K = reinterpret_cast<const __nv_bfloat16*>(st);
-    const __nv_bfloat16* Vv = reinterpret_cast<const __nv_bfloat16*>(st + kWeightBytes / 2);
-    if (!__any_sync(0xffffffffu, quit)) {
-      if (p.d == 128)
-        attend_group<4>(K, Vv, nk);
-      else
-        attend_group<2>(K, Vv, nk);
+    if ((int)(i % kConsumerWarps) == warp) {
+      const unsigned char* st = stage_wait();
+      if (!__any_sync(0xffffffffu, quit)) attend_chunk(st, nk);
+      stage_release();
     }
-    // Every consumer warp reads a KV chunk; the stage is released once, after
-    // all of them are done with it.
-    quit = consumer_sync_or(quit);
-    if (tid == 0) mbar_arrive(&r.empty[stage]);
     advance();
   }
 
   __device__ __forceinline__ void attn_end(int layer, int, const Item& x) {
     // No early exit before the first barrier: threads may disagree on quit here.
     tr(layer, 14);
-    const int d = p.d, rep = p.nq / p.nkv, E = d / 32;
-    if (x.owner && warp == 0 && !quit) {
-      float kk[4] = {0.f, 0.f, 0.f, 0.f}, vv[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        if (e < E) {
-          kk[e] = k_s()[lane * E + e];
-          vv[e] = v_s()[lane * E + e];
-        }
-      }
-      attend(kk, vv, rep);
-    }
+    const int d = p.d, rep = p.nq / p.nkv;
+    constexpr int NSL = kConsumerWarps + 1;  // states: one per warp, then the new key
     float* ml = ml_s();
     float* ac = acc_s();
+    // this warp's state: lanes (g, t < rep) hold head t's columns of O^T
+    {
+      const int g = lane >> 2, t4 = lane & 3;
+      if (t4 < rep) {
+        if (g == 0) {
+          ml[(warp * rep + t4) * 2] = mh;
+          ml[(warp * rep + t4) * 2 + 1] = lh;
+        }
+        float* a = ac + (warp * rep + t4) * d;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      if (h >= rep) break;
-      if (lane == 0) {
-        ml[(warp * rep + h) * 2] = m[h];
-        ml[(warp * rep + h) * 2 + 1] = l[h];
+        for (int dt = 0; dt < 8; ++dt) {
+          if (dt * 16 < d) {
+            a[dt * 16 + g] = o[dt][0] + o[dt][1];
+            a[dt * 16 + g + 8] = o[dt][2] + o[dt][3];
+          }
+        }
       }
+    }
+    // the last state: the current position's key, in the item that holds it
+    if (warp == 0) {
+      const float scale = 1.f / sqrtf((float)d);
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (e < E) ac[(warp * rep + h) * d + lane * E + e] = acc[h][e];
+      for (int h = 0; h < 2; ++h) {
+        if (h >= rep) break;
+        float sh = 0.f;
+        for (int c = lane; c < d; c += 32) sh = fmaf(q_s()[h * d + c] * scale, k_s()[c], sh);
+        for (int o2 = 16; o2 > 0; o2 >>= 1) sh += __shfl_xor_sync(0xffffffffu, sh, o2);
+        if (lane == 0) {
+          ml[(kConsumerWarps * rep + h) * 2] = x.owner ? sh : -INFINITY;
+          ml[(kConsumerWarps * rep + h) * 2 + 1] = x.owner ? 1.f : 0.f;
+        }
+        for (int c = lane; c < d; c += 32)
+          ac[(kConsumerWarps * rep + h) * d + c] = x.owner ? v_s()[c] : 0.f;
+      }
     }
     quit = consumer_sync_or(quit);
     if (quit) return;
     const int ns = p.n_splits;
     const uint32_t t2 = tag(layer, 2);
-    // merge the warps: thread per (head, dim)
+    // merge the warps: first each warp's factor exp(m_w - M) per head (q's
+    // space is free now), then one thread per (head, dim)
+    float* fq = q_s();  // [state][rep] factors, then [rep] maxima
+    if (tid < NSL * rep) {
+      const int h = tid / NSL, w = tid - h * NSL;
+      float M = -INFINITY;
+      for (int w2 = 0; w2 < NSL; ++w2) M = fmaxf(M, ml[(w2 * rep + h) * 2]);
+      const float mw = ml[(w * rep + h) * 2];
+      fq[w * rep + h] = (mw == -INFINITY) ? 0.f : expf(mw - M);
+      if (w == 0) fq[NSL * rep + h] = M;
+    }
+    consumer_sync();
     for (int t = tid; t < rep * d; t += kConsumers) {
       const int h = t / d, c = t % d;
-      float M = -INFINITY;
-      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ml[(w * rep + h) * 2]);
+      const float M = fq[NSL * rep + h];
       float L = 0.f, O = 0.f;
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        const float mw = ml[(w * rep + h) * 2];
-        const float f = (mw == -INFINITY) ? 0.f : expf(mw - M);
-        L += ml[(w * rep + h) * 2 + 1] * f;
-        O += ac[(w * rep + h) * d + c] * f;
+      for (int w = 0; w < NSL; ++w) {
+        const float f = fq[w * rep + h];
+        L = fmaf(ml[(w * rep + h) * 2 + 1], f, L);
+        O = fmaf(ac[(w * rep + h) * d + c], f, O);
       }
       const int qh = x.g * rep + h;
       if (ns == 1) {
@@ -1295,7 +1350,9 @@ struct Consumer {
 };
 
 template <int NB, bool Q8W>
-__global__ void __launch_bounds__(kThreads, 1) decode_mega_kernel(const __grid_constant__ Params p) {
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_mega_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v) {
   extern __shared__ __align__(1024) unsigned char smem[];
   Ring ring;
   ring.stages = smem;
@@ -1334,7 +1391,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mega_kernel(const __grid_c
   if (warp == kConsumerWarps) {
     // producer warp: one lane issues, the others go straight to the end
     if ((threadIdx.x & 31) == 0) {
-      Producer pr(p, ring);
+      Producer pr(p, ring, &tm_k, &tm_v);
       walk(p, blockIdx.x, gridDim.x, pr);
       if (p.trace) p.trace[((size_t)blockIdx.x * (p.L + 1) + p.L) * 16 + 3] = clock64();
       reinterpret_cast<volatile unsigned int*>(smem + p.off_misc + 8 * kMaxB + 8)[0] = pr.i;
@@ -1393,9 +1450,20 @@ struct MegaState {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Keys per attention item of a decode step (the items of a kv head are merged
-// by the last one to finish).
-constexpr int kKeysPerSplit = 64;
+// Keys per attention item of a decode step: one KV chunk per consumer warp,
+// all attended at once (the items of a kv head are merged by the last one to
+// finish).
+#ifndef FS_MEGA_LONG_CHUNKS
+#define FS_MEGA_LONG_CHUNKS 4
+#endif
+// A context that fits one item of a chunk per consumer warp takes one item per
+// kv head (no merge of splits); a longer one is cut into items of
+// FS_MEGA_LONG_CHUNKS chunks, spread over more CTAs (each CTA then streams
+// fewer KV bytes per block).
+int keys_per_split(int d, int context) {
+  const int one = mega::kConsumerWarps * mega::keys_per_chunk(d);
+  return context <= one ? one : FS_MEGA_LONG_CHUNKS * mega::keys_per_chunk(d);
+}
 
 }  // namespace
 
@@ -1540,8 +1608,9 @@ fs_status decode_mega(fs_model* m, const fs_kv* kv, const RowMap& map, int B, co
   p.split_cnt = st->split_cnt;
   p.am_key = st->am_key;
   p.am_cnt = st->am_cnt;
-  // ~64 keys per attention item, at most one item per CTA
-  int ns = (cmax + kKeysPerSplit - 1) / kKeysPerSplit;
+  // at most one item per CTA
+  const int kps = keys_per_split(s.d, cmax);
+  int ns = (cmax + kps - 1) / kps;
   ns = std::max(1, std::min(ns, std::min(st->max_splits, st->sms / (B * s.nkv))));
   p.n_splits = ns;
   p.l0 = l0;
@@ -1579,8 +1648,8 @@ fs_status decode_mega(fs_model* m, const fs_kv* kv, const RowMap& map, int B, co
   size_t off = 0;
   const size_t fixed_hs = align_up((size_t)B * s.H * 4, 128);
   const size_t fixed_xs = align_up((size_t)B * maxK * 4, 128);
-  const size_t attn = align_up((16 + rep * s.d + 2 * s.d + mega::kConsumerWarps * rep * 2 +
-                                mega::kConsumerWarps * rep * s.d) * 4, 128);
+  const size_t attn = align_up((16 + rep * s.d + 2 * s.d + (mega::kConsumerWarps + 1) * rep * 2 +
+                                (mega::kConsumerWarps + 1) * rep * s.d + 512) * 4, 128);
   const size_t bars = 2 * mega::kMaxStages * 8;
   const size_t misc = 128;
   const size_t bt_bytes = (size_t)B * kv->pages_per_seq * sizeof(int32_t);
@@ -1604,7 +1673,14 @@ fs_status decode_mega(fs_model* m, const fs_kv* kv, const RowMap& map, int B, co
   p.off_tab = (int)off; off += tab;
   p.bt_in_smem = bt_smem ? 1 : 0;
   p.n_stages = n_stages;
-  void* args[] = {&p};
+  // the KV cache as [rows][d] bf16 for the attention items' TMA loads
+  const long long kv_rows = (long long)s.L * kv->n_pages * s.nkv * kPage;
+  if (kv_rows + 64 >= (1LL << 31)) return FS_ERR_UNSUPPORTED;
+  CUtensorMap tm_k, tm_v;
+  if (!make_tmap_16(&tm_k, kv->k, kv_rows, s.d, 32, true) ||
+      !make_tmap_16(&tm_v, kv->v, kv_rows, s.d, 32, true))
+    return FS_ERR_UNSUPPORTED;
+  void* args[] = {&p, &tm_k, &tm_v};
   count_launches();
   const void* fn = B == 1 ? (m->q8 ? (const void*)mega::decode_mega_kernel<1, true>
                                     : (const void*)mega::decode_mega_kernel<1, false>)
