@@ -945,7 +945,7 @@ struct Consumer {
       case kLM: {
         if (p.logits) p.logits[(size_t)b * p.V + n] = y;
         if (isfinite(y)) {
-          const uint32_t uu = __float_as_uint(y);
+          const uint32_t uu = (y == 0.f) ? 0u : __float_as_uint(y);  // -0 ranks as +0
           const uint32_t ord = (uu & 0x80000000u) ? ~uu : (uu | 0x80000000u);
           const unsigned long long key =
               ((unsigned long long)ord << 32) | (0xffffffffu - (uint32_t)n);
