@@ -1,92 +1,90 @@
 // Weight-streaming linear layer for 5..16 rows (batched decode, bf16
-// weights): y[r, n] (+)= sum_k x[r, k] W[n, k].
+// weights): y[r, n] (+)= sum_k x[r, k] W[n, k], on the tensor cores.
 //
-// One warp owns 8 weight rows and a 256-wide slice of the input axis: every
-// lane loads 8 consecutive bf16 weights of each of the 8 rows (16-byte loads,
-// 512 contiguous bytes per row per warp) and the matching 8 activations of
-// each batch row, so an activation load serves 8 weight rows and a weight
-// load serves every batch row. The 8 x R partial sums are reduced across the
-// warp by a transposing butterfly (4 sums per lane at the end) and added
-// into y with fp32 atomics, which combine the slices of the input axis.
-// Many short warps keep enough weight bytes in flight to stream HBM.
+// mma.sync m16n8k16 (bf16 in, fp32 accumulate) with the batch rows as M (16,
+// rows past `rows` zero) and 8 weight rows as N. A CTA takes one 256-wide
+// slice of the input axis: it stages the slice of x once in shared memory as
+// two bf16 terms (hi and the lo remainder, about 16 significant bits), and
+// its 8 warps each stream tasks of 8 weight rows of it straight from global
+// memory into registers (16-byte loads); a warp runs `tpw` tasks (more than
+// one only for very wide outputs, to share the staged slice). The k order inside an MMA is a fixed
+// permutation of the physical k: lane (g, t) holds weights 8t .. 8t + 7 of
+// a 32-wide group, used as the B pairs (8t, 8t + 1 | 8t + 2, 8t + 3) of one
+// MMA and (8t + 4, .. | 8t + 6, ..) of the next, and the A fragments of x
+// are read with the same mapping, so every product pairs matching k. The
+// accumulators need no shuffles: each lane adds its 4 outputs into y with
+// fp32 atomics, which combine the slices of the input axis.
 #include "fs_internal.h"
 
 namespace fs {
 
 namespace {
 
-constexpr int kRowsPerWarp = 8;
-constexpr int kSlice = 256;  // input-axis slice of one warp
-constexpr int kWarps = 4;
+constexpr int kSlice = 256;        // input-axis slice of a CTA
+constexpr int kWarps = 8;
+constexpr int kRowsPerWarp = 8;    // weight rows of a warp task (one n8 tile)
+constexpr int kXStride = kSlice + 32;  // bf16 per staged row (64-byte pad: no bank conflicts)
 
-__device__ __forceinline__ float lo16(uint32_t u) { return __uint_as_float(u << 16); }
-__device__ __forceinline__ float hi16(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
-
-// Transposing butterfly over the warp: 128 partial sums per lane in, the
-// warp totals of 4 of them per lane out. Rounds with masks 16, 8, 4, 2, 1
-// halve the values a lane keeps (64, 32, 16, 8, 4); afterwards lane l holds
-// in v[q] the total of index 64*b4 + 32*b3 + 16*b2 + 8*b1 + 4*b0 + q, with
-// b4..b0 the bits of l.
-__device__ __forceinline__ void reduce128(float (&v)[128], int lane) {
-#pragma unroll
-  for (int w = 64, mask = 16; w >= 4; w >>= 1, mask >>= 1) {
-    const bool upper = (lane & mask) != 0;
-#pragma unroll
-    for (int i = 0; i < w; ++i) {
-      const float send = upper ? v[i] : v[i + w];
-      const float keep = upper ? v[i + w] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
-    }
-  }
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-template <int R>
-__global__ void __launch_bounds__(kWarps * 32) gemv_splitk_kernel(
+__global__ void __launch_bounds__(kWarps * 32) gemv_mma_kernel(
     const float* __restrict__ x, int rows, int K, const __nv_bfloat16* __restrict__ W, int N,
-    float* __restrict__ out, int ldo) {
-  const int lane = threadIdx.x & 31;
-  const int gw = blockIdx.x * kWarps + (threadIdx.x >> 5);
-  const int slices = K / kSlice;
-  const int n_groups = (N + kRowsPerWarp - 1) / kRowsPerWarp;
-  if (gw >= n_groups * slices) return;
-  const int grp = gw / slices, sl = gw % slices;
-  const int n0 = grp * kRowsPerWarp;
-  const int k = sl * kSlice + lane * 8;
-
-  uint4 w[kRowsPerWarp];
+    float* __restrict__ out, int ldo, int ctas_per_slice, int tpw) {
+  // [term][16 rows][kXStride] bf16
+  __shared__ __align__(16) __nv_bfloat16 xs[2][16][kXStride];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int slice = blockIdx.x / ctas_per_slice, cs = blockIdx.x % ctas_per_slice;
+  const int k0 = slice * kSlice;
+  const int g = lane >> 2, t = lane & 3;
+  const int n_tasks = (N + kRowsPerWarp - 1) / kRowsPerWarp;
+  // The first task's weights are requested before the slice of x is staged,
+  // so the HBM latency overlaps the staging. Weights: row n0 + g, 8 groups of
+  // 32 k; lane t holds 8t .. 8t + 7 of each.
+  uint4 w[8];
+  auto load_w = [&](int task) {
+    const int n = min(task * kRowsPerWarp + g, N - 1);  // rows past N repeat the last; dropped
+    const __nv_bfloat16* wr = W + (size_t)n * K + k0 + 8 * t;
 #pragma unroll
-  for (int j = 0; j < kRowsPerWarp; ++j) {
-    const int n = min(n0 + j, N - 1);  // rows past N repeat the last one; dropped below
-    w[j] = __ldg(reinterpret_cast<const uint4*>(W + (size_t)n * K + k));
+    for (int q = 0; q < 8; ++q) w[q] = __ldg(reinterpret_cast<const uint4*>(wr + 32 * q));
+  };
+  int task = cs * tpw * kWarps + warp;
+  if (task < n_tasks) load_w(task);
+  for (int e = tid; e < 16 * kSlice; e += kWarps * 32) {
+    const int r = e / kSlice, c = e % kSlice;
+    const float v = r < rows ? x[(size_t)r * K + k0 + c] : 0.f;
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    xs[0][r][c] = h;
+    xs[1][r][c] = __float2bfloat16_rn(v - __bfloat162float(h));
   }
-  float v[128];
+  __syncthreads();
+  for (int it = 0; it < tpw; ++it, task += kWarps) {
+    if (task >= n_tasks) break;
+    if (it > 0) load_w(task);
+    const int n0 = task * kRowsPerWarp;
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // hi, lo chains
 #pragma unroll
-  for (int i = 0; i < 128; ++i) v[i] = 0.f;
+    for (int q = 0; q < 8; ++q) {
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    if (r >= rows) break;
-    const float4 a = __ldg(reinterpret_cast<const float4*>(x + (size_t)r * K + k));
-    const float4 b = __ldg(reinterpret_cast<const float4*>(x + (size_t)r * K + k + 4));
-#pragma unroll
-    for (int j = 0; j < kRowsPerWarp; ++j) {
-      float s = lo16(w[j].x) * a.x;
-      s = fmaf(hi16(w[j].x), a.y, s);
-      s = fmaf(lo16(w[j].y), a.z, s);
-      s = fmaf(hi16(w[j].y), a.w, s);
-      s = fmaf(lo16(w[j].z), b.x, s);
-      s = fmaf(hi16(w[j].z), b.y, s);
-      s = fmaf(lo16(w[j].w), b.z, s);
-      s = fmaf(hi16(w[j].w), b.w, s);
-      v[r * 8 + j] = s;
+      for (int term = 0; term < 2; ++term) {
+        const uint4 xa = *reinterpret_cast<const uint4*>(&xs[term][g][32 * q + 8 * t]);
+        const uint4 xb = *reinterpret_cast<const uint4*>(&xs[term][g + 8][32 * q + 8 * t]);
+        mma_bf16(acc[term], xa.x, xb.x, xa.y, xb.y, w[q].x, w[q].y);
+        mma_bf16(acc[term], xa.z, xb.z, xa.w, xb.w, w[q].z, w[q].w);
+      }
     }
-  }
-  reduce128(v, lane);
-  const int base = ((lane >> 4) & 1) * 64 + ((lane >> 3) & 1) * 32 + ((lane >> 2) & 1) * 16 +
-                   ((lane >> 1) & 1) * 8 + (lane & 1) * 4;
+    // D[batch row][weight row]: (g, 2t), (g, 2t + 1), (g + 8, 2t), (g + 8, 2t + 1)
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int idx = base + q, r = idx >> 3, j = idx & 7;
-    if (r < rows && n0 + j < N) atomicAdd(out + (size_t)r * ldo + n0 + j, v[q]);
+    for (int e = 0; e < 4; ++e) {
+      const int r = g + (e >> 1) * 8, n = n0 + 2 * t + (e & 1);
+      if (r < rows && n < N) atomicAdd(out + (size_t)r * ldo + n, acc[0][e] + acc[1][e]);
+    }
   }
 }
 
@@ -159,10 +157,16 @@ cudaError_t launch_gemv_splitk(const float* x, int rows, int K, const __nv_bfloa
                                       rows, st);
     if (e != cudaSuccess) return e;
   }
-  const int warps = (N + kRowsPerWarp - 1) / kRowsPerWarp * (K / kSlice);
-  const int blocks = (warps + kWarps - 1) / kWarps;
+  const int n_tasks = (N + kRowsPerWarp - 1) / kRowsPerWarp;
+  const int slices = K / kSlice;
+  // one task per warp unless the grid would exceed ~4 waves of 3 CTAs per SM
+  int tpw = 1;
+  while (tpw < 8 && (long long)n_tasks * slices / (kWarps * tpw) > 148LL * 3 * 4) tpw *= 2;
+  const int ctas_per_slice = (n_tasks + kWarps * tpw - 1) / (kWarps * tpw);
+  const int blocks = ctas_per_slice * slices;
   count_launches();
-  gemv_splitk_kernel<16><<<blocks, kWarps * 32, 0, st>>>(x, rows, K, W, N, out, ldo);
+  gemv_mma_kernel<<<blocks, kWarps * 32, 0, st>>>(x, rows, K, W, N, out, ldo, ctas_per_slice,
+                                                  tpw);
   return cudaGetLastError();
 }
 
