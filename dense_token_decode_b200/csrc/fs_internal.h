@@ -107,6 +107,11 @@ cudaError_t launch_gemv_swiglu(const float* x, int rows, int K, const void* Wg, 
 bool gemv_splitk_ok(int rows, int K, const __half* scales);
 cudaError_t launch_gemv_splitk(const float* x, int rows, int K, const __nv_bfloat16* W, int N,
                                float* out, int ldo, bool accumulate, cudaStream_t st);
+// The same for n (2 or 3) matrices of one input in one launch, written side by
+// side from out0 (cleared first): q | k | v, gate | up.
+cudaError_t launch_gemv_splitk_multi(const float* x, int rows, int K, int n,
+                                     const __nv_bfloat16* const* W, const int* N, float* out0,
+                                     int ldo, cudaStream_t st);
 // Greedy id per row of fp32 logits [rows][V] (lowest id on exact ties).
 cudaError_t launch_argmax_rows(const float* logits, int rows, int V, int32_t* argmax,
                                cudaStream_t st);

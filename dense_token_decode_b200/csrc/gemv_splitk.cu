@@ -34,23 +34,38 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Up to three products of the same input in one launch (q, k, v; gate, up):
+// segment i multiplies x by W[i] (N[i] rows) into out[i]. Tasks of 8 weight
+// rows are numbered across the segments.
+struct Segs {
+  const __nv_bfloat16* W[3];
+  float* out[3];
+  int N[3];
+  int tasks[3];  // cumulative task counts
+  int n;
+};
+
 __global__ void __launch_bounds__(kWarps * 32) gemv_mma_kernel(
-    const float* __restrict__ x, int rows, int K, const __nv_bfloat16* __restrict__ W, int N,
-    float* __restrict__ out, int ldo, int ctas_per_slice, int tpw) {
+    const float* __restrict__ x, int rows, int K, const Segs sg, int ldo, int ctas_per_slice,
+    int tpw) {
   // [term][16 rows][kXStride] bf16
   __shared__ __align__(16) __nv_bfloat16 xs[2][16][kXStride];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int slice = blockIdx.x / ctas_per_slice, cs = blockIdx.x % ctas_per_slice;
   const int k0 = slice * kSlice;
   const int g = lane >> 2, t = lane & 3;
-  const int n_tasks = (N + kRowsPerWarp - 1) / kRowsPerWarp;
+  const int n_tasks = sg.tasks[sg.n - 1];
   // The first task's weights are requested before the slice of x is staged,
   // so the HBM latency overlaps the staging. Weights: row n0 + g, 8 groups of
   // 32 k; lane t holds 8t .. 8t + 7 of each.
   uint4 w[8];
+  int seg = 0, n0 = 0;
   auto load_w = [&](int task) {
-    const int n = min(task * kRowsPerWarp + g, N - 1);  // rows past N repeat the last; dropped
-    const __nv_bfloat16* wr = W + (size_t)n * K + k0 + 8 * t;
+    seg = task < sg.tasks[0] ? 0 : (task < sg.tasks[1] ? 1 : 2);
+    n0 = (task - (seg ? sg.tasks[seg - 1] : 0)) * kRowsPerWarp;
+    const int N = sg.N[seg];
+    const int n = min(n0 + g, N - 1);  // rows past N repeat the last one; dropped below
+    const __nv_bfloat16* wr = sg.W[seg] + (size_t)n * K + k0 + 8 * t;
 #pragma unroll
     for (int q = 0; q < 8; ++q) w[q] = __ldg(reinterpret_cast<const uint4*>(wr + 32 * q));
   };
@@ -67,7 +82,6 @@ __global__ void __launch_bounds__(kWarps * 32) gemv_mma_kernel(
   for (int it = 0; it < tpw; ++it, task += kWarps) {
     if (task >= n_tasks) break;
     if (it > 0) load_w(task);
-    const int n0 = task * kRowsPerWarp;
     float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // hi, lo chains
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
@@ -80,6 +94,8 @@ __global__ void __launch_bounds__(kWarps * 32) gemv_mma_kernel(
       }
     }
     // D[batch row][weight row]: (g, 2t), (g, 2t + 1), (g + 8, 2t), (g + 8, 2t + 1)
+    float* out = sg.out[seg];
+    const int N = sg.N[seg];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int r = g + (e >> 1) * 8, n = n0 + 2 * t + (e & 1);
@@ -147,6 +163,23 @@ bool gemv_splitk_ok(int rows, int K, const __half* scales) {
   return scales == nullptr && rows >= 1 && rows <= 16 && K % kSlice == 0;
 }
 
+namespace {
+
+cudaError_t launch_segs(const float* x, int rows, int K, Segs sg, int ldo, cudaStream_t st) {
+  const int n_tasks = sg.tasks[sg.n - 1];
+  const int slices = K / kSlice;
+  // one task per warp unless the grid would exceed ~4 waves of 3 CTAs per SM
+  int tpw = 1;
+  while (tpw < 8 && (long long)n_tasks * slices / (kWarps * tpw) > 148LL * 3 * 4) tpw *= 2;
+  const int ctas_per_slice = (n_tasks + kWarps * tpw - 1) / (kWarps * tpw);
+  const int blocks = ctas_per_slice * slices;
+  count_launches();
+  gemv_mma_kernel<<<blocks, kWarps * 32, 0, st>>>(x, rows, K, sg, ldo, ctas_per_slice, tpw);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 // y (+)= x W^T over `rows` rows; out rows are ldo floats apart. Without
 // `accumulate` the output block is cleared first.
 cudaError_t launch_gemv_splitk(const float* x, int rows, int K, const __nv_bfloat16* W, int N,
@@ -157,17 +190,41 @@ cudaError_t launch_gemv_splitk(const float* x, int rows, int K, const __nv_bfloa
                                       rows, st);
     if (e != cudaSuccess) return e;
   }
-  const int n_tasks = (N + kRowsPerWarp - 1) / kRowsPerWarp;
-  const int slices = K / kSlice;
-  // one task per warp unless the grid would exceed ~4 waves of 3 CTAs per SM
-  int tpw = 1;
-  while (tpw < 8 && (long long)n_tasks * slices / (kWarps * tpw) > 148LL * 3 * 4) tpw *= 2;
-  const int ctas_per_slice = (n_tasks + kWarps * tpw - 1) / (kWarps * tpw);
-  const int blocks = ctas_per_slice * slices;
-  count_launches();
-  gemv_mma_kernel<<<blocks, kWarps * 32, 0, st>>>(x, rows, K, W, N, out, ldo, ctas_per_slice,
-                                                  tpw);
-  return cudaGetLastError();
+  Segs sg{};
+  sg.W[0] = W;
+  sg.out[0] = out;
+  sg.N[0] = N;
+  sg.tasks[0] = (N + kRowsPerWarp - 1) / kRowsPerWarp;
+  sg.n = 1;
+  return launch_segs(x, rows, K, sg, ldo, st);
+}
+
+// Products of one input with n (2 or 3) matrices, written side by side: W[i]
+// (N[i] rows) into columns out0 + sum_{j<i} N[j] of rows ldo floats apart,
+// which are cleared first (one memset, then one launch).
+cudaError_t launch_gemv_splitk_multi(const float* x, int rows, int K, int n,
+                                     const __nv_bfloat16* const* W, const int* N, float* out0,
+                                     int ldo, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  if (n < 1 || n > 3) return cudaErrorInvalidValue;
+  int width = 0;
+  for (int i = 0; i < n; ++i) width += N[i];
+  cudaError_t e = cudaMemset2DAsync(out0, (size_t)ldo * sizeof(float), 0,
+                                    (size_t)width * sizeof(float), rows, st);
+  if (e != cudaSuccess) return e;
+  Segs sg{};
+  int col = 0, tasks = 0;
+  for (int i = 0; i < n; ++i) {
+    sg.W[i] = W[i];
+    sg.out[i] = out0 + col;
+    sg.N[i] = N[i];
+    tasks += (N[i] + kRowsPerWarp - 1) / kRowsPerWarp;
+    sg.tasks[i] = tasks;
+    col += N[i];
+  }
+  for (int i = n; i < 3; ++i) sg.tasks[i] = tasks;
+  sg.n = n;
+  return launch_segs(x, rows, K, sg, ldo, st);
 }
 
 }  // namespace fs

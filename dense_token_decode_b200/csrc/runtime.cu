@@ -384,9 +384,19 @@ fs_status layer_general(fs_model* m, const fs_kv* kv, const RowMap& map, int row
   const int H = s.H, qd = s.q_dim(), kvd = s.kv_dim(), qkvd = s.qkv_dim();
   const LayerDev& Lw = m->layers[l];
   FS_CUDA(launch_rmsnorm(m->h, rows, H, Lw.attn_norm, s.eps, m->xn, st));
-  FS_CUDA(linear(m, m->xn, rows, H, l, kWq, qd, m->qkv, qkvd, false, st));
-  FS_CUDA(linear(m, m->xn, rows, H, l, kWk, kvd, m->qkv + qd, qkvd, false, st));
-  FS_CUDA(linear(m, m->xn, rows, H, l, kWv, kvd, m->qkv + qd + kvd, qkvd, false, st));
+  const bool splitk = rows > 4 && gemv_splitk_ok(rows, H, Lw.s[kWq]);
+  if (splitk) {
+    // q | k | v in one launch
+    const __nv_bfloat16* W3[3] = {static_cast<const __nv_bfloat16*>(Lw.w[kWq]),
+                                  static_cast<const __nv_bfloat16*>(Lw.w[kWk]),
+                                  static_cast<const __nv_bfloat16*>(Lw.w[kWv])};
+    const int N3[3] = {qd, kvd, kvd};
+    FS_CUDA(launch_gemv_splitk_multi(m->xn, rows, H, 3, W3, N3, m->qkv, qkvd, st));
+  } else {
+    FS_CUDA(linear(m, m->xn, rows, H, l, kWq, qd, m->qkv, qkvd, false, st));
+    FS_CUDA(linear(m, m->xn, rows, H, l, kWk, kvd, m->qkv + qd, qkvd, false, st));
+    FS_CUDA(linear(m, m->xn, rows, H, l, kWv, kvd, m->qkv + qd + kvd, qkvd, false, st));
+  }
   FS_CUDA(launch_qk_norm_rope_append(m->qkv, rows, map, s, Lw.q_norm, Lw.k_norm, m->rope, m->q,
                                      kvv, l, st));
   if (attention_decode_supported(s, rows)) {
@@ -402,6 +412,13 @@ fs_status layer_general(fs_model* m, const fs_kv* kv, const RowMap& map, int row
   if (rows <= 16 && !(rows > 4 && gemv_splitk_ok(rows, H, Lw.s[kWg]))) {
     FS_CUDA(launch_gemv_swiglu(m->xn, rows, H, Lw.w[kWg], Lw.s[kWg], Lw.w[kWu], Lw.s[kWu], s.I,
                                m->act, st));
+  } else if (rows > 4 && gemv_splitk_ok(rows, H, Lw.s[kWg])) {
+    // gate | up in one launch
+    const __nv_bfloat16* W2[2] = {static_cast<const __nv_bfloat16*>(Lw.w[kWg]),
+                                  static_cast<const __nv_bfloat16*>(Lw.w[kWu])};
+    const int N2[2] = {s.I, s.I};
+    FS_CUDA(launch_gemv_splitk_multi(m->xn, rows, H, 2, W2, N2, m->gu, 2 * s.I, st));
+    FS_CUDA(launch_swiglu(m->gu, rows, s.I, m->act, st));
   } else {
     FS_CUDA(linear(m, m->xn, rows, H, l, kWg, s.I, m->gu, 2 * s.I, false, st));
     FS_CUDA(linear(m, m->xn, rows, H, l, kWu, s.I, m->gu + s.I, 2 * s.I, false, st));
