@@ -95,7 +95,8 @@ struct Shape {
 cudaError_t launch_embed(const int32_t* tokens, int rows, const __nv_bfloat16* E, int H, int V,
                          float* h, int* err, cudaStream_t st);
 cudaError_t launch_rmsnorm(const float* x, int rows, int H, const __nv_bfloat16* g, float eps,
-                           float* out, cudaStream_t st);
+                           float* out, cudaStream_t st, float* zero = nullptr, int zero_w = 0,
+                           int zero_ld = 0);
 // y = x . W^T over rows; epilogue: 0 store y, 1 y += into out (residual).
 cudaError_t launch_gemv(const float* x, int rows, int K, const void* W, const __half* scales,
                         int N, float* out, int ldo, bool accumulate, cudaStream_t st);
@@ -111,7 +112,11 @@ cudaError_t launch_gemv_splitk(const float* x, int rows, int K, const __nv_bfloa
 // side from out0 (cleared first): q | k | v, gate | up.
 cudaError_t launch_gemv_splitk_multi(const float* x, int rows, int K, int n,
                                      const __nv_bfloat16* const* W, const int* N, float* out0,
-                                     int ldo, cudaStream_t st);
+                                     int ldo, bool cleared, cudaStream_t st);
+// y += silu(gate) * up times W^T, the SwiGLU computed while the input is
+// staged: `gu` rows are [gate (K) | up (K)].
+cudaError_t launch_gemv_splitk_swiglu(const float* gu, int rows, int K, const __nv_bfloat16* W,
+                                      int N, float* out, int ldo, cudaStream_t st);
 // Greedy id per row of fp32 logits [rows][V] (lowest id on exact ties).
 cudaError_t launch_argmax_rows(const float* logits, int rows, int V, int32_t* argmax,
                                cudaStream_t st);

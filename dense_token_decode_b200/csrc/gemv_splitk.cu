@@ -45,9 +45,11 @@ struct Segs {
   int n;
 };
 
+// With `swiglu`, x rows are [gate (K) | up (K)] and the staged input is
+// silu(gate) * up (the same expression as swiglu_kernel).
 __global__ void __launch_bounds__(kWarps * 32) gemv_mma_kernel(
     const float* __restrict__ x, int rows, int K, const Segs sg, int ldo, int ctas_per_slice,
-    int tpw) {
+    int tpw, int swiglu) {
   // [term][16 rows][kXStride] bf16
   __shared__ __align__(16) __nv_bfloat16 xs[2][16][kXStride];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -73,7 +75,15 @@ __global__ void __launch_bounds__(kWarps * 32) gemv_mma_kernel(
   if (task < n_tasks) load_w(task);
   for (int e = tid; e < 16 * kSlice; e += kWarps * 32) {
     const int r = e / kSlice, c = e % kSlice;
-    const float v = r < rows ? x[(size_t)r * K + k0 + c] : 0.f;
+    float v = 0.f;
+    if (r < rows) {
+      if (swiglu) {
+        const float gt = x[(size_t)r * 2 * K + k0 + c], up = x[(size_t)r * 2 * K + K + k0 + c];
+        v = gt / (1.f + expf(-gt)) * up;
+      } else {
+        v = x[(size_t)r * K + k0 + c];
+      }
+    }
     const __nv_bfloat16 h = __float2bfloat16_rn(v);
     xs[0][r][c] = h;
     xs[1][r][c] = __float2bfloat16_rn(v - __bfloat162float(h));
@@ -165,7 +175,8 @@ bool gemv_splitk_ok(int rows, int K, const __half* scales) {
 
 namespace {
 
-cudaError_t launch_segs(const float* x, int rows, int K, Segs sg, int ldo, cudaStream_t st) {
+cudaError_t launch_segs(const float* x, int rows, int K, Segs sg, int ldo, cudaStream_t st,
+                        int swiglu = 0) {
   const int n_tasks = sg.tasks[sg.n - 1];
   const int slices = K / kSlice;
   // one task per warp unless the grid would exceed ~4 waves of 3 CTAs per SM
@@ -174,7 +185,8 @@ cudaError_t launch_segs(const float* x, int rows, int K, Segs sg, int ldo, cudaS
   const int ctas_per_slice = (n_tasks + kWarps * tpw - 1) / (kWarps * tpw);
   const int blocks = ctas_per_slice * slices;
   count_launches();
-  gemv_mma_kernel<<<blocks, kWarps * 32, 0, st>>>(x, rows, K, sg, ldo, ctas_per_slice, tpw);
+  gemv_mma_kernel<<<blocks, kWarps * 32, 0, st>>>(x, rows, K, sg, ldo, ctas_per_slice, tpw,
+                                                  swiglu);
   return cudaGetLastError();
 }
 
@@ -201,17 +213,19 @@ cudaError_t launch_gemv_splitk(const float* x, int rows, int K, const __nv_bfloa
 
 // Products of one input with n (2 or 3) matrices, written side by side: W[i]
 // (N[i] rows) into columns out0 + sum_{j<i} N[j] of rows ldo floats apart,
-// which are cleared first (one memset, then one launch).
+// which are cleared first unless the caller has (`cleared`).
 cudaError_t launch_gemv_splitk_multi(const float* x, int rows, int K, int n,
                                      const __nv_bfloat16* const* W, const int* N, float* out0,
-                                     int ldo, cudaStream_t st) {
+                                     int ldo, bool cleared, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
   if (n < 1 || n > 3) return cudaErrorInvalidValue;
   int width = 0;
   for (int i = 0; i < n; ++i) width += N[i];
-  cudaError_t e = cudaMemset2DAsync(out0, (size_t)ldo * sizeof(float), 0,
-                                    (size_t)width * sizeof(float), rows, st);
-  if (e != cudaSuccess) return e;
+  if (!cleared) {
+    cudaError_t e = cudaMemset2DAsync(out0, (size_t)ldo * sizeof(float), 0,
+                                      (size_t)width * sizeof(float), rows, st);
+    if (e != cudaSuccess) return e;
+  }
   Segs sg{};
   int col = 0, tasks = 0;
   for (int i = 0; i < n; ++i) {
@@ -225,6 +239,19 @@ cudaError_t launch_gemv_splitk_multi(const float* x, int rows, int K, int n,
   for (int i = n; i < 3; ++i) sg.tasks[i] = tasks;
   sg.n = n;
   return launch_segs(x, rows, K, sg, ldo, st);
+}
+
+// y += silu(gate) * up times W^T over `rows` rows (accumulating into out).
+cudaError_t launch_gemv_splitk_swiglu(const float* gu, int rows, int K, const __nv_bfloat16* W,
+                                      int N, float* out, int ldo, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  Segs sg{};
+  sg.W[0] = W;
+  sg.out[0] = out;
+  sg.N[0] = N;
+  sg.tasks[0] = (N + kRowsPerWarp - 1) / kRowsPerWarp;
+  sg.n = 1;
+  return launch_segs(gu, rows, K, sg, ldo, st, 1);
 }
 
 }  // namespace fs

@@ -55,11 +55,17 @@ cudaError_t launch_embed(const int32_t* tokens, int rows, const __nv_bfloat16* E
 }
 
 // ---------------------------------------------------------------------------
-// RMSNorm of each row: out = x / sqrt(mean(x^2) + eps) * g, fp32.
+// RMSNorm of each row: out = x / sqrt(mean(x^2) + eps) * g, fp32. With
+// `zero`, row r also clears zero_w floats at zero + r * zero_ld (the output
+// block of the accumulating product that reads `out` next).
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ x, int H,
                                                       const __nv_bfloat16* __restrict__ g,
-                                                      float eps, float* __restrict__ out) {
+                                                      float eps, float* __restrict__ out,
+                                                      float* __restrict__ zero, int zero_w,
+                                                      int zero_ld) {
   __shared__ float red[8];
+  if (zero)
+    for (int c = threadIdx.x; c < zero_w; c += 256) zero[(size_t)blockIdx.x * zero_ld + c] = 0.f;
   const float4* xr = reinterpret_cast<const float4*>(x + (size_t)blockIdx.x * H);
   float ss = 0.f;
   for (int c = threadIdx.x; c < H / 4; c += 256) {
@@ -79,10 +85,10 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ 
 }
 
 cudaError_t launch_rmsnorm(const float* x, int rows, int H, const __nv_bfloat16* g, float eps,
-                           float* out, cudaStream_t st) {
+                           float* out, cudaStream_t st, float* zero, int zero_w, int zero_ld) {
   if (rows <= 0) return cudaSuccess;
   count_launches();
-  rmsnorm_kernel<<<rows, 256, 0, st>>>(x, H, g, eps, out);
+  rmsnorm_kernel<<<rows, 256, 0, st>>>(x, H, g, eps, out, zero, zero_w, zero_ld);
   return cudaGetLastError();
 }
 

@@ -383,15 +383,18 @@ fs_status layer_general(fs_model* m, const fs_kv* kv, const RowMap& map, int row
   const KVView kvv = kv_view(kv);
   const int H = s.H, qd = s.q_dim(), kvd = s.kv_dim(), qkvd = s.qkv_dim();
   const LayerDev& Lw = m->layers[l];
-  FS_CUDA(launch_rmsnorm(m->h, rows, H, Lw.attn_norm, s.eps, m->xn, st));
   const bool splitk = rows > 4 && gemv_splitk_ok(rows, H, Lw.s[kWq]);
+  // the split-K products accumulate: their output blocks are cleared by the
+  // RMSNorm kernel before them
+  FS_CUDA(launch_rmsnorm(m->h, rows, H, Lw.attn_norm, s.eps, m->xn, st, splitk ? m->qkv : nullptr,
+                         qkvd, qkvd));
   if (splitk) {
     // q | k | v in one launch
     const __nv_bfloat16* W3[3] = {static_cast<const __nv_bfloat16*>(Lw.w[kWq]),
                                   static_cast<const __nv_bfloat16*>(Lw.w[kWk]),
                                   static_cast<const __nv_bfloat16*>(Lw.w[kWv])};
     const int N3[3] = {qd, kvd, kvd};
-    FS_CUDA(launch_gemv_splitk_multi(m->xn, rows, H, 3, W3, N3, m->qkv, qkvd, st));
+    FS_CUDA(launch_gemv_splitk_multi(m->xn, rows, H, 3, W3, N3, m->qkv, qkvd, true, st));
   } else {
     FS_CUDA(linear(m, m->xn, rows, H, l, kWq, qd, m->qkv, qkvd, false, st));
     FS_CUDA(linear(m, m->xn, rows, H, l, kWk, kvd, m->qkv + qd, qkvd, false, st));
@@ -408,17 +411,25 @@ fs_status layer_general(fs_model* m, const fs_kv* kv, const RowMap& map, int row
     FS_CUDA(launch_attention_simple(m->q, rows, map, s, kvv, l, m->o, st));
   }
   FS_CUDA(linear(m, m->o, rows, qd, l, kWo, H, m->h, H, true, st));
-  FS_CUDA(launch_rmsnorm(m->h, rows, H, Lw.ffn_norm, s.eps, m->xn, st));
-  if (rows <= 16 && !(rows > 4 && gemv_splitk_ok(rows, H, Lw.s[kWg]))) {
-    FS_CUDA(launch_gemv_swiglu(m->xn, rows, H, Lw.w[kWg], Lw.s[kWg], Lw.w[kWu], Lw.s[kWu], s.I,
-                               m->act, st));
-  } else if (rows > 4 && gemv_splitk_ok(rows, H, Lw.s[kWg])) {
-    // gate | up in one launch
+  const bool splitk_mlp = rows > 4 && gemv_splitk_ok(rows, H, Lw.s[kWg]) &&
+                         gemv_splitk_ok(rows, s.I, Lw.s[kWd]);
+  FS_CUDA(launch_rmsnorm(m->h, rows, H, Lw.ffn_norm, s.eps, m->xn, st,
+                         splitk_mlp ? m->gu : nullptr, 2 * s.I, 2 * s.I));
+  if (splitk_mlp) {
+    // gate | up in one launch, then down with the SwiGLU computed as its input
+    // is staged
     const __nv_bfloat16* W2[2] = {static_cast<const __nv_bfloat16*>(Lw.w[kWg]),
                                   static_cast<const __nv_bfloat16*>(Lw.w[kWu])};
     const int N2[2] = {s.I, s.I};
-    FS_CUDA(launch_gemv_splitk_multi(m->xn, rows, H, 2, W2, N2, m->gu, 2 * s.I, st));
-    FS_CUDA(launch_swiglu(m->gu, rows, s.I, m->act, st));
+    FS_CUDA(launch_gemv_splitk_multi(m->xn, rows, H, 2, W2, N2, m->gu, 2 * s.I, true, st));
+    FS_CUDA(launch_gemv_splitk_swiglu(m->gu, rows, s.I,
+                                      static_cast<const __nv_bfloat16*>(Lw.w[kWd]), H, m->h, H,
+                                      st));
+    return FS_OK;
+  }
+  if (rows <= 16 && !(rows > 4 && gemv_splitk_ok(rows, H, Lw.s[kWg]))) {
+    FS_CUDA(launch_gemv_swiglu(m->xn, rows, H, Lw.w[kWg], Lw.s[kWg], Lw.w[kWu], Lw.s[kWu], s.I,
+                               m->act, st));
   } else {
     FS_CUDA(linear(m, m->xn, rows, H, l, kWg, s.I, m->gu, 2 * s.I, false, st));
     FS_CUDA(linear(m, m->xn, rows, H, l, kWu, s.I, m->gu + s.I, 2 * s.I, false, st));
