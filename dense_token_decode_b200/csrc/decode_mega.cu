@@ -5,20 +5,25 @@
 // rows of every weight matrix. A producer warp streams the CTA's slices —
 // QKV rows, the old K/V pages of the CTA's attention items, O rows, gate/up
 // row pairs, down rows, per layer, then its rows of the tied embedding for
-// the LM head — through a ring of shared-memory stages with cp.async.bulk.
-// Weights do not depend on activations, so the producer runs ahead across
-// phase and layer boundaries and HBM never waits for the dependency chain.
+// the LM head — through a ring of shared-memory stages, weights with
+// cp.async.bulk and K/V with TMA tensor copies (128-byte swizzle, for the
+// tensor cores). Weights do not depend on activations, so the producer runs
+// ahead across phase and layer boundaries and HBM never waits for the
+// dependency chain.
 //
-// Eleven consumer warps compute: weight chunk i belongs to warp i mod 11;
-// KV chunks are shared by all of them. Activations move between CTAs as 64-bit
+// Eleven consumer warps compute: chunk i of the stream (weights or K/V)
+// belongs to warp i mod 11, which alone computes it and releases its stage.
+// Activations move between CTAs as 64-bit
 // words (fp32 value | 32-bit tag): a consumer polls the words it needs until
 // their tag is the one of the current phase, so there is no grid barrier and
 // no separate flag. Tags grow monotonically across steps; nothing is reset.
 //
 // Phases of block l (tag t_l,p): P1 RMSNorm + QKV rows -> xq; P2 attention
 // items (b, kv head g, split s): q/k head RMSNorm + RoPE, append of the new
-// K/V to the page, online-softmax attention over the split's keys, merge of
-// splits by the last arriving item -> xo; P3 O rows + residual -> xh0;
+// K/V to the page, online-softmax attention over the split's keys on the
+// tensor cores (one owner warp per 32-key chunk, mma.sync), merge of the
+// warps' states, merge of splits by the last arriving item -> xo;
+// P3 O rows + residual -> xh0;
 // P4 RMSNorm + gate/up pairs + SwiGLU -> xa; P5 down rows + residual -> xh1.
 // LM head: final RMSNorm, logits of the CTA's vocab rows, greedy key (value,
 // lowest id) folded with a 64-bit atomicMax; the last CTA writes the ids.
