@@ -77,6 +77,8 @@ __device__ __forceinline__ float reduce_transpose(float (&v)[NV], int lane) {
 
 template <int D, int G>
 __global__ void __launch_bounds__(kWarps * 32) attention_decode_kernel(const DecParams p) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int E = D / 32;              // dims per lane
   constexpr int NV = kGroupKeys * G;     // partial scores per lane per group
   constexpr int LOG_NV = NV == 8 ? 3 : NV == 16 ? 4 : 5;
@@ -211,6 +213,8 @@ __global__ void __launch_bounds__(kWarps * 32) attention_decode_kernel(const Dec
 // o[r, h, :] = sum_s w_s o_s / sum_s w_s l_s, w_s = 2^(m_s - max m).
 template <int D>
 __global__ void __launch_bounds__(D) attention_merge_kernel(const DecParams p) {
+  pdl_trigger();
+  pdl_wait();
   const int h = blockIdx.x, r = blockIdx.y, c = threadIdx.x;
   const float* src = p.part + ((size_t)r * p.nq + h) * p.splits * (D + 2);
   float M = -INFINITY;
@@ -230,9 +234,9 @@ template <int D, int G>
 cudaError_t launch_dec(const DecParams& p, int rows, cudaStream_t st) {
   dim3 grid(p.splits, p.nkv, rows);
   count_launches(2);
-  attention_decode_kernel<D, G><<<grid, kWarps * 32, 0, st>>>(p);
-  attention_merge_kernel<D><<<dim3(p.nq, rows), D, 0, st>>>(p);
-  return cudaGetLastError();
+  cudaError_t e = launch_pdl(attention_decode_kernel<D, G>, grid, dim3(kWarps * 32), 0, st, p);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(attention_merge_kernel<D>, dim3(p.nq, rows), dim3(D), 0, st, p);
 }
 
 }  // namespace

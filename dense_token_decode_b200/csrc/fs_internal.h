@@ -16,6 +16,35 @@ namespace fs {
 // Kernel launches issued by the library (fs_debug_kernel_launches).
 void count_launches(int n = 1);
 
+// Programmatic dependent launch. A kernel started with launch_pdl may begin
+// while the kernel before it on the stream is still running: before reading
+// anything an earlier kernel wrote (or writing what it reads) it calls
+// pdl_wait(), which returns once the earlier grids have completed and their
+// memory is visible; only immutable inputs (weights) may be read before it.
+// pdl_trigger() lets the next kernel start early. Both are no-ops for a
+// kernel launched without the attribute.
+#ifdef __CUDACC__
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+#endif
+
 constexpr int kPage = 64;        // positions per KV page
 constexpr int kMaxBatch = 64;    // rows of one decode step
 constexpr int kMaxHeadDim = 128;

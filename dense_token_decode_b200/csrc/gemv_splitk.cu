@@ -73,6 +73,9 @@ __global__ void __launch_bounds__(kWarps * 32) gemv_mma_kernel(
   };
   int task = cs * tpw * kWarps + warp;
   if (task < n_tasks) load_w(task);
+  // everything below reads or writes what earlier kernels wrote or read
+  pdl_trigger();
+  pdl_wait();
   for (int e = tid; e < 16 * kSlice; e += kWarps * 32) {
     const int r = e / kSlice, c = e % kSlice;
     float v = 0.f;
@@ -185,9 +188,8 @@ cudaError_t launch_segs(const float* x, int rows, int K, Segs sg, int ldo, cudaS
   const int ctas_per_slice = (n_tasks + kWarps * tpw - 1) / (kWarps * tpw);
   const int blocks = ctas_per_slice * slices;
   count_launches();
-  gemv_mma_kernel<<<blocks, kWarps * 32, 0, st>>>(x, rows, K, sg, ldo, ctas_per_slice, tpw,
-                                                  swiglu);
-  return cudaGetLastError();
+  return launch_pdl(gemv_mma_kernel, dim3(blocks), dim3(kWarps * 32), 0, st, x, rows, K, sg, ldo,
+                    ctas_per_slice, tpw, swiglu);
 }
 
 }  // namespace

@@ -64,6 +64,8 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ 
                                                       float* __restrict__ zero, int zero_w,
                                                       int zero_ld) {
   __shared__ float red[8];
+  pdl_trigger();
+  pdl_wait();
   if (zero)
     for (int c = threadIdx.x; c < zero_w; c += 256) zero[(size_t)blockIdx.x * zero_ld + c] = 0.f;
   const float4* xr = reinterpret_cast<const float4*>(x + (size_t)blockIdx.x * H);
@@ -88,8 +90,8 @@ cudaError_t launch_rmsnorm(const float* x, int rows, int H, const __nv_bfloat16*
                            float* out, cudaStream_t st, float* zero, int zero_w, int zero_ld) {
   if (rows <= 0) return cudaSuccess;
   count_launches();
-  rmsnorm_kernel<<<rows, 256, 0, st>>>(x, H, g, eps, out, zero, zero_w, zero_ld);
-  return cudaGetLastError();
+  return launch_pdl(rmsnorm_kernel, dim3(rows), dim3(256), 0, st, x, H, g, eps, out, zero, zero_w,
+                    zero_ld);
 }
 
 // ---------------------------------------------------------------------------
@@ -130,6 +132,8 @@ __global__ void qk_norm_rope_append_kernel(const float* __restrict__ qkv, const 
                                            const __nv_bfloat16* __restrict__ k_norm,
                                            const float2* __restrict__ rope,
                                            float* __restrict__ q_out, KVView kv, int layer) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int d = 64 * E, half = 32 * E;
   const int r = blockIdx.x, w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qkv_dim = (nq + 2 * nkv) * d;
@@ -189,14 +193,10 @@ cudaError_t launch_qk_norm_rope_append(const float* qkv, int rows, const RowMap&
   if (s.d != 128 && s.d != 64) return cudaErrorInvalidValue;
   count_launches();
   if (s.d == 128)
-    qk_norm_rope_append_kernel<2><<<rows, threads, 0, st>>>(qkv, map, s.nq, s.nkv, s.eps,
-                                                            q_norm, k_norm, rope, q_out, kv,
-                                                            layer);
-  else
-    qk_norm_rope_append_kernel<1><<<rows, threads, 0, st>>>(qkv, map, s.nq, s.nkv, s.eps,
-                                                            q_norm, k_norm, rope, q_out, kv,
-                                                            layer);
-  return cudaGetLastError();
+    return launch_pdl(qk_norm_rope_append_kernel<2>, dim3(rows), dim3(threads), 0, st, qkv, map,
+                      s.nq, s.nkv, s.eps, q_norm, k_norm, rope, q_out, kv, layer);
+  return launch_pdl(qk_norm_rope_append_kernel<1>, dim3(rows), dim3(threads), 0, st, qkv, map, s.nq,
+                    s.nkv, s.eps, q_norm, k_norm, rope, q_out, kv, layer);
 }
 
 // ---------------------------------------------------------------------------
