@@ -102,6 +102,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attention_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap map_k,
                         const __grid_constant__ CUtensorMap map_v) {
+  pdl_trigger();
+  pdl_wait();  // launched early by dependent launch: nothing before this point
   using Lay = Layout<D>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -455,8 +457,7 @@ cudaError_t launch(const Params& p, const CUtensorMap& mk, const CUtensorMap& mv
   const size_t smem = Lay::kSmemBytes;
   const Params& q = p;
   count_launches();
-  attention_tc_kernel<D><<<grid, kThreads, smem, st>>>(q, mk, mv);
-  return cudaGetLastError();
+  return launch_pdl(attention_tc_kernel<D>, dim3(grid), dim3(kThreads), smem, st, q, mk, mv);
 }
 
 }  // namespace attn_tc

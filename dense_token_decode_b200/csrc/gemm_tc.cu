@@ -153,6 +153,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap map_a_lo,
                    const __grid_constant__ CUtensorMap map_b,
                    const __grid_constant__ CUtensorMap map_b2) {
+  pdl_trigger();
+  pdl_wait();  // launched early by dependent launch: nothing before this point
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // 1024-byte aligned base for the swizzled tiles
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -448,9 +450,8 @@ cudaError_t launch_bn(const CUtensorMap* a, const CUtensorMap* a_lo, const CUten
   const int units = p.n_tiles_m * p.n_tiles_n * p.ksplit;
   const int grid = std::min(units, num_sms);
   count_launches();
-  tc::gemm_tc_kernel<BN><<<grid, tc::kThreads, smem, st>>>(p, *a, a_lo ? *a_lo : *a, *b,
-                                                           b2 ? *b2 : *b);
-  return cudaGetLastError();
+  return launch_pdl(tc::gemm_tc_kernel<BN>, dim3(grid), dim3(tc::kThreads), smem, st, p, *a,
+                    a_lo ? *a_lo : *a, *b, b2 ? *b2 : *b);
 }
 }  // namespace
 

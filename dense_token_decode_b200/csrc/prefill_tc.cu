@@ -52,6 +52,8 @@ __global__ void __launch_bounds__(256) rmsnorm_f16_kernel(const float* __restric
                                                           const __nv_bfloat16* __restrict__ g,
                                                           float eps, __half* __restrict__ hi,
                                                           __half* __restrict__ lo) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red[8];
   const float* xr = x + (size_t)blockIdx.x * H;
   float ss = 0.f;
@@ -227,9 +229,9 @@ fs_status layer_tc(fs_model* m, const fs_kv* kv, const RowMap& map, int rows, in
     }                                                                 \
   } while (0)
   count_launches();
-  rmsnorm_f16_kernel<<<rows, 256, 0, st>>>(m->h, s.H, Lw.attn_norm, s.eps, t->xn_hi,
-                                           split ? t->xn_lo : nullptr);
-  FS_TRY(cudaGetLastError());
+  FS_TRY(launch_pdl(rmsnorm_f16_kernel, dim3(rows), dim3(256), 0, st, (const float*)m->h, s.H,
+                    (const __nv_bfloat16*)Lw.attn_norm, s.eps, t->xn_hi,
+                    split ? t->xn_lo : (__half*)nullptr));
   if (map.n_list == 0 && bn_qkv(s) % s.d == 0 && s.d % 64 == 0) {
     // the per-head RMSNorm, RoPE and the K/V append run in the GEMM epilogue
     FS_TRY(launch_gemm_tc_qkv_heads(&t->a_xn_hi, split ? &t->a_xn_lo : nullptr, &mp.qkv, rows,
@@ -255,8 +257,8 @@ fs_status layer_tc(fs_model* m, const fs_kv* kv, const RowMap& map, int rows, in
   FS_TRY(launch_gemm_tc(&t->a_o, nullptr, &mp.o, nullptr, rows, s.H, s.q_dim(), 1, m->h, s.H,
                         nullptr, nullptr, 0, m->err, m->num_sms, st, 128));
   count_launches();
-  rmsnorm_f16_kernel<<<rows, 256, 0, st>>>(m->h, s.H, Lw.ffn_norm, s.eps, t->xn_hi, nullptr);
-  FS_TRY(cudaGetLastError());
+  FS_TRY(launch_pdl(rmsnorm_f16_kernel, dim3(rows), dim3(256), 0, st, (const float*)m->h, s.H,
+                    (const __nv_bfloat16*)Lw.ffn_norm, s.eps, t->xn_hi, (__half*)nullptr));
   FS_TRY(launch_gemm_tc(&t->a_xn_hi, nullptr, &mp.g, &mp.u, rows, 2 * s.I, s.H, 2, nullptr, 0,
                         t->act_hi, nullptr, s.I, m->err, m->num_sms, st, bn_gu(s)));
   FS_TRY(launch_gemm_tc(&t->a_act, nullptr, &mp.d, nullptr, rows, s.H, s.I, 1, m->h, s.H, nullptr,
