@@ -21,7 +21,12 @@ Three consumer protocols are modelled:
   pending release as chunk i - n's, so it only narrows the window;
 * ``all_warps``: every warp waits on every chunk in order (a K/V page pair
   two at a time) and arrives on its release barrier, whose arrival count is
-  the number of warps (the current kernel).
+  the number of warps (the cooperative kernel's chunks);
+* ``owner_all``: every chunk, weight rows and K/V alike, is consumed and
+  released by warp i % 11 alone, which first tests that chunk i - n was
+  released, then chunk i's full barrier; CTA barriers around each attention
+  item (the row-split kernel, which refuses rings of fewer stages than
+  consumer warps: a warp's owned chunks are then at most a ring apart).
 
 A violation is a warp reading a stage that does not hold its chunk yet
 (stale bytes, or a copy into it still in flight); a deadlock is a state in
@@ -97,6 +102,17 @@ def warp_programs(plan, protocol):
                     else:
                         progs[w].append(("skip", i + c))
             i += count
+        elif protocol == "owner_all":  # K/V chunks: one owner warp each
+            for c in range(count):
+                for w in range(WARPS):
+                    if (i + c) % WARPS == w:
+                        progs[w] += [("wait", i + c), ("release", i + c)]
+                    else:
+                        progs[w].append(("skip", i + c))
+            for w in range(WARPS):
+                progs[w].append(("bar", nbar))
+            nbar += 1
+            i += count
         else:  # K/V pairs: every warp reads both chunks of a pair
             for c in range(0, count, 2):
                 for w in range(WARPS):
@@ -149,7 +165,7 @@ def simulate(n_stages, batch, protocol, seed):
         par = (x // n_stages) & 1
         if op == "wait":
             ready = full[s].try_wait(par)
-            if protocol == "owner_fixed":
+            if protocol in ("owner_fixed", "owner_all"):
                 ready = ready and empty[s].try_wait(par ^ 1)
             if not ready:
                 return False
@@ -239,3 +255,18 @@ def test_waiting_for_the_previous_release_is_not_enough(n_stages):
 @pytest.mark.parametrize("n_stages", list(range(2, 17)))
 def test_all_warps_protocol_never_misreads_or_deadlocks(n_stages, batch):
     assert outcomes(n_stages, batch, "all_warps", 6) == {"ok"}
+
+
+@pytest.mark.parametrize("batch", [1, 2, 3, 4])
+@pytest.mark.parametrize("n_stages", list(range(11, 17)))
+def test_row_split_owner_protocol_never_misreads_or_deadlocks(n_stages, batch):
+    """The row-split kernel's protocol at the ring sizes it accepts."""
+    assert outcomes(n_stages, batch, "owner_all", 6) == {"ok"}
+
+
+@pytest.mark.parametrize("n_stages", [4, 8])
+def test_row_split_owner_protocol_needs_a_stage_per_warp(n_stages):
+    """Why the row-split kernel refuses smaller rings: with fewer stages than
+    consumer warps a warp can be two rings ahead of a pending chunk, and the
+    release test then reads the wrong phase."""
+    assert "violation" in outcomes(n_stages, 2, "owner_all", 60)
