@@ -76,3 +76,50 @@ def test_outputs_land_where_the_kernel_stores_them():
         for e in range(4):
             seen.add((g + (e >> 1) * 8, 2 * t + (e & 1)))
     assert seen == {(r, n) for r in range(16) for n in range(8)}
+
+
+def bf16(v):
+    """Round to bf16 (nearest even), as float64."""
+    a = np.asarray(v, dtype=np.float32).copy()
+    u = a.view(np.uint32)
+    u += 0x7FFF + ((u >> 16) & 1)
+    u &= 0xFFFF0000
+    return a.astype(np.float64)
+
+
+def test_attention_p_fragments_come_from_the_right_lanes():
+    """Row-split decode attention, one 16-key half: after S = K q^T, lane
+    (g, t) holds p(key g) and p(key g + 8) of head t (t < 2). The P V MMA's B
+    column g is head g / 2, term g % 2 (bf16 hi, then the remainder); the
+    kernel reads key 2t and 2t + 1 (b0 b1) and 2t + 8, 2t + 9 (b2 b3) from
+    lanes (2t) * 4 + g / 2 and (2t + 1) * 4 + g / 2. With A = V^T, columns
+    2h and 2h + 1 of D then add up to head h's P V."""
+    rng = np.random.default_rng(3)
+    p = rng.random((16, 2))           # p[key][head]
+    V = rng.standard_normal((16, 16)) # V[key][dim]
+    # lane registers after the softmax: pr0 = p(key g, head t), pr1 = p(key g + 8, head t)
+    pr0 = np.zeros(32)
+    pr1 = np.zeros(32)
+    for lane in range(32):
+        g, t = lane >> 2, lane & 3
+        if t < 2:
+            pr0[lane], pr1[lane] = p[g, t], p[g + 8, t]
+    B = np.zeros((16, 8))
+    for lane in range(32):
+        g, t = lane >> 2, lane & 3
+        hn, lo = g >> 1, g & 1
+        if g >= 4:  # columns past the two heads' terms are zero
+            continue
+        q00, q01 = pr0[(2 * t) * 4 + hn], pr0[(2 * t + 1) * 4 + hn]
+        q10, q11 = pr1[(2 * t) * 4 + hn], pr1[(2 * t + 1) * 4 + hn]
+
+        def term(v):
+            h = bf16(v)
+            return bf16(v - h) if lo else h
+
+        B[2 * t, g], B[2 * t + 1, g] = term(q00), term(q01)
+        B[2 * t + 8, g], B[2 * t + 9, g] = term(q10), term(q11)
+    D = V.T @ B  # A = V^T: rows = dims, columns = keys
+    for h in range(2):
+        np.testing.assert_allclose(D[:, 2 * h] + D[:, 2 * h + 1], V.T @ p[:, h],
+                                   rtol=2e-5, atol=2e-5)
